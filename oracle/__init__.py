@@ -1,0 +1,188 @@
+"""CPU oracle for the FP8_DYNAMIC quantized Linear.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  The product
+path (the CUDA library and its Python binding) never imports it, and this
+package never imports the product.
+
+The arithmetic lives in ``mfp8_oracle.c`` (plain C, fp64/int64, OpenMP); this
+module only marshals numpy arrays into it.  What each function follows:
+
+* ``e4m3_encode`` / ``e4m3_decode`` - the float8_e4m3fn format named by the
+  "MOSS-VL quantization README", FP8-Dynamic recipe section, and described as
+  "4 exponent bits, 3 mantissa bits" in the "MOSS-VL-Realtime-FP8
+  mixed-precision strategy" article, section "252 个主力 Linear 层为什么用
+  FP8 E4M3".  Rounding (nearest-even) and saturation to 448 are this
+  project's reading; the pages state neither.
+* ``quantize_rows`` - one scale per row: per output channel for weights
+  ("channel-wise static"), per token for activations ("per-token dynamic"),
+  same README section.  Scale = fl32(absmax / 448), floored at FLT_MIN
+  (reading; the pages give no formula).
+* ``linear_ref`` - exact fp64 contraction of the decoded codes, rescaled by
+  s_a[m] * s_w[n]; ``dot_int64`` is the same contraction in integers.
+* ``within_tolerance`` - the acceptance rule for BF16 outputs:
+  |y - y_ref| <= 2^-7 |y_ref| + 1e-5 * s_abs.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+
+class Oracle:
+    """ctypes view of one build of ``mfp8_oracle.c`` (the default build, or a
+    copy compiled by a test that plants a mistake in it)."""
+
+    def __init__(self, path: str):
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.orc_bf16_to_f32.restype = ctypes.c_float
+        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_e4m3_encode_array.argtypes = [P, i64, P]
+        L.orc_e4m3_decode_array.argtypes = [P, i64, P]
+        L.orc_e4m3_encode_bits_range.argtypes = [ctypes.c_uint64, ctypes.c_uint64, P]
+        L.orc_row_scale.restype = ctypes.c_float
+        L.orc_row_scale.argtypes = [P, i64]
+        L.orc_quantize_rows.argtypes = [P, i64, i64, P, P]
+        L.orc_linear_ref.argtypes = [P, P, i64, P, P, i64, i64, P, P]
+        L.orc_dot_int64.argtypes = [P, i64, P, i64, i64, P]
+        L.orc_num_threads.restype = ctypes.c_int
+        self.L = L
+        self.path = path
+
+    def num_threads(self) -> int:
+        return int(self.L.orc_num_threads())
+
+    def e4m3_decode(self, codes):
+        codes = _c(codes, np.uint8)
+        out = np.empty(codes.shape, dtype=np.float64)
+        self.L.orc_e4m3_decode_array(_ptr(codes), codes.size, _ptr(out))
+        return out
+
+    def e4m3_encode(self, values):
+        values = _c(values, np.float32)
+        out = np.empty(values.shape, dtype=np.uint8)
+        self.L.orc_e4m3_encode_array(_ptr(values), values.size, _ptr(out))
+        return out
+
+    def e4m3_encode_bits_range(self, lo: int, hi: int):
+        """Codes of every fp32 bit pattern in [lo, hi)."""
+        out = np.empty(hi - lo, dtype=np.uint8)
+        self.L.orc_e4m3_encode_bits_range(ctypes.c_uint64(lo), ctypes.c_uint64(hi), _ptr(out))
+        return out
+
+    def row_scale(self, row_bits) -> np.float32:
+        row_bits = _c(row_bits, np.uint16)
+        return np.float32(self.L.orc_row_scale(_ptr(row_bits), row_bits.size))
+
+    def quantize_rows(self, x_bits):
+        """x_bits: uint16 [R, K] holding bf16 bit patterns.
+        Returns (codes uint8 [R, K], scales float32 [R])."""
+        x_bits = _c(x_bits, np.uint16)
+        R, K = x_bits.shape
+        q = np.empty((R, K), dtype=np.uint8)
+        s = np.empty((R,), dtype=np.float32)
+        self.L.orc_quantize_rows(_ptr(x_bits), R, K, _ptr(q), _ptr(s))
+        return q, s
+
+    def linear_ref(self, x8, s_a, w8, s_w, want_abs: bool = True):
+        """Exact reference of the rescaled FP8 contraction.
+        x8 uint8 [M,K], s_a f32 [M], w8 uint8 [N,K], s_w f32 [N].
+        Returns (y_ref f64 [M,N], s_abs f64 [M,N] or None)."""
+        x8 = _c(x8, np.uint8)
+        w8 = _c(w8, np.uint8)
+        s_a = _c(s_a, np.float32)
+        s_w = _c(s_w, np.float32)
+        M, K = x8.shape
+        N, K2 = w8.shape
+        assert K == K2 and s_a.shape == (M,) and s_w.shape == (N,)
+        y = np.empty((M, N), dtype=np.float64)
+        sa = np.empty((M, N), dtype=np.float64) if want_abs else None
+        self.L.orc_linear_ref(_ptr(x8), _ptr(s_a), M, _ptr(w8), _ptr(s_w), N, K,
+                              _ptr(y), _ptr(sa) if want_abs else None)
+        return y, sa
+
+    def dot_int64(self, x8, w8):
+        """Integer form of the contraction: sum_k (2^9 dec(x)) * (2^9 dec(w))."""
+        x8 = _c(x8, np.uint8)
+        w8 = _c(w8, np.uint8)
+        M, K = x8.shape
+        N, _ = w8.shape
+        out = np.empty((M, N), dtype=np.int64)
+        self.L.orc_dot_int64(_ptr(x8), M, _ptr(w8), N, K, _ptr(out))
+        return out
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(_build.build())
+    return _default
+
+
+def num_threads() -> int:
+    return default().num_threads()
+
+
+def e4m3_decode(codes):
+    return default().e4m3_decode(codes)
+
+
+def e4m3_encode(values):
+    return default().e4m3_encode(values)
+
+
+def e4m3_encode_bits_range(lo: int, hi: int):
+    return default().e4m3_encode_bits_range(lo, hi)
+
+
+def row_scale(row_bits):
+    return default().row_scale(row_bits)
+
+
+def quantize_rows(x_bits):
+    return default().quantize_rows(x_bits)
+
+
+def linear_ref(x8, s_a, w8, s_w, want_abs: bool = True):
+    return default().linear_ref(x8, s_a, w8, s_w, want_abs)
+
+
+def dot_int64(x8, w8):
+    return default().dot_int64(x8, w8)
+
+
+def bf16_bits_to_f32(bits):
+    bits = _c(bits, np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+TOL_REL = 2.0 ** -7
+TOL_ABS_FRAC = 1e-5
+
+
+def tolerance(y_ref, s_abs):
+    return TOL_REL * np.abs(y_ref) + TOL_ABS_FRAC * s_abs
+
+
+def within_tolerance(y, y_ref, s_abs):
+    """Element mask of |y - y_ref| <= 2^-7 |y_ref| + 1e-5 s_abs."""
+    y = np.asarray(y, dtype=np.float64)
+    return np.abs(y - y_ref) <= tolerance(y_ref, s_abs)

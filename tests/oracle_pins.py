@@ -1,0 +1,236 @@
+"""Checks that pin the CPU oracle to facts outside itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with what the format definition, a library
+implementation of float8_e4m3fn, exact rational arithmetic or a closed form
+fixes.  ``test_oracle_pins.py`` runs them on the oracle; ``test_oracle_mutants.py``
+runs them on copies of the oracle with a planted mistake and expects a failure.
+"""
+import math
+import os
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+FLT_MIN = np.float32(np.finfo(np.float32).tiny)
+
+
+def lib_decode(codes):
+    """float8_e4m3fn decode by ml_dtypes (a library implementation)."""
+    return np.asarray(codes, np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+
+
+def lib_encode(values):
+    """float8_e4m3fn encode by ml_dtypes: round to nearest even; it does not
+    saturate, so only compare for |v| <= 464."""
+    return np.asarray(values, np.float32).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+
+
+def bf16_bits(x_f32):
+    """Round fp32 values to bf16 with torch and return the bit patterns."""
+    t = torch.from_numpy(np.ascontiguousarray(x_f32, np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_f32(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ------------------------------------------------------------------ codec --
+
+def pin_decode_table(o):
+    codes = np.arange(256, dtype=np.uint8)
+    d = o.e4m3_decode(codes)
+    ref = lib_decode(codes)
+    nan = np.isnan(d)
+    assert np.array_equal(nan, np.isnan(ref)), "NaN codes differ from the library"
+    assert set(np.nonzero(nan)[0].tolist()) == {0x7F, 0xFF}, "NaN must be S.1111.111 only"
+    assert np.array_equal(d[~nan], ref[~nan]), "decoded values differ from the library"
+    assert not np.isinf(d).any(), "e4m3fn has no infinities"
+    assert np.nanmax(d) == 448.0 and np.nanmin(d) == -448.0
+    assert d[0x01] == 2.0 ** -9 and d[0x08] == 2.0 ** -6 and d[0x38] == 1.0
+    assert (~nan).sum() == 254
+
+
+def pin_roundtrip(o):
+    codes = np.arange(256, dtype=np.uint8)
+    d = o.e4m3_decode(codes).astype(np.float32)
+    back = o.e4m3_encode(d)
+    finite = ~np.isnan(d)
+    assert np.array_equal(back[finite], codes[finite]), "decode -> encode is not the identity"
+    assert set(back[~finite].tolist()) <= {0x7F, 0xFF}
+
+
+def read_rounding_cases():
+    cases = []
+    with open(os.path.join(GOLDEN, "e4m3_rounding_cases.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            tok = line.split()
+            v, code = tok[0], int(tok[1], 16)
+            if v.lstrip("-").startswith("0x"):
+                val = float.fromhex(v)
+            else:
+                val = float(v)
+            cases.append((np.float32(val), code, line))
+    return cases
+
+
+def pin_rounding_cases(o):
+    cases = read_rounding_cases()
+    vals = np.array([c[0] for c in cases], dtype=np.float32)
+    got = o.e4m3_encode(vals)
+    for (v, code, line), g in zip(cases, got):
+        if np.isnan(v):
+            assert (g & 0x7F) == 0x7F, line
+        else:
+            assert g == code, f"{line}: got 0x{g:02x}"
+
+
+def pin_encode_vs_library(o, n=400_000, seed=11):
+    rng = np.random.default_rng(seed)
+    # magnitudes log-uniform over the whole e4m3 range and below it
+    mag = np.exp2(rng.uniform(-14.0, math.log2(464.0), n)).astype(np.float32)
+    v = np.where(rng.random(n) < 0.5, -mag, mag).astype(np.float32)
+    # every midpoint between adjacent finite codes, and one fp32 ulp either side
+    d = np.unique(lib_decode(np.arange(0, 0x7F, dtype=np.uint8)))
+    mids = ((d[1:] + d[:-1]) / 2).astype(np.float32)
+    near = np.concatenate([mids, np.nextafter(mids, np.float32(np.inf)),
+                           np.nextafter(mids, np.float32(0))])
+    v = np.concatenate([v, near, -near]).astype(np.float32)
+    v = v[np.abs(v) <= 464.0]
+    got = o.e4m3_encode(v)
+    ref = lib_encode(v)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, f"{bad.size} mismatches vs library, first {v[bad[:4]]}"
+    tv = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, tv), "mismatch vs torch float8_e4m3fn"
+
+
+def pin_saturation(o):
+    big = np.array([448.0, 448.5, 463.99, 464.0, 464.01, 500.0, 1e5, 3.0e38, np.inf],
+                   dtype=np.float32)
+    assert (o.e4m3_encode(big) == 0x7E).all()
+    assert (o.e4m3_encode(-big) == 0xFE).all()
+    assert (o.e4m3_encode(np.array([np.nan], np.float32))[0] & 0x7F) == 0x7F
+
+
+# ----------------------------------------------------------------- scales --
+
+def _random_rows(rng, R, K, lo=-20, hi=20):
+    x = rng.standard_normal((R, K)).astype(np.float32)
+    x *= np.exp2(rng.uniform(lo, hi, (R, 1))).astype(np.float32)
+    return bf16_bits(x)
+
+
+def pin_scale_invariants(o, seed=5):
+    rng = np.random.default_rng(seed)
+    R, K = 64, 257
+    xb = _random_rows(rng, R, K)
+    x = bits_to_f32(xb).astype(np.float64)
+    q, s = o.quantize_rows(xb)
+    dq = o.e4m3_decode(q)
+    # every code finite and within +-448
+    assert not np.isnan(dq).any() and np.abs(dq).max() <= 448.0
+    # a row's largest magnitude maps to +-448
+    j = np.argmax(np.abs(x), axis=1)
+    top = q[np.arange(R), j]
+    assert np.all((top == 0x7E) | (top == 0xFE)), "absmax element must encode to +-448"
+    # scale is the absmax over 448, up to one fp32 rounding
+    amax = np.abs(x).max(axis=1)
+    assert np.all(np.abs(s.astype(np.float64) * 448.0 - amax) <= amax * 2.0 ** -23)
+    # reconstruction: half a 3-bit-mantissa step (2^-4 relative) in the
+    # normal range, half the subnormal step (2^-10 * s) below it
+    err = np.abs(dq * s[:, None] - x)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * s[:, None].astype(np.float64))
+    assert np.all(err <= bound * (1 + 2.0 ** -20)), "reconstruction error too large"
+    # a scale depends on its own row only (data-free, no calibration set)
+    perm = rng.permutation(R)
+    q2, s2 = o.quantize_rows(xb[perm])
+    assert np.array_equal(s2, s[perm]) and np.array_equal(q2, q[perm])
+    # all-zero row: floor scale, all codes zero (sign kept)
+    z = np.zeros((2, 32), np.uint16)
+    z[1, :] = 0x8000  # -0.0
+    qz, sz = o.quantize_rows(z)
+    assert np.all(sz == FLT_MIN)
+    assert np.all(qz[0] == 0x00) and np.all(qz[1] == 0x80)
+    # tiny rows (bf16 subnormals) do not divide by zero and still reach 448
+    t = np.zeros((1, 16), np.uint16)
+    t[0, 3] = 0x0001  # smallest positive bf16 subnormal
+    t[0, 5] = 0x8001
+    qt, st = o.quantize_rows(t)
+    assert st[0] == FLT_MIN
+    assert qt[0, 3] != 0 and qt[0, 5] != 0 and np.all(np.delete(qt[0], [3, 5]) == 0)
+
+
+# ------------------------------------------------------------------- GEMM --
+
+def pin_gemm_bruteforce(o, seed=3):
+    """Exact rationals on tiny shapes: the library decodes the codes, Fraction
+    sums them, and the oracle's fp64 result must be that value rounded once."""
+    rng = np.random.default_rng(seed)
+    for (M, N, K) in [(1, 1, 16), (3, 5, 32), (6, 4, 64), (2, 7, 48)]:
+        x8, sa = o.quantize_rows(_random_rows(rng, M, K, -3, 3))
+        w8, sw = o.quantize_rows(_random_rows(rng, N, K, -8, -4))
+        y, sabs = o.linear_ref(x8, sa, w8, sw)
+        xd, wd = lib_decode(x8), lib_decode(w8)
+        for m in range(M):
+            for n in range(N):
+                dot = sum(Fraction(float(xd[m, k])) * Fraction(float(wd[n, k])) for k in range(K))
+                dab = sum(abs(Fraction(float(xd[m, k])) * Fraction(float(wd[n, k]))) for k in range(K))
+                sc = Fraction(float(sa[m])) * Fraction(float(sw[n]))
+                exact, exact_abs = dot * sc, dab * sc
+                assert abs(Fraction(y[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 52), (M, N, K, m, n)
+                assert abs(Fraction(sabs[m, n]) - exact_abs) <= exact_abs * Fraction(1, 2 ** 52)
+
+
+def pin_gemm_int_vs_fp(o, seed=4):
+    """The int64 and fp64 contractions agree exactly (the sum is exact)."""
+    rng = np.random.default_rng(seed)
+    M, N, K = 5, 9, 4096
+    x8, sa = o.quantize_rows(_random_rows(rng, M, K, 0, 1))
+    w8, sw = o.quantize_rows(_random_rows(rng, N, K, -6, -5))
+    ones_a = np.ones(M, np.float32)
+    ones_w = np.ones(N, np.float32)
+    y, _ = o.linear_ref(x8, ones_a, w8, ones_w, want_abs=False)
+    di = o.dot_int64(x8, w8)
+    assert np.array_equal(y * 2.0 ** 18, di.astype(np.float64)), "fp64 sum is not exact"
+    # all-448 worst case, K = 12288: the largest possible sum stays exact
+    K2 = 12288
+    a = np.full((1, K2), 0x7E, np.uint8)
+    y2, _ = o.linear_ref(a, np.ones(1, np.float32), a, np.ones(1, np.float32), want_abs=False)
+    assert y2[0, 0] == 448.0 * 448.0 * K2
+
+
+def pin_onehot_closed_form(o, seed=6):
+    """W rows with a single non-zero entry c_n at column j_n quantize to code
+    +-448 there and 0 elsewhere, so y[m,n] = dec(X8[m,j_n]) * (+-448) * s_a[m] *
+    s_w[n] exactly: checks the rescale and the (m, n) index mapping."""
+    rng = np.random.default_rng(seed)
+    M, N, K = 3, 7, 96
+    x8, sa = o.quantize_rows(_random_rows(rng, M, K, -2, 2))
+    j = rng.integers(0, K, N)
+    c = (rng.standard_normal(N) * 3).astype(np.float32)
+    w = np.zeros((N, K), np.float32)
+    w[np.arange(N), j] = c
+    wb = bf16_bits(w)
+    w8, sw = o.quantize_rows(wb)
+    cb = bits_to_f32(wb[np.arange(N), j])
+    assert np.all(o.e4m3_decode(w8[np.arange(N), j]) == np.sign(cb) * 448.0)
+    y, _ = o.linear_ref(x8, sa, w8, sw)
+    xd = o.e4m3_decode(x8)
+    for m in range(M):
+        for n in range(N):
+            expect = float(Fraction(float(xd[m, j[n]])) * Fraction(float(np.sign(cb[n]) * 448.0))
+                           * Fraction(float(sa[m])) * Fraction(float(sw[n])))
+            assert y[m, n] == expect, (m, n)
+
+
+ALL_PINS = [pin_decode_table, pin_roundtrip, pin_rounding_cases, pin_encode_vs_library,
+            pin_saturation, pin_scale_invariants, pin_gemm_bruteforce, pin_gemm_int_vs_fp,
+            pin_onehot_closed_form]

@@ -1,0 +1,61 @@
+"""Plant a mistake in a copy of the CPU oracle and check that a pin catches it.
+
+Each mutant is a textual edit of ``oracle/mfp8_oracle.c`` compiled into a
+temporary library; the real oracle is untouched.  A mutant that every pin
+accepts would mean the pins cannot see that class of mistake.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import oracle_pins as P
+from oracle import build as obuild
+
+MUTANTS = {
+    # rounding: truncate instead of nearest-even
+    "truncate": ("double steps = nearbyint(ldexp(a, -q));", "double steps = trunc(ldexp(a, -q));"),
+    # rounding: ties away from zero instead of ties to even
+    "ties_away": ("double steps = nearbyint(ldexp(a, -q));", "double steps = round(ldexp(a, -q));"),
+    # exponent bias off by one in the decoder
+    "bias": ("else mag = ldexp(1.0 + m / 8.0, e - 7);", "else mag = ldexp(1.0 + m / 8.0, e - 8);"),
+    # scale constant wrong
+    "scale_240": ("float s = amax / 448.0f;", "float s = amax / 240.0f;"),
+    # multiply instead of divide when quantizing
+    "mul_not_div": ("float q = orc_bf16_to_f32(row[k]) / sr;", "float q = orc_bf16_to_f32(row[k]) * sr;"),
+    # sign of zero dropped
+    "zero_sign": ("if (r == 0.0) return sign;", "if (r == 0.0) return 0;"),
+    # transposed output index
+    "transpose_out": ("if (y_ref) y_ref[m * N + n] = dot * sc;", "if (y_ref) y_ref[n * M + m] = dot * sc;"),
+    # a dropped term in the dot product
+    "dropped_term": ("for (k = 0; k < K; ++k) {\n                    double p", "for (k = 1; k < K; ++k) {\n                    double p"),
+    # the activation scale is not applied
+    "no_sa": ("double sc = (double)s_a[m] * (double)s_w[n];", "double sc = (double)s_w[n];"),
+    # saturation missing (values above 448 become NaN)
+    "no_satfinite": ("if (a >= 448.0) return (uint8_t)(sign | 0x7E);", "if (a >= 464.0) return (uint8_t)(sign | 0x7F);"),
+}
+
+
+@pytest.fixture(scope="module")
+def src():
+    with open(obuild.SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, src, tmp_path):
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    c = tmp_path / f"mut_{name}.c"
+    c.write_text(src.replace(old, new))
+    so = tmp_path / f"libmut_{name}.so"
+    subprocess.run(["gcc", *obuild.CFLAGS, str(c), "-o", str(so), "-lm"], check=True)
+    mut = oracle.Oracle(str(so))
+    caught = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(mut)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches mutant {name}"
