@@ -1,0 +1,466 @@
+"""Benchmark of the FP8_DYNAMIC Linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one decode pass through the seven projections of one language
+layer (q, k, v, o, gate, up, down) at M = 1, 4 and 8 tokens: 21 FP8_DYNAMIC
+Linears, each quantizing its activations per token and running the FP8 GEMM.
+The three M values use three separate weight sets, so a step streams 579 MB
+of e4m3 weights (more than the 126 MB L2) and no step hits L2 for weights.
+
+Headline: weight-read GB/s = (N*K + 4N) bytes summed over the step / step
+time, from CUDA-graph replays with inputs resident in HBM.  The same line
+carries the end-to-end figure through the C ABI with host buffers, the
+roofline of the dominant kernel, the prefill (M = 2048) TFLOPS with its
+tensor roofline, the one-time weight quantization, and the CPU oracle timed
+on a bounded sample as a baseline.
+
+Multi-GPU (torchrun): every rank runs its own independent decode batch
+(data parallel, no collective on the data path); value = all ranks' bytes /
+the slowest rank's time.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DECODE_MS = (1, 4, 8)
+PREFILL_M = 2048
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------- workload --
+
+class Layer:
+    """One layer's seven projections: BF16 activations per M, FP8 weights."""
+
+    def __init__(self, torch, mfp8, W, seed, weight_sets, Ms, device, x_kind):
+        self.lins = W.LAYER_LINEARS
+        self.Ms = Ms
+        self.x = {}
+        self.y = {}
+        self.ws = {}
+        for M in Ms:
+            for i, lin in enumerate(self.lins):
+                self.x[(M, i)] = W.make_x(M, lin.K, seed=seed, stream=M * 16 + i, kind=x_kind, device=device)
+                self.y[(M, i)] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=device)
+                self.ws[(M, i)] = mfp8.workspace_for(M, lin.N, lin.K, device)
+        # weights: one BF16 draw per projection, quantized into `weight_sets` copies
+        self.w8 = [[None] * len(self.lins) for _ in range(weight_sets)]
+        self.sw = [[None] * len(self.lins) for _ in range(weight_sets)]
+        self.wq_time_ms = 0.0
+        self.wq_bytes = 0
+        for i, lin in enumerate(self.lins):
+            for s in range(weight_sets):
+                w = W.make_w(lin.N, lin.K, seed=seed, stream=100 * s + i, device=device)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                self.w8[s][i], self.sw[s][i] = mfp8.quantize_weight(w)
+                e1.record()
+                torch.cuda.synchronize()
+                self.wq_time_ms += e0.elapsed_time(e1)
+                self.wq_bytes += lin.N * lin.K * 3 + lin.N * 4
+                del w
+        self.weight_sets = weight_sets
+
+    def weight_set(self, mi):
+        return mi % self.weight_sets
+
+    def step(self, mfp8, stream):
+        for mi, M in enumerate(self.Ms):
+            s = self.weight_set(mi)
+            for i, lin in enumerate(self.lins):
+                ws = self.ws[(M, i)]
+                st = mfp8.mfp8_linear(self.x[(M, i)].data_ptr(), M, lin.K, self.w8[s][i].data_ptr(),
+                                      self.sw[s][i].data_ptr(), lin.N, self.y[(M, i)].data_ptr(),
+                                      ws.data_ptr(), ws.numel(), stream)
+                if st != mfp8.OK:
+                    raise mfp8.Mfp8Error(st, "mfp8_linear")
+
+    def weight_bytes_per_step(self):
+        return sum(lin.N * lin.K + 4 * lin.N for lin in self.lins) * len(self.Ms)
+
+    def flops_per_step(self):
+        return sum(2 * M * lin.N * lin.K for M in self.Ms for lin in self.lins)
+
+    def launches_per_step(self):
+        return 2 * len(self.Ms) * len(self.lins)
+
+
+def time_graph(torch, fn, steps, warmup, dist_ctx):
+    """Capture fn() in a CUDA graph; time `steps` replays after `warmup`."""
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        fn(stream.cuda_stream)  # populate lazy state outside capture
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn(torch.cuda.current_stream().cuda_stream)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    ms = e0.elapsed_time(e1)
+    del g
+    return dist_ctx.max(ms)
+
+
+def kernel_times(torch, mfp8, layer, reps):
+    """Per-launch CUDA-event times of the GEMM kernel and the quantize
+    kernel, launched one at a time on the current stream."""
+    stream = torch.cuda.current_stream()
+    h = stream.cuda_stream
+    gemm_ms, gemm_bytes, gemm_flops, gemm_n = 0.0, 0, 0, 0
+    quant_ms, quant_bytes, quant_n = 0.0, 0, 0
+    x8 = {}
+    for mi, M in enumerate(layer.Ms):
+        for i, lin in enumerate(layer.lins):
+            x8[(M, i)] = mfp8.quantize_act(layer.x[(M, i)])
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        for mi, M in enumerate(layer.Ms):
+            s = layer.weight_set(mi)
+            for i, lin in enumerate(layer.lins):
+                q8, qs = x8[(M, i)]
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                e[0].record(stream)
+                st = mfp8.mfp8_quantize_act(layer.x[(M, i)].data_ptr(), M, lin.K, q8.data_ptr(), qs.data_ptr(), h)
+                e[1].record(stream)
+                e[2].record(stream)
+                st2 = mfp8.mfp8_gemm(q8.data_ptr(), qs.data_ptr(), M, lin.K, layer.w8[s][i].data_ptr(),
+                                     layer.sw[s][i].data_ptr(), lin.N, layer.y[(M, i)].data_ptr(), 0, h)
+                e[3].record(stream)
+                if st != mfp8.OK or st2 != mfp8.OK:
+                    raise mfp8.Mfp8Error(st or st2, "kernel timing")
+                torch.cuda.synchronize()
+                quant_ms += e[0].elapsed_time(e[1])
+                gemm_ms += e[2].elapsed_time(e[3])
+                quant_bytes += 3 * M * lin.K + 4 * M
+                gemm_bytes += lin.N * lin.K + 4 * lin.N + M * lin.K + 4 * M + 2 * M * lin.N
+                gemm_flops += 2 * M * lin.N * lin.K
+                gemm_n += 1
+                quant_n += 1
+    return dict(gemm_ms=gemm_ms, gemm_bytes=gemm_bytes, gemm_flops=gemm_flops, gemm_n=gemm_n,
+                quant_ms=quant_ms, quant_bytes=quant_bytes, quant_n=quant_n)
+
+
+def e2e_time(torch, mfp8, layer, steps, warmup, dist_ctx):
+    """Through the C ABI with host buffers: every step copies the step's
+    activations from pinned host memory, runs the 21 Linears, and reads the
+    outputs back."""
+    host_x = {k: v.cpu().pin_memory() for k, v in layer.x.items()}
+    host_y = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in layer.y.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_x.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_y.values())
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for k, v in host_x.items():
+            layer.x[k].copy_(v, non_blocking=True)
+        layer.step(mfp8, stream.cuda_stream)
+        for k, v in host_y.items():
+            v.copy_(layer.y[k], non_blocking=True)
+        torch.cuda.synchronize()
+
+    for _ in range(warmup):
+        one()
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one()
+    torch.cuda.synchronize()
+    ms = (time.perf_counter() - t0) * 1e3
+    dist_ctx.barrier()
+    return dist_ctx.max(ms), h2d, d2h
+
+
+# ----------------------------------------------------------- CPU oracle --
+
+def oracle_decode_sample(budget_s=12.0):
+    """The CPU oracle on decode steps of the same workload (BF16 inputs drawn
+    on the CPU with the same recipe), until about `budget_s` seconds:
+    per-token quantization of X and the exact contraction, per Linear.
+    Weights are quantized once, outside the timing (one-time, offline).
+    Returns (weight-read GB/s, threads, sample description)."""
+    import numpy as np
+    import torch
+    import oracle
+    from fp8_w8a8_dynamic_b200 import workloads as W
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    lins = W.LAYER_LINEARS
+    wq = []
+    for i, lin in enumerate(lins):
+        w8, sw = oracle.quantize_rows(bits(W.make_w(lin.N, lin.K, seed=1, stream=i, device="cpu")))
+        wq.append((w8, sw))
+    xs = {(M, i): bits(W.make_x(M, lin.K, seed=1, stream=M * 16 + i, device="cpu"))
+          for M in DECODE_MS for i, lin in enumerate(lins)}
+    done_bytes, elapsed, n_lin = 0, 0.0, 0
+    while elapsed < budget_s:
+        for M in DECODE_MS:
+            for i, lin in enumerate(lins):
+                t0 = time.perf_counter()
+                x8, sa = oracle.quantize_rows(xs[(M, i)])
+                oracle.linear_ref(x8, sa, wq[i][0], wq[i][1], want_abs=False)
+                elapsed += time.perf_counter() - t0
+                done_bytes += lin.N * lin.K + 4 * lin.N
+                n_lin += 1
+    return done_bytes / elapsed / 1e9, oracle.num_threads(), \
+        f"{n_lin} Linears of the decode step (M in {{1,4,8}}, q/k/v/o/gate/up/down), {elapsed:.1f} s of CPU time"
+
+
+# ---------------------------------------------------------------- dist --
+
+class DistCtx:
+    def __init__(self, torch):
+        self.torch = torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local_rank))
+            self.dist = dist
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, v):
+        if self.world == 1:
+            return v
+        t = self.torch.tensor([v], dtype=self.torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on the decode workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        gbs, cores, sample = oracle_decode_sample(budget_s=per_step)
+        if i >= args.warmup:
+            vals.append(gbs)
+    v = statistics.median(vals)
+    out = {
+        "impl": "reference", "metric": "FP8-dynamic Linear weight-read GB/s (decode, M in {1,4,8})",
+        "value": round(v, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": decode_config(),
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+def decode_config():
+    return {"workload": "decode: q/k/v/o/gate/up/down of one layer (hidden 4096, 32 Q / 8 KV heads, "
+                        "MLP 12288) at M in {1,4,8}, X ~N(0,1) + 0.1% x50 outliers, W ~N(0,0.02), seed 1",
+            "linears_per_step": 21, "weight_sets": 3, "l2": "inputs larger than L2: 579 MB of distinct e4m3 "
+            "weights per step (126 MB L2)", "graph": True}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    from fp8_w8a8_dynamic_b200 import build as B
+    from fp8_w8a8_dynamic_b200 import mfp8
+    from fp8_w8a8_dynamic_b200 import workloads as W
+
+    ctx = DistCtx(torch)
+    device = torch.device("cuda", ctx.local_rank)
+    torch.cuda.set_device(device)
+    B.build()
+    peaks = load_peaks()
+
+    # ---- decode (headline) ----
+    layer = Layer(torch, mfp8, W, seed=1 + 1000 * ctx.rank, weight_sets=3, Ms=DECODE_MS, device=device,
+                  x_kind="normal")
+    wbytes = layer.weight_bytes_per_step()
+    with ClockSampler(ctx.local_rank) as clocks:
+        ms = time_graph(torch, lambda h: layer.step(mfp8, h), args.steps, args.warmup, ctx)
+    assert mfp8.device_status() == mfp8.OK
+    step_ms = ms / args.steps
+    value = wbytes * ctx.world * args.steps / (ms * 1e-3) / 1e9
+
+    kt = kernel_times(torch, mfp8, layer, reps=max(3, min(args.steps, 10)))
+    gemm_gbs = kt["gemm_bytes"] / (kt["gemm_ms"] * 1e-3) / 1e9
+    quant_gbs = kt["quant_bytes"] / (kt["quant_ms"] * 1e-3) / 1e9
+
+    e2e_ms, h2d, d2h = e2e_time(torch, mfp8, layer, max(3, args.steps // 5), 3, ctx)
+    e2e_val = wbytes * ctx.world * max(3, args.steps // 5) / (e2e_ms * 1e-3) / 1e9
+    wq = {"GB/s": round(layer.wq_bytes / (layer.wq_time_ms * 1e-3) / 1e9, 1),
+          "bytes": layer.wq_bytes, "ms": round(layer.wq_time_ms, 3),
+          "frac_of_hbm": round(layer.wq_bytes / (layer.wq_time_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    del layer
+    torch.cuda.empty_cache()
+
+    # ---- prefill M = 2048 (the TFLOPS half of the metric) ----
+    prefill = None
+    if not args.no_prefill:
+        pl = Layer(torch, mfp8, W, seed=2 + 1000 * ctx.rank, weight_sets=1, Ms=(PREFILL_M,), device=device,
+                   x_kind="rowscale")
+        psteps = max(5, args.steps // 2)
+        pms = time_graph(torch, lambda h: pl.step(mfp8, h), psteps, args.warmup, ctx)
+        tflops = pl.flops_per_step() * psteps / (pms * 1e-3) / 1e12
+        pk = kernel_times(torch, mfp8, pl, reps=3)
+        g_tf = pk["gemm_flops"] / (pk["gemm_ms"] * 1e-3) / 1e12
+        fp8_peak = 2.0 * peaks["bf16_tflops"]
+        prefill = {"metric": "FP8-dynamic Linear TFLOPS (M=2048, 7 Linears, quantize included)",
+                   "value": round(tflops, 1), "unit": "TFLOP/s", "ms_per_step": round(pms / psteps, 4),
+                   "frac_of_fp8_peak": round(tflops / fp8_peak, 4),
+                   "roofline": {"bound": "tensor", "achieved": round(g_tf, 1), "peak": round(fp8_peak, 1),
+                                "unit": "TFLOP/s", "frac": round(g_tf / fp8_peak, 4), "traffic": None,
+                                "kernel": "gemm_tiled_kernel", "peak_source": f"{peaks['source']} bf16 x 2 (fp8/bf16 nominal ratio)"}}
+        del pl
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
+        gbs, cores, sample = oracle_decode_sample(budget_s=12.0)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    out = {
+        "metric": "FP8-dynamic Linear weight-read GB/s (decode, M in {1,4,8})",
+        "value": round(value, 1), "unit": "GB/s", "n_gpus": ctx.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 -> bf16",
+        "data": "synthetic", "config": decode_config(),
+        "frac_of_hbm": round(value / ctx.world / peaks["hbm_gbs"], 4),
+        "roofline": {"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "kernel": "gemm_splitk_kernel", "launches_timed": kt["gemm_n"],
+                     "avg_launch_us": round(kt["gemm_ms"] * 1e3 / kt["gemm_n"], 3),
+                     "peak_source": peaks["source"]},
+        "quantize_act": {"GB/s": round(quant_gbs, 1), "avg_launch_us": round(kt["quant_ms"] * 1e3 / kt["quant_n"], 3)},
+        "weight_quant": wq,
+        "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": layer_launches(args.steps),
+        "clocks": clocks.summary(),
+        "prefill": prefill,
+        "cpu_baseline": cpu,
+    }
+    if ctx.rank == 0:
+        print(json.dumps(out))
+    ctx.close()
+
+
+def layer_launches(steps):
+    return 2 * len(DECODE_MS) * 7 * steps
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,443 @@
+// mfp8.cu — the C ABI declared in include/mfp8.h: argument checks, kernel
+// choice, TMA descriptor set-up and launches.  The whole library is this
+// one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mfp8.h"
+#include "status.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+#include "gemm_tiled.cuh"
+#include "gemm_splitk.cuh"
+
+namespace mfp8 {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxDim = int64_t(1) << 30;  // rows / columns accepted per dimension
+
+struct DeviceInfo {
+    bool ready = false;
+    bool supported = false;
+    int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+mfp8_status current_device(int* dev_out, DeviceInfo* info_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return MFP8_ERR_CUDA;
+        }
+        d.supported = (major == 10 && minor == 0);
+        d.sm_count = sms;
+        d.ready = true;
+    }
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr) {
+            cudaGetLastError();
+            return MFP8_ERR_CUDA;
+        }
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (!d.supported) return MFP8_ERR_DEVICE;
+    *dev_out = dev;
+    *info_out = d;
+    return MFP8_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [rows, cols] row-major 8-bit matrix, tiles of box_rows x 128 bytes with
+// the 128-byte swizzle.
+mfp8_status make_map_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(cols)};
+    cuuint32_t box[2] = {128u, cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MFP8_OK : MFP8_ERR_CUDA;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+mfp8_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? MFP8_OK : MFP8_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- quantize --
+
+mfp8_status quantize_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
+    if (R == 0) return MFP8_OK;
+    const int64_t nvec = K / 8;
+    const uint4* x = static_cast<const uint4*>(X);
+    uint2* q = static_cast<uint2*>(Q);
+    const dim3 grid(static_cast<unsigned>(R)), block(kQuantThreads);
+    if (nvec <= 256) quant_rows_reg_kernel<1><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 512) quant_rows_reg_kernel<2><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 1024) quant_rows_reg_kernel<4><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 1536) quant_rows_reg_kernel<6><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 2048) quant_rows_reg_kernel<8><<<grid, block, 0, stream>>>(x, K, q, S);
+    else quant_rows_loop_kernel<<<grid, block, 0, stream>>>(x, K, q, S);
+    return launch_status();
+}
+
+mfp8_status check_quant_args(const void* X, int64_t R, int64_t K, const void* Q, const float* S) {
+    if (R < 0 || K < 0) return MFP8_ERR_INVALID_ARG;
+    if (K == 0 || K % 16 != 0 || K > kMaxDim || R > kMaxDim) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (R == 0) return MFP8_OK;
+    if (!X || !Q || !S) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Q) || !aligned16(S)) return MFP8_ERR_MISALIGNED;
+    if (ranges_overlap(X, size_t(R * K * 2), Q, size_t(R * K)) ||
+        ranges_overlap(X, size_t(R * K * 2), S, size_t(R * 4)) ||
+        ranges_overlap(Q, size_t(R * K), S, size_t(R * 4)))
+        return MFP8_ERR_INVALID_ARG;
+    return MFP8_OK;
+}
+
+// ----------------------------------------------------------------- GEMM --
+
+constexpr int kTiledBN = 256;
+constexpr int kTiledStages = 4;
+constexpr int64_t kSplitKMaxM = 128;
+
+template <class Kern>
+mfp8_status set_smem(Kern kern, int bytes, int dev, bool* done) {
+    if (done[dev]) return MFP8_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    done[dev] = true;
+    return MFP8_OK;
+}
+
+mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
+                         const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                         cudaStream_t stream) {
+    using L = tiled::Layout<kTiledBN, kTiledStages>;
+    auto kern = tiled::gemm_tiled_kernel<kTiledBN, kTiledStages>;
+    static bool attr_done[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
+    if (st != MFP8_OK) return st;
+    CUtensorMap tmX, tmW;
+    if ((st = make_map_u8(&tmX, X8, M, K, tiled::BM)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmW, W8, N, K, kTiledBN)) != MFP8_OK) return st;
+    const int64_t tiles = ((M + tiled::BM - 1) / tiled::BM) * ((N + kTiledBN - 1) / kTiledBN);
+    const unsigned grid = static_cast<unsigned>(tiles < info.sm_count ? tiles : info.sm_count);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(tiled::kThreads);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
+                           int(K)) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
+template <int MP, int STAGES>
+mfp8_status launch_splitk_mp(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
+                             const float* s_w, int64_t N, void* Y, bool dependent, int dev,
+                             const DeviceInfo& info, cudaStream_t stream) {
+    using L = splitk::Layout<MP, STAGES>;
+    auto kern = splitk::gemm_splitk_kernel<MP, STAGES>;
+    static bool attr_done[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
+    if (st != MFP8_OK) return st;
+    CUtensorMap tmW, tmX;
+    if ((st = make_map_u8(&tmW, W8, N, K, splitk::BW)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmX, X8, M, K, MP)) != MFP8_OK) return st;
+
+    const int64_t tiles = (N + splitk::BW - 1) / splitk::BW;
+    const int64_t kb_total = (K + splitk::BK - 1) / splitk::BK;
+    // Split K so that the grid covers the SMs about twice (two CTAs fit per
+    // SM for the small MP), without giving any CTA an empty K range.
+    const int per_sm = (2 * L::SMEM_BYTES <= 227 * 1024) ? 2 : 1;
+    int64_t S = (int64_t(info.sm_count) * per_sm + tiles - 1) / tiles;
+    if (S > splitk::kMaxCluster) S = splitk::kMaxCluster;
+    if (S > kb_total) S = kb_total;
+    if (S < 1) S = 1;
+    if (tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(S), unsigned(tiles));
+    cfg.blockDim = dim3(splitk::kThreads);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tmW, tmX, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
+                           int(K)) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
+mfp8_status launch_splitk(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
+                          const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                          cudaStream_t stream) {
+    if (M <= 16) return launch_splitk_mp<16, 5>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    if (M <= 32) return launch_splitk_mp<32, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    if (M <= 64) return launch_splitk_mp<64, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    if (M <= 128) return launch_splitk_mp<128, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    return MFP8_ERR_UNSUPPORTED_SHAPE;
+}
+
+int choose_path(int64_t M, int64_t N, int64_t K) {
+    (void)N;
+    (void)K;
+    return M <= 64 ? MFP8_PATH_SPLITK : MFP8_PATH_TILED;
+}
+
+mfp8_status check_gemm_args(int64_t M, int64_t N, int64_t K, const void* W8, const float* s_w, const void* Y) {
+    if (M < 0 || N < 0 || K < 0) return MFP8_ERR_INVALID_ARG;
+    if (K == 0 || K % 16 != 0 || N == 0 || N % 8 != 0 || K > kMaxDim || N > kMaxDim || M > kMaxDim)
+        return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (M > 0 && M * (K > N ? K : N) > (int64_t(1) << 40)) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (!W8 || !s_w || (M > 0 && !Y)) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(W8) || !aligned16(s_w) || !aligned16(Y)) return MFP8_ERR_MISALIGNED;
+    if (M > 0 && (ranges_overlap(Y, size_t(M * N * 2), W8, size_t(N * K)) ||
+                  ranges_overlap(Y, size_t(M * N * 2), s_w, size_t(N * 4))))
+        return MFP8_ERR_INVALID_ARG;
+    return MFP8_OK;
+}
+
+mfp8_status run_gemm(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+                     int64_t N, void* Y, int path, bool dependent, int dev, const DeviceInfo& info,
+                     cudaStream_t stream) {
+    if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
+    // The tiled kernel takes M, N, K as 32-bit; tile counts must fit too.
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_TILED) return launch_tiled(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    if (path == MFP8_PATH_SPLITK) {
+        if (M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+        return launch_splitk(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    }
+    return MFP8_ERR_INVALID_ARG;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace: X8 [M, K] then s_a [M], each 256-byte aligned.
+size_t workspace_bytes(int64_t M, int64_t K) {
+    return round_up(size_t(M) * size_t(K), 256) + round_up(size_t(M) * 4, 256);
+}
+
+__global__ void bounded_wait_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // Nothing ever arrives on this barrier: the wait must give up.
+        mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+    }
+}
+
+}  // namespace
+}  // namespace mfp8
+
+using namespace mfp8;
+
+extern "C" {
+
+mfp8_status mfp8_quantize_weight(const void* W_bf16, int64_t N, int64_t K, void* W_fp8, float* w_scale,
+                                 void* stream) {
+    mfp8_status st = check_quant_args(W_bf16, N, K, W_fp8, w_scale);
+    if (st != MFP8_OK || N == 0) return st;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
+    return quantize_rows(W_bf16, N, K, W_fp8, w_scale, static_cast<cudaStream_t>(stream));
+}
+
+mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K, void* X_fp8, float* x_scale,
+                              void* stream) {
+    mfp8_status st = check_quant_args(X_bf16, M, K, X_fp8, x_scale);
+    if (st != MFP8_OK || M == 0) return st;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
+    return quantize_rows(X_bf16, M, K, X_fp8, x_scale, static_cast<cudaStream_t>(stream));
+}
+
+size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || K > kMaxDim) return 0;
+    return workspace_bytes(M, K);
+}
+
+mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
+                           int64_t N, void* Y_bf16, void* workspace, size_t workspace_bytes_given, int path,
+                           void* X_fp8_out, float* x_scale_out, void* stream) {
+    mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
+    if (st != MFP8_OK) return st;
+    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_SPLITK) return MFP8_ERR_INVALID_ARG;
+    if (path == MFP8_PATH_SPLITK && M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return MFP8_OK;
+    if (!X_bf16) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(X_bf16)) return MFP8_ERR_MISALIGNED;
+    if ((X_fp8_out == nullptr) != (x_scale_out == nullptr)) return MFP8_ERR_INVALID_ARG;
+    if (ranges_overlap(X_bf16, size_t(M * K * 2), Y_bf16, size_t(M * N * 2))) return MFP8_ERR_INVALID_ARG;
+
+    void* X8;
+    float* s_a;
+    if (X_fp8_out) {
+        if (!aligned16(X_fp8_out) || !aligned16(x_scale_out)) return MFP8_ERR_MISALIGNED;
+        X8 = X_fp8_out;
+        s_a = x_scale_out;
+    } else {
+        const size_t need = workspace_bytes(M, K);
+        if (!workspace || workspace_bytes_given < need) return MFP8_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
+        X8 = workspace;
+        s_a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(size_t(M) * size_t(K), 256));
+    }
+    if ((st = check_quant_args(X_bf16, M, K, X8, s_a)) != MFP8_OK) return st;
+    if (ranges_overlap(X8, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
+        ranges_overlap(s_a, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
+        return MFP8_ERR_INVALID_ARG;
+
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = quantize_rows(X_bf16, M, K, X8, s_a, s)) != MFP8_OK) return st;
+    return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, path, /*dependent=*/true, dev, info, s);
+}
+
+mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
+                        int64_t N, void* Y_bf16, void* workspace, size_t workspace_bytes_given, void* stream) {
+    return mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes_given,
+                          MFP8_PATH_AUTO, nullptr, nullptr, stream);
+}
+
+mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K, const void* W_fp8,
+                      const float* w_scale, int64_t N, void* Y_bf16, int path, void* stream) {
+    mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
+    if (st != MFP8_OK) return st;
+    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_SPLITK) return MFP8_ERR_INVALID_ARG;
+    if (path == MFP8_PATH_SPLITK && M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return MFP8_OK;
+    if (!X_fp8 || !x_scale) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(X_fp8) || !aligned16(x_scale)) return MFP8_ERR_MISALIGNED;
+    if (ranges_overlap(X_fp8, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
+        ranges_overlap(x_scale, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
+        return MFP8_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
+    return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, /*dependent=*/false, dev, info,
+                    static_cast<cudaStream_t>(stream));
+}
+
+mfp8_status mfp8_e4m3_encode_f32(const float* in, int64_t n, uint8_t* out, void* stream) {
+    if (n < 0) return MFP8_ERR_INVALID_ARG;
+    if (n == 0) return MFP8_OK;
+    if (!in || !out) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(in) || !aligned16(out)) return MFP8_ERR_MISALIGNED;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    const int64_t pairs = (n + 1) / 2;
+    int64_t blocks = (pairs + 255) / 256;
+    const int64_t cap = int64_t(info.sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    e4m3_encode_kernel<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(in, n, out);
+    return launch_status();
+}
+
+mfp8_status mfp8_debug_bounded_wait(int64_t timeout_us, void* stream) {
+    if (timeout_us < 1 || timeout_us > 100000) return MFP8_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(timeout_us) * 1000u);
+    return launch_status();
+}
+
+mfp8_status mfp8_get_device_status(void* stream) {
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    int word = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_device_status, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return static_cast<mfp8_status>(word);
+}
+
+const char* mfp8_status_string(mfp8_status status) {
+    switch (status) {
+        case MFP8_OK: return "ok";
+        case MFP8_ERR_INVALID_ARG: return "invalid argument";
+        case MFP8_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case MFP8_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (K must be a positive multiple of 16, N of 8)";
+        case MFP8_ERR_WORKSPACE: return "workspace missing or too small";
+        case MFP8_ERR_CUDA: return "CUDA runtime error";
+        case MFP8_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+        case MFP8_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
+    }
+    return "unknown status";
+}
+
+int mfp8_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// quant.cuh — per-row (per-token / per-output-channel) e4m3 quantization.
+//
+// Source of the rule: "MOSS-VL quantization README", FP8-Dynamic recipe
+// section (weights float8_e4m3fn channel-wise static; activations FP8
+// per-token dynamic) and the "MOSS-VL-Realtime-FP8 mixed-precision strategy"
+// article, section "252 个主力 Linear 层为什么用 FP8 E4M3".  One rule serves
+// both: a weight row is an output channel, an activation row is a token.
+//   s    = fl32(max_k |x_k| / 448), raised to FLT_MIN when smaller
+//   q_k  = e4m3_rn_satfinite(fl32(x_k / s))
+// The divisions are IEEE round-to-nearest (__fdiv_rn), never a reciprocal
+// multiply, so the codes are bit-identical to the CPU oracle's.
+//
+// Memory-bound: each row is read once (16-byte loads, 8 bf16 per load),
+// held in registers while the block reduces its absmax, then converted and
+// stored as packed 8-byte groups of codes.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace mfp8 {
+
+constexpr float kFltMin = 1.17549435082228750797e-38f;  // 2^-126
+constexpr float kE4m3Max = 448.0f;
+
+// Two fp32 values -> two e4m3 codes, `lo` in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    // The first source operand lands in the upper byte.
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// |x| of a bf16 orders like its 15 low bits read as an unsigned integer, so
+// the absmax is an integer max (exact, and NaN-free inputs assumed).
+__device__ __forceinline__ uint32_t absmax_bits_u4(uint4 v, uint32_t acc) {
+    const uint32_t m = 0x7fff7fffu;
+    acc = __vmaxu2(acc, v.x & m);
+    acc = __vmaxu2(acc, v.y & m);
+    acc = __vmaxu2(acc, v.z & m);
+    acc = __vmaxu2(acc, v.w & m);
+    return acc;
+}
+
+__device__ __forceinline__ float scale_from_absmax_bits(uint32_t amax16) {
+    const float amax = __uint_as_float(amax16 << 16);
+    float s = __fdiv_rn(amax, kE4m3Max);
+    return s < kFltMin ? kFltMin : s;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 8 bf16 values -> 8 e4m3 codes (byte i = value i).
+__device__ __forceinline__ uint2 quantize8(uint4 v, float s) {
+    uint2 q;
+    q.x = e4m3x2(__fdiv_rn(bf16_lo(v.x), s), __fdiv_rn(bf16_hi(v.x), s)) |
+          (e4m3x2(__fdiv_rn(bf16_lo(v.y), s), __fdiv_rn(bf16_hi(v.y), s)) << 16);
+    q.y = e4m3x2(__fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s)) |
+          (e4m3x2(__fdiv_rn(bf16_lo(v.w), s), __fdiv_rn(bf16_hi(v.w), s)) << 16);
+    return q;
+}
+
+constexpr int kQuantThreads = 256;
+
+// Block-wide max of a 16-bit magnitude held by every thread.
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red /* [8] */) {
+    v = __reduce_max_sync(0xffffffffu, v);
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[warp] = v;
+    __syncthreads();
+    uint32_t r = red[0];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) r = max(r, red[w]);
+    return r;
+}
+
+// One block per row; the row (K/8 16-byte vectors) lives in registers,
+// VPT vectors per thread.  Requires K/8 <= VPT * 256.
+template <int VPT>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
+                      float* __restrict__ S) {
+    grid_launch_dependents();
+    __shared__ uint32_t red[kQuantThreads / 32];
+    const int64_t row = blockIdx.x;
+    const int64_t nvec = K >> 3;
+    const uint4* xr = X + row * nvec;
+    uint4 v[VPT];
+    uint32_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int64_t j = threadIdx.x + int64_t(i) * kQuantThreads;
+        if (j < nvec) {
+            v[i] = __ldg(xr + j);
+            acc = absmax_bits_u4(v[i], acc);
+        } else {
+            v[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    const uint32_t amax = block_max_u32(max(acc & 0xffffu, acc >> 16), red);
+    const float s = scale_from_absmax_bits(amax);
+    if (threadIdx.x == 0) S[row] = s;
+    uint2* qr = Q + row * nvec;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int64_t j = threadIdx.x + int64_t(i) * kQuantThreads;
+        if (j < nvec) qr[j] = quantize8(v[i], s);
+    }
+}
+
+// Any K: two passes over the row (the second one is served by L2).
+__global__ void __launch_bounds__(kQuantThreads)
+quant_rows_loop_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
+                       float* __restrict__ S) {
+    grid_launch_dependents();
+    __shared__ uint32_t red[kQuantThreads / 32];
+    const int64_t row = blockIdx.x;
+    const int64_t nvec = K >> 3;
+    const uint4* xr = X + row * nvec;
+    uint32_t acc = 0;
+    for (int64_t j = threadIdx.x; j < nvec; j += kQuantThreads) acc = absmax_bits_u4(__ldg(xr + j), acc);
+    const uint32_t amax = block_max_u32(max(acc & 0xffffu, acc >> 16), red);
+    const float s = scale_from_absmax_bits(amax);
+    if (threadIdx.x == 0) S[row] = s;
+    uint2* qr = Q + row * nvec;
+    for (int64_t j = threadIdx.x; j < nvec; j += kQuantThreads) qr[j] = quantize8(__ldg(xr + j), s);
+}
+
+// Diagnostic: the e4m3 conversion alone, on arbitrary fp32 values.
+__global__ void e4m3_encode_kernel(const float* __restrict__ in, int64_t n, uint8_t* __restrict__ out) {
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t p = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; 2 * p < n; p += stride) {
+        const int64_t i = 2 * p;
+        if (i + 1 < n) {
+            const uint32_t c = e4m3x2(in[i], in[i + 1]);
+            out[i] = uint8_t(c & 0xff);
+            out[i + 1] = uint8_t(c >> 8);
+        } else {
+            out[i] = uint8_t(e4m3x2(in[i], 0.0f) & 0xff);
+        }
+    }
+}
+
+}  // namespace mfp8

@@ -1,0 +1,200 @@
+"""Python binding of the C ABI in include/mfp8.h.
+
+The ``mfp8_*`` functions here have the C names and arguments (integer device
+pointers, sizes, a cudaStream_t as an integer) and only marshal arguments.
+The torch helpers below them allocate outputs with torch and pass pointers;
+every step of the computation runs in the CUDA kernels of libmfp8.so.  There
+is no CPU fallback: without the built library every call raises.
+"""
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmfp8.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_MISALIGNED = 2
+ERR_UNSUPPORTED_SHAPE = 3
+ERR_WORKSPACE = 4
+ERR_CUDA = 5
+ERR_TIMEOUT = 6
+ERR_DEVICE = 7
+
+PATH_AUTO = 0
+PATH_TILED = 1
+PATH_SPLITK = 2
+
+
+class Mfp8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {mfp8_status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(python -m fp8_w8a8_dynamic_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        sig = {
+            "mfp8_quantize_weight": (i32, [P, i64, i64, P, P, P]),
+            "mfp8_quantize_act": (i32, [P, i64, i64, P, P, P]),
+            "mfp8_linear_workspace_bytes": (sz, [i64, i64, i64]),
+            "mfp8_linear": (i32, [P, i64, i64, P, P, i64, P, P, sz, P]),
+            "mfp8_linear_ex": (i32, [P, i64, i64, P, P, i64, P, P, sz, i32, P, P, P]),
+            "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, i32, P]),
+            "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
+            "mfp8_debug_bounded_wait": (i32, [i64, P]),
+            "mfp8_get_device_status": (i32, [P]),
+            "mfp8_status_string": (ctypes.c_char_p, [i32]),
+            "mfp8_version": (i32, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- C names --
+
+def mfp8_quantize_weight(W_bf16, N, K, W_fp8, w_scale, stream=0):
+    return lib().mfp8_quantize_weight(W_bf16, N, K, W_fp8, w_scale, stream)
+
+
+def mfp8_quantize_act(X_bf16, M, K, X_fp8, x_scale, stream=0):
+    return lib().mfp8_quantize_act(X_bf16, M, K, X_fp8, x_scale, stream)
+
+
+def mfp8_linear_workspace_bytes(M, N, K):
+    return lib().mfp8_linear_workspace_bytes(M, N, K)
+
+
+def mfp8_linear(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, stream=0):
+    return lib().mfp8_linear(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, stream)
+
+
+def mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, path,
+                   X_fp8_out, x_scale_out, stream=0):
+    return lib().mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes,
+                                path, X_fp8_out, x_scale_out, stream)
+
+
+def mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path=PATH_AUTO, stream=0):
+    return lib().mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, stream)
+
+
+def mfp8_e4m3_encode_f32(inp, n, out, stream=0):
+    return lib().mfp8_e4m3_encode_f32(inp, n, out, stream)
+
+
+def mfp8_debug_bounded_wait(timeout_us, stream=0):
+    return lib().mfp8_debug_bounded_wait(timeout_us, stream)
+
+
+def mfp8_get_device_status(stream=0):
+    return lib().mfp8_get_device_status(stream)
+
+
+def mfp8_status_string(status):
+    return lib().mfp8_status_string(int(status)).decode()
+
+
+def mfp8_version():
+    return lib().mfp8_version()
+
+
+# ---------------------------------------------------------- torch helpers --
+
+def _check(status, where):
+    if status != OK:
+        raise Mfp8Error(status, where)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t):
+    return t.data_ptr() if t is not None else None
+
+
+def quantize_weight(W, stream=None):
+    """W: bf16 [N, K] CUDA tensor -> (W_fp8 uint8 [N, K], w_scale fp32 [N])."""
+    import torch
+    N, K = W.shape
+    W8 = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    sw = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _check(mfp8_quantize_weight(_ptr(W), N, K, _ptr(W8), _ptr(sw), _stream_handle(stream)),
+           "mfp8_quantize_weight")
+    return W8, sw
+
+
+def quantize_act(X, stream=None):
+    """X: bf16 [M, K] CUDA tensor -> (X_fp8 uint8 [M, K], x_scale fp32 [M])."""
+    import torch
+    M, K = X.shape
+    X8 = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    sa = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _check(mfp8_quantize_act(_ptr(X), M, K, _ptr(X8), _ptr(sa), _stream_handle(stream)),
+           "mfp8_quantize_act")
+    return X8, sa
+
+
+def workspace_for(M, N, K, device):
+    import torch
+    nbytes = mfp8_linear_workspace_bytes(M, N, K)
+    return torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=device)
+
+
+def linear(X, W8, w_scale, out=None, workspace=None, path=PATH_AUTO, x8_out=None, xs_out=None,
+           stream=None):
+    """Y = FP8_DYNAMIC Linear(X) with pre-quantized weights.  X bf16 [M, K]."""
+    import torch
+    M, K = X.shape
+    N = W8.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if workspace is None and x8_out is None:
+        workspace = workspace_for(M, N, K, X.device)
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(mfp8_linear_ex(_ptr(X), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), _ptr(workspace),
+                          ws_bytes, path, _ptr(x8_out), _ptr(xs_out), _stream_handle(stream)),
+           "mfp8_linear_ex")
+    return out
+
+
+def gemm(X8, x_scale, W8, w_scale, out=None, path=PATH_AUTO, stream=None):
+    """The contraction alone on pre-quantized activations."""
+    import torch
+    M, K = X8.shape
+    N = W8.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X8.device)
+    _check(mfp8_gemm(_ptr(X8), _ptr(x_scale), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), path,
+                     _stream_handle(stream)), "mfp8_gemm")
+    return out
+
+
+def e4m3_encode(values, stream=None):
+    """fp32 CUDA tensor -> uint8 codes from the device's conversion."""
+    import torch
+    out = torch.empty(values.shape, dtype=torch.uint8, device=values.device)
+    _check(mfp8_e4m3_encode_f32(_ptr(values), values.numel(), _ptr(out), _stream_handle(stream)),
+           "mfp8_e4m3_encode_f32")
+    return out
+
+
+def device_status(stream=None):
+    return mfp8_get_device_status(_stream_handle(stream))

@@ -1,0 +1,165 @@
+/*
+ * mfp8.h — C ABI of the B200 (sm_100a) FP8_DYNAMIC quantized Linear.
+ *
+ * The method (stated by the "MOSS-VL quantization README", github OpenMOSS/
+ * MOSS-VL quantization/, FP8-Dynamic recipe section, and by the
+ * "MOSS-VL-Realtime-FP8 mixed-precision strategy" article, section
+ * "252 个主力 Linear 层为什么用 FP8 E4M3"):
+ *   - weights are float8_e4m3fn with one static scale per output channel,
+ *     computed once, offline;
+ *   - the input activations of the quantized kernels are float8_e4m3fn with
+ *     one scale per token, computed at run time;
+ *   - the product of the two is rescaled and written back as BF16 (the
+ *     recipe runs the model in bfloat16).
+ * Readings taken where the pages are silent (the same in the CPU oracle):
+ *   scale      s = fl32(max|row| / 448), raised to FLT_MIN (2^-126) if smaller;
+ *   code       e4m3(fl32(x / s)) with an IEEE round-to-nearest fp32 divide,
+ *              then round-to-nearest-even to e4m3, saturating to +-448;
+ *   product    fp32 accumulation of the e4m3 x e4m3 products on the tensor
+ *              cores, then y = bf16_rn(acc * s_a[m] * s_w[n]); no bias.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless stated; the caller allocates and
+ *     owns every buffer, including any workspace.  Nothing here allocates
+ *     device memory or keeps a pointer after the call returns.
+ *   - Matrices are row-major and contiguous.  X is [M, K] (one row per
+ *     token), W is [N, K] (one row per output channel: the Linear's
+ *     (out_features, in_features) layout), Y is [M, N].  BF16 buffers hold
+ *     IEEE bfloat16 bit patterns; FP8 buffers hold float8_e4m3fn codes, one
+ *     byte each; scales are fp32.
+ *   - Every pointer must be 16-byte aligned.  K must be a positive multiple
+ *     of 16, N a positive multiple of 8, M >= 0 (M == 0 is a no-op).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued on it; no call blocks the host except mfp8_get_device_status.
+ *     The calls do not synchronise and may be captured in a CUDA graph.
+ *   - Argument errors are returned before anything is enqueued.  Errors that
+ *     arise on the device (a bounded wait that ran out) are recorded in a
+ *     per-device status word that mfp8_get_device_status reads and clears.
+ *     Nothing is thrown across this boundary.
+ *   - Inputs holding Inf or NaN are outside the contract: the kernels still
+ *     terminate, but the outputs are unspecified.
+ */
+#ifndef MFP8_H
+#define MFP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MFP8_API __attribute__((visibility("default")))
+#else
+#define MFP8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MFP8_OK = 0,
+    MFP8_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, overlapping in/out */
+    MFP8_ERR_MISALIGNED = 2,        /* a pointer is not 16-byte aligned */
+    MFP8_ERR_UNSUPPORTED_SHAPE = 3, /* K not a positive multiple of 16, N not a positive multiple of 8, too large */
+    MFP8_ERR_WORKSPACE = 4,         /* workspace missing or smaller than mfp8_linear_workspace_bytes */
+    MFP8_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    MFP8_ERR_TIMEOUT = 6,           /* a kernel's bounded wait ran out (device status) */
+    MFP8_ERR_DEVICE = 7             /* the current device is not compute capability 10.0 */
+} mfp8_status;
+
+/* Per-channel weight quantization (one-time, offline).
+ * Source: README FP8-Dynamic section, "float8_e4m3fn channel-wise static";
+ * Realtime-FP8 article: per-channel scales computed once, zero run-time cost.
+ *   W_bf16  [N, K] bf16, read only.
+ *   W_fp8   [N, K] e4m3 codes, written.      w_scale [N] fp32, written.
+ *   W_fp8[n,k] = e4m3(fl32(W[n,k] / w_scale[n])), w_scale[n] = fl32(max_k |W[n,k]| / 448).
+ * Bit-exact with the CPU oracle. */
+MFP8_API mfp8_status mfp8_quantize_weight(const void* W_bf16, int64_t N, int64_t K,
+                                 void* W_fp8, float* w_scale, void* stream);
+
+/* Per-token activation quantization (every call).
+ * Source: README FP8-Dynamic section, "FP8 per-token dynamic"; Realtime-FP8
+ * article: the scale is computed for each token at run time.
+ *   X_bf16 [M, K] bf16, read only.
+ *   X_fp8  [M, K] e4m3 codes, written.       x_scale [M] fp32, written.
+ * Same rule as mfp8_quantize_weight, one scale per row of X. */
+MFP8_API mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K,
+                              void* X_fp8, float* x_scale, void* stream);
+
+/* Bytes of device workspace mfp8_linear needs for these sizes (0 when the
+ * chosen kernel quantizes X on chip).  Never fails; returns 0 for invalid
+ * sizes (mfp8_linear then reports the error). */
+MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* The FP8_DYNAMIC Linear: Y = bf16(  (Xq . Wq^T) * x_scale (x) w_scale  ).
+ * Source: README FP8-Dynamic section (FP8 weights, per-token FP8 inputs to
+ * "the quantized kernels", model in bfloat16).
+ *   X_bf16   [M, K] bf16 activations, read only.
+ *   W_fp8    [N, K] e4m3 weight codes and w_scale [N] fp32, both from
+ *            mfp8_quantize_weight, read only.
+ *   Y_bf16   [M, N] bf16, written.  Must not overlap any input.
+ *   workspace / workspace_bytes: device scratch of at least
+ *            mfp8_linear_workspace_bytes(M, N, K) bytes (may be NULL when
+ *            that is 0).  Its contents on entry do not matter; they are
+ *            garbage on exit.  Concurrent calls need separate workspaces.
+ * The activation quantization (per-token scale + e4m3 codes) happens inside
+ * this call: its codes and scales are bit-identical to mfp8_quantize_act.
+ * Outputs are within |y - y_ref| <= 2^-7 |y_ref| + 1e-5 * sum_k |a_k w_k| s_a s_w
+ * of the exact rescaled product y_ref. */
+MFP8_API mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K,
+                        const void* W_fp8, const float* w_scale, int64_t N,
+                        void* Y_bf16, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Kernel choice for mfp8_linear_ex. */
+typedef enum {
+    MFP8_PATH_AUTO = 0,   /* what mfp8_linear does: chosen from M, N, K */
+    MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
+    MFP8_PATH_SPLITK = 2  /* weight-streaming split-K tcgen05 GEMM (M <= 128) */
+} mfp8_path;
+
+/* mfp8_linear with an explicit kernel choice, and optional copies of the
+ * activation codes and scales it computed (X_fp8_out [M, K] and
+ * x_scale_out [M]; pass NULL for none).  Used to test each kernel on the
+ * same shapes and to check that the activation bytes of every path are
+ * bit-identical to mfp8_quantize_act.  Returns MFP8_ERR_UNSUPPORTED_SHAPE if
+ * the chosen kernel cannot take these sizes. */
+MFP8_API mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K,
+                           const void* W_fp8, const float* w_scale, int64_t N,
+                           void* Y_bf16, void* workspace, size_t workspace_bytes,
+                           int path, void* X_fp8_out, float* x_scale_out,
+                           void* stream);
+
+/* The contraction and epilogue alone, on activations already quantized by
+ * mfp8_quantize_act: Y = bf16((X_fp8 . W_fp8^T) * x_scale (x) w_scale).
+ * Lets the GEMM be timed and checked without the quantize pass. */
+MFP8_API mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K,
+                      const void* W_fp8, const float* w_scale, int64_t N,
+                      void* Y_bf16, int path, void* stream);
+
+/* Diagnostic: encode n fp32 values with the device's e4m3 conversion (the
+ * one the quantize kernels use).  in [n] fp32, out [n] codes.  Used to check
+ * the hardware conversion against the oracle on every fp32 bit pattern. */
+MFP8_API mfp8_status mfp8_e4m3_encode_f32(const float* in, int64_t n, uint8_t* out, void* stream);
+
+/* Diagnostic: one kernel waits on a barrier that nothing releases, with a
+ * bound of `timeout_us` microseconds (at most 100000), then records
+ * MFP8_ERR_TIMEOUT in the status word and returns.  Exercises the
+ * device-error path without faulting or hanging the GPU. */
+MFP8_API mfp8_status mfp8_debug_bounded_wait(int64_t timeout_us, void* stream);
+
+/* Synchronises `stream`, then reads and clears the current device's status
+ * word.  Returns MFP8_OK, MFP8_ERR_TIMEOUT, or MFP8_ERR_CUDA if the
+ * synchronisation itself failed. */
+MFP8_API mfp8_status mfp8_get_device_status(void* stream);
+
+/* Static description of a status code (never NULL). */
+MFP8_API const char* mfp8_status_string(mfp8_status status);
+
+/* Library version, as major * 10000 + minor * 100 + patch. */
+MFP8_API int mfp8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MFP8_H */

@@ -1,0 +1,106 @@
+"""The C ABI library: it builds, loads without a GPU, exports every symbol the
+header declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_w8a8_dynamic_b200 import build as B
+from fp8_w8a8_dynamic_b200 import mfp8
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "mfp8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return mfp8.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MFP8_API\s+[\w\s\*]+?\b(mfp8_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for required in ("mfp8_quantize_weight", "mfp8_quantize_act", "mfp8_linear",
+                     "mfp8_linear_workspace_bytes", "mfp8_get_device_status", "mfp8_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(mfp8.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(raw, name), f"{name} declared in mfp8.h but not exported"
+
+
+def test_library_does_not_need_libcuda():
+    # The driver is reached through cudaGetDriverEntryPoint at run time.
+    out = os.popen(f"ldd {mfp8.LIB_PATH}").read()
+    assert "libcuda.so" not in out and "libtorch" not in out
+
+
+def test_status_strings_and_version(lib):
+    for code in range(8):
+        assert mfp8.mfp8_status_string(code)
+    assert "unknown" in mfp8.mfp8_status_string(99)
+    assert mfp8.mfp8_version() >= 100
+
+
+def test_workspace_bytes(lib):
+    # X8 [M, K] then s_a [M], each rounded up to 256 bytes
+    assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == 65536 + 256
+    assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == 256 + 256
+    assert mfp8.mfp8_linear_workspace_bytes(0, 8, 48) == 0
+    assert mfp8.mfp8_linear_workspace_bytes(4, 8, -1) == 0
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null address; never dereferenced
+
+
+def test_argument_errors_are_reported_before_any_launch(lib):
+    q = mfp8.mfp8_quantize_act
+    assert q(FAKE, 4, 0, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # K == 0
+    assert q(FAKE, 4, 40, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # K % 16
+    assert q(FAKE, -1, 64, FAKE * 2, FAKE * 3, None) == mfp8.ERR_INVALID_ARG
+    assert q(None, 4, 64, FAKE * 2, FAKE * 3, None) == mfp8.ERR_INVALID_ARG
+    assert q(FAKE + 8, 4, 64, FAKE * 2, FAKE * 3, None) == mfp8.ERR_MISALIGNED
+    assert q(FAKE, 4, 64, FAKE + 16, FAKE * 3, None) == mfp8.ERR_INVALID_ARG  # output overlaps input
+    assert q(FAKE, 0, 64, None, None, None) == mfp8.OK  # empty: nothing to do
+    w = mfp8.mfp8_quantize_weight
+    assert w(FAKE, 8, 24, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+
+    L = mfp8.mfp8_linear_ex
+    args = dict(X=FAKE, M=4, K=64, W=FAKE * 2, sw=FAKE * 3, N=64, Y=FAKE * 4, ws=FAKE * 5, wsb=1 << 16)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return L(a["X"], a["M"], a["K"], a["W"], a["sw"], a["N"], a["Y"], a["ws"], a["wsb"],
+                 kw.get("path", 0), kw.get("x8", None), kw.get("xs", None), None)
+
+    assert call(N=12) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(N=0) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(K=8) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(W=None) == mfp8.ERR_INVALID_ARG
+    assert call(Y=FAKE * 4 + 4) == mfp8.ERR_MISALIGNED
+    assert call(ws=None) == mfp8.ERR_WORKSPACE
+    assert call(wsb=100) == mfp8.ERR_WORKSPACE
+    assert call(path=7) == mfp8.ERR_INVALID_ARG
+    assert call(path=mfp8.PATH_SPLITK, M=129) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
+    assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X
+    assert call(M=0) == mfp8.OK
+    G = mfp8.mfp8_gemm
+    assert G(None, FAKE, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, 0, None) == mfp8.ERR_INVALID_ARG
+    assert mfp8.mfp8_e4m3_encode_f32(FAKE, -1, FAKE * 2, None) == mfp8.ERR_INVALID_ARG
+    assert mfp8.mfp8_debug_bounded_wait(0, None) == mfp8.ERR_INVALID_ARG
+    assert mfp8.mfp8_debug_bounded_wait(10 ** 6, None) == mfp8.ERR_INVALID_ARG
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(mfp8, "_lib", None)
+    monkeypatch.setattr(mfp8, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        mfp8.lib()

@@ -1,0 +1,149 @@
+"""The FP8_DYNAMIC Linear on the GPU against the CPU oracle.
+
+Activation and weight codes/scales: bit-exact.  BF16 outputs: within
+|y - y_ref| <= 2^-7 |y_ref| + 1e-5 * sum_k |a_k w_k| s_a s_w of the exact
+rescaled product, element by element."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_w8a8_dynamic_b200 import mfp8
+from fp8_w8a8_dynamic_b200 import workloads as W
+from helpers import assert_linear_parity, bits16, f32, u8
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_case(M, N, K, path, seed=0, kind="normal", rows=None, check_codes=True):
+    x = W.make_x(M, K, seed=seed, stream=M, kind=kind, device=DEV)
+    w = W.make_w(N, K, seed=seed, stream=N, device=DEV)
+    W8, sw = mfp8.quantize_weight(w)
+    x8 = torch.empty((M, K), dtype=torch.uint8, device=DEV)
+    xs = torch.empty((M,), dtype=torch.float32, device=DEV)
+    y = mfp8.linear(x, W8, sw, path=path, x8_out=x8, xs_out=xs)
+    torch.cuda.synchronize()
+    assert mfp8.device_status() == mfp8.OK
+    w8_h, sw_h = u8(W8), f32(sw)
+    x8_h, xs_h = u8(x8), f32(xs)
+    if check_codes:
+        w8_ref, sw_ref = oracle.quantize_rows(bits16(w))
+        assert np.array_equal(w8_h, w8_ref) and np.array_equal(sw_h.view(np.uint32), sw_ref.view(np.uint32))
+        x8_ref, xs_ref = oracle.quantize_rows(bits16(x))
+        assert np.array_equal(x8_h, x8_ref), "activation codes differ from the oracle"
+        assert np.array_equal(xs_h.view(np.uint32), xs_ref.view(np.uint32)), "activation scales differ"
+    assert_linear_parity(y, x8_h, xs_h, w8_h, sw_h, rows=rows, what=f"M={M} N={N} K={K} path={path}")
+    return x, W8, sw, y
+
+
+SMALL = [  # (M, N, K): several tiles, ragged tails in M, N and K
+    (1, 128, 128), (5, 256, 256), (16, 4096, 4096), (17, 384, 272), (64, 1024, 4096),
+    (3, 136, 48), (2, 8, 16), (128, 512, 640), (33, 264, 400),
+]
+TILED_ONLY = [(130, 264, 384), (300, 520, 1040), (256, 1024, 4096), (1000, 2056, 528), (129, 4096, 128)]
+
+
+@pytest.mark.parametrize("M,N,K", SMALL)
+@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_AUTO])
+def test_linear_small(M, N, K, path):
+    run_case(M, N, K, path, seed=M * 7 + N)
+
+
+@pytest.mark.parametrize("M,N,K", TILED_ONLY)
+def test_linear_tiled_ragged(M, N, K):
+    run_case(M, N, K, mfp8.PATH_TILED, seed=11, kind="rowscale")
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 4096, 4096), (130, 264, 384), (64, 1024, 4096)])
+def test_gemm_entry_point_matches_linear(M, N, K):
+    x, W8, sw, y = run_case(M, N, K, mfp8.PATH_AUTO, seed=5, check_codes=False)
+    x8, xs = mfp8.quantize_act(x)
+    y2 = mfp8.gemm(x8, xs, W8, sw)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_deterministic():
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK):
+        x = W.make_x(16, 4096, seed=0, device=DEV)
+        W8, sw = mfp8.quantize_weight(W.make_w(4096, 4096, seed=0, device=DEV))
+        ys = [mfp8.linear(x, W8, sw, path=path) for _ in range(3)]
+        torch.cuda.synchronize()
+        assert all(torch.equal(ys[0].view(torch.int16), t.view(torch.int16)) for t in ys[1:])
+
+
+def test_onehot_weights_exact_product():
+    """W rows with one non-zero at column j_n give y[m,n] = dec(x8[m,j_n]) *
+    448 * s_a[m] * s_w[n]: a single product, so even the bf16 rounding is
+    fixed.  Checks the (m, n) mapping and the rescale of each kernel."""
+    M, N, K = 37, 264, 384
+    g = torch.Generator().manual_seed(3)
+    j = torch.randint(0, K, (N,), generator=g)
+    c = torch.randn(N, generator=g) * 3
+    w = torch.zeros(N, K)
+    w[torch.arange(N), j] = c
+    w = w.to(torch.bfloat16).to(DEV)
+    x = W.make_x(M, K, seed=3, device=DEV)
+    W8, sw = mfp8.quantize_weight(w)
+    x8, xs = mfp8.quantize_act(x)
+    xd = oracle.e4m3_decode(u8(x8))
+    wd = oracle.e4m3_decode(u8(W8))
+    expect = (xd[:, j.numpy()] * wd[np.arange(N), j.numpy()][None, :]
+              * f32(xs)[:, None].astype(np.float64) * f32(sw)[None, :].astype(np.float64))
+    expect_bf16 = torch.from_numpy(expect).to(torch.bfloat16)
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK):
+        y = mfp8.linear(x, W8, sw, path=path).cpu()
+        # one product, rounded once: equal unless the kernel's fp32 rounding of
+        # the product lands on the other side of a bf16 tie
+        diff = (y.double() - expect_bf16.double()).abs()
+        ulp = expect_bf16.double().abs() * 2.0 ** -7
+        assert (diff <= ulp).all()
+        assert (y.view(torch.int16) == expect_bf16.view(torch.int16)).float().mean() > 0.99
+
+
+def test_zero_activation_rows_give_zero_outputs():
+    M, N, K = 20, 256, 512
+    x = W.make_x(M, K, seed=4, device=DEV)
+    x[3] = 0
+    x[17] = 0
+    W8, sw = mfp8.quantize_weight(W.make_w(N, K, seed=4, device=DEV))
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK):
+        y = mfp8.linear(x, W8, sw, path=path)
+        torch.cuda.synchronize()
+        assert (y[3] == 0).all() and (y[17] == 0).all()
+
+
+def test_empty_m_is_a_noop():
+    W8, sw = mfp8.quantize_weight(W.make_w(64, 64, seed=0, device=DEV))
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
+    y = mfp8.linear(x, W8, sw)
+    assert y.shape == (0, 64)
+
+
+# ---------------------------------------------------- full-size workloads --
+
+def sampled_rows(M, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    r = set(rng.choice(M, size=min(n, M), replace=False).tolist()) | {0, M - 1}
+    return np.array(sorted(r))
+
+
+@pytest.mark.parametrize("lin", W.LAYER_LINEARS, ids=lambda l: l.name)
+def test_decode_layer_full_size(lin):
+    """Decode: the 7 Linears of one layer at M in {1, 4, 8}, every output."""
+    for M in (1, 4, 8):
+        run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=1, kind="normal")
+
+
+@pytest.mark.parametrize("lin", W.LAYER_LINEARS, ids=lambda l: l.name)
+def test_prefill_layer_full_size_sampled(lin):
+    """Prefill M=2048: every code and scale, sampled output rows."""
+    M = 2048
+    run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=2, kind="rowscale", rows=sampled_rows(M, 32, lin.N))
+
+
+@pytest.mark.parametrize("lin", W.MLP_LINEARS, ids=lambda l: l.name)
+def test_long_video_full_size_sampled(lin):
+    M = 16384
+    run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=3, kind="rowscale", rows=sampled_rows(M, 16, lin.K))
