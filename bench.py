@@ -145,11 +145,12 @@ class Layer:
             s = self.weight_set(mi)
             for i, lin in enumerate(self.lins):
                 ws = self.ws[(M, i)]
-                st = mfp8.mfp8_linear(self.x[(M, i)].data_ptr(), M, lin.K, self.w8[s][i].data_ptr(),
-                                      self.sw[s][i].data_ptr(), lin.N, self.y[(M, i)].data_ptr(),
-                                      ws.data_ptr(), ws.numel(), stream)
+                st = mfp8.mfp8_linear_ex(self.x[(M, i)].data_ptr(), M, lin.K, self.w8[s][i].data_ptr(),
+                                         self.sw[s][i].data_ptr(), lin.N, self.y[(M, i)].data_ptr(),
+                                         ws.data_ptr(), ws.numel(), mfp8.PATH_AUTO, mfp8.FLAG_STATIC_WEIGHTS,
+                                         None, None, stream)
                 if st != mfp8.OK:
-                    raise mfp8.Mfp8Error(st, "mfp8_linear")
+                    raise mfp8.Mfp8Error(st, "mfp8_linear_ex")
 
     def weight_bytes_per_step(self):
         return sum(lin.N * lin.K + 4 * lin.N for lin in self.lins) * len(self.Ms)
@@ -190,42 +191,51 @@ def time_graph(torch, fn, steps, warmup, dist_ctx):
 
 
 def kernel_times(torch, mfp8, layer, reps):
-    """Per-launch CUDA-event times of the GEMM kernel and the quantize
-    kernel, launched one at a time on the current stream."""
-    stream = torch.cuda.current_stream()
-    h = stream.cuda_stream
-    gemm_ms, gemm_bytes, gemm_flops, gemm_n = 0.0, 0, 0, 0
-    quant_ms, quant_bytes, quant_n = 0.0, 0, 0
+    """Per-launch CUDA-event times of the GEMM kernel and of the quantize
+    kernel.  Each launch sits between two event-record nodes of one CUDA
+    graph, so the host's launch latency never shows up as a gap between the
+    events."""
     x8 = {}
     for mi, M in enumerate(layer.Ms):
         for i, lin in enumerate(layer.lins):
             x8[(M, i)] = mfp8.quantize_act(layer.x[(M, i)])
     torch.cuda.synchronize()
-    for _ in range(reps):
-        for mi, M in enumerate(layer.Ms):
+    keys = [(mi, M, i, lin) for mi, M in enumerate(layer.Ms) for i, lin in enumerate(layer.lins)]
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in keys]
+
+    def body(h):
+        for (mi, M, i, lin), e in zip(keys, ev):
             s = layer.weight_set(mi)
-            for i, lin in enumerate(layer.lins):
-                q8, qs = x8[(M, i)]
-                e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-                e[0].record(stream)
-                st = mfp8.mfp8_quantize_act(layer.x[(M, i)].data_ptr(), M, lin.K, q8.data_ptr(), qs.data_ptr(), h)
-                e[1].record(stream)
-                e[2].record(stream)
-                st2 = mfp8.mfp8_gemm(q8.data_ptr(), qs.data_ptr(), M, lin.K, layer.w8[s][i].data_ptr(),
-                                     layer.sw[s][i].data_ptr(), lin.N, layer.y[(M, i)].data_ptr(), 0, h)
-                e[3].record(stream)
-                if st != mfp8.OK or st2 != mfp8.OK:
-                    raise mfp8.Mfp8Error(st or st2, "kernel timing")
-                torch.cuda.synchronize()
-                quant_ms += e[0].elapsed_time(e[1])
-                gemm_ms += e[2].elapsed_time(e[3])
-                quant_bytes += 3 * M * lin.K + 4 * M
-                gemm_bytes += lin.N * lin.K + 4 * lin.N + M * lin.K + 4 * M + 2 * M * lin.N
-                gemm_flops += 2 * M * lin.N * lin.K
-                gemm_n += 1
-                quant_n += 1
-    return dict(gemm_ms=gemm_ms, gemm_bytes=gemm_bytes, gemm_flops=gemm_flops, gemm_n=gemm_n,
-                quant_ms=quant_ms, quant_bytes=quant_bytes, quant_n=quant_n)
+            q8, qs = x8[(M, i)]
+            e[0].record()
+            st = mfp8.mfp8_quantize_act(layer.x[(M, i)].data_ptr(), M, lin.K, q8.data_ptr(), qs.data_ptr(), h)
+            e[1].record()
+            e[2].record()
+            st2 = mfp8.mfp8_gemm(q8.data_ptr(), qs.data_ptr(), M, lin.K, layer.w8[s][i].data_ptr(),
+                                 layer.sw[s][i].data_ptr(), lin.N, layer.y[(M, i)].data_ptr(), 0, h)
+            e[3].record()
+            if st != mfp8.OK or st2 != mfp8.OK:
+                raise mfp8.Mfp8Error(st or st2, "kernel timing")
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        body(torch.cuda.current_stream().cuda_stream)
+    out = dict(gemm_ms=0.0, gemm_bytes=0, gemm_flops=0, gemm_n=0, quant_ms=0.0, quant_bytes=0, quant_n=0)
+    g.replay()
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        g.replay()
+        torch.cuda.synchronize()
+        for (mi, M, i, lin), e in zip(keys, ev):
+            out["quant_ms"] += e[0].elapsed_time(e[1])
+            out["gemm_ms"] += e[2].elapsed_time(e[3])
+            out["quant_bytes"] += 3 * M * lin.K + 4 * M
+            out["gemm_bytes"] += lin.N * lin.K + 4 * lin.N + M * lin.K + 4 * M + 2 * M * lin.N
+            out["gemm_flops"] += 2 * M * lin.N * lin.K
+            out["gemm_n"] += 1
+            out["quant_n"] += 1
+    del g
+    return out
 
 
 def e2e_time(torch, mfp8, layer, steps, warmup, dist_ctx):

@@ -15,6 +15,8 @@
 #include "quant.cuh"
 #include "gemm_tiled.cuh"
 #include "gemm_splitk.cuh"
+#include "gemm_decode.cuh"
+#include "gemm_pair.cuh"
 
 namespace mfp8 {
 namespace {
@@ -94,19 +96,30 @@ mfp8_status launch_status() {
 
 // ------------------------------------------------------------- quantize --
 
-mfp8_status quantize_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
+template <bool EARLY_TRIGGER>
+mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
     if (R == 0) return MFP8_OK;
     const int64_t nvec = K / 8;
     const uint4* x = static_cast<const uint4*>(X);
     uint2* q = static_cast<uint2*>(Q);
     const dim3 grid(static_cast<unsigned>(R)), block(kQuantThreads);
-    if (nvec <= 256) quant_rows_reg_kernel<1><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 512) quant_rows_reg_kernel<2><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 1024) quant_rows_reg_kernel<4><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 1536) quant_rows_reg_kernel<6><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 2048) quant_rows_reg_kernel<8><<<grid, block, 0, stream>>>(x, K, q, S);
-    else quant_rows_loop_kernel<<<grid, block, 0, stream>>>(x, K, q, S);
+    if (nvec <= 256) quant_rows_reg_kernel<1, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 512) quant_rows_reg_kernel<2, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 1024) quant_rows_reg_kernel<4, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 1536) quant_rows_reg_kernel<6, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
+    else if (nvec <= 2048) quant_rows_reg_kernel<8, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
+    else quant_rows_loop_kernel<EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
     return launch_status();
+}
+
+// Activations: the GEMM launched next may start its prologue early.
+mfp8_status quantize_act_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
+    return quantize_rows_t<true>(X, R, K, Q, S, stream);
+}
+
+// Weights: no early start for whatever follows.
+mfp8_status quantize_weight_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
+    return quantize_rows_t<false>(X, R, K, Q, S, stream);
 }
 
 mfp8_status check_quant_args(const void* X, int64_t R, int64_t K, const void* Q, const float* S) {
@@ -171,6 +184,48 @@ mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K,
     return MFP8_OK;
 }
 
+int64_t splitk_cluster(int64_t tiles, int64_t kb_total, int per_sm, const DeviceInfo& info);
+
+#ifndef MFP8_PAIR_STAGES
+#define MFP8_PAIR_STAGES 6
+#endif
+
+mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+                        int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info, cudaStream_t stream) {
+    using L = pair::Layout<MFP8_PAIR_STAGES>;
+    auto kern = pair::gemm_pair_kernel<MFP8_PAIR_STAGES>;
+    static bool attr_done[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
+    if (st != MFP8_OK) return st;
+    CUtensorMap tmX, tmW;
+    if ((st = make_map_u8(&tmX, X8, M, K, pair::HALF)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmW, W8, N, K, pair::HALF)) != MFP8_OK) return st;
+    const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN);
+    const int64_t max_pairs = info.sm_count / 2;
+    const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(2 * pairs));
+    cfg.blockDim = dim3(pair::kThreads);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
+                           int(K)) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
 template <int MP, int STAGES>
 mfp8_status launch_splitk_mp(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
                              const float* s_w, int64_t N, void* Y, bool dependent, int dev,
@@ -189,10 +244,7 @@ mfp8_status launch_splitk_mp(const void* X8, const float* s_a, int64_t M, int64_
     // Split K so that the grid covers the SMs about twice (two CTAs fit per
     // SM for the small MP), without giving any CTA an empty K range.
     const int per_sm = (2 * L::SMEM_BYTES <= 227 * 1024) ? 2 : 1;
-    int64_t S = (int64_t(info.sm_count) * per_sm + tiles - 1) / tiles;
-    if (S > splitk::kMaxCluster) S = splitk::kMaxCluster;
-    if (S > kb_total) S = kb_total;
-    if (S < 1) S = 1;
+    const int64_t S = splitk_cluster(tiles, kb_total, per_sm, info);
     if (tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
 
     cudaLaunchConfig_t cfg = {};
@@ -227,10 +279,96 @@ mfp8_status launch_splitk(const void* X8, const float* s_a, int64_t M, int64_t K
     return MFP8_ERR_UNSUPPORTED_SHAPE;
 }
 
+constexpr int64_t kFusedMaxM = 64;
+
+// Cluster size (K-split) for the weight-streaming kernels: enough CTAs to
+// cover every SM `per_sm` times, at most 8 (portable cluster size), and no
+// CTA with an empty K range.
+int64_t splitk_cluster(int64_t tiles, int64_t kb_total, int per_sm, const DeviceInfo& info) {
+    int64_t S = (int64_t(info.sm_count) * per_sm + tiles - 1) / tiles;
+    if (S > 8) S = 8;
+    if (S > kb_total) S = kb_total;
+    if (S < 1) S = 1;
+    return S;
+}
+
+// Decode kernel sizing: CTAs per SM the grid aims to fill, at most.
+#ifndef MFP8_DECODE_CTAS_PER_SM
+#define MFP8_DECODE_CTAS_PER_SM 2
+#endif
+#ifndef MFP8_DECODE_STAGES
+#define MFP8_DECODE_STAGES 4
+#endif
+
+template <int MP, int ITEMS>
+mfp8_status launch_decode_mp(const void* X, int64_t M, int64_t K, const void* W8, const float* s_w, int64_t N,
+                             void* Y, bool weights_static, void* x8_out, float* sa_out, int dev,
+                             const DeviceInfo& info, cudaStream_t stream) {
+    constexpr int STAGES = MFP8_DECODE_STAGES;
+    using L = decode::Layout<MP, STAGES>;
+    auto kern = decode::gemm_decode_kernel<MP, STAGES, ITEMS>;
+    const int64_t tiles = (N + decode::BW - 1) / decode::BW;
+    const int64_t kb_total = (K + decode::BK - 1) / decode::BK;
+    if (tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    // K-split: fill the SMs without a second wave, then split further if one
+    // CTA's slice of X would not fit in its registers.
+    int64_t S = (int64_t(info.sm_count) * MFP8_DECODE_CTAS_PER_SM) / tiles;
+    if (S < 1) S = 1;
+    if (S > decode::kMaxCluster) S = decode::kMaxCluster;
+    if (S > kb_total) S = kb_total;
+    auto nkb_cap_of = [&](int64_t s) { return (kb_total + s - 1) / s; };
+    while (S < decode::kMaxCluster && S < kb_total &&
+           M * nkb_cap_of(S) * decode::kGroupsPerBlock > int64_t(ITEMS) * decode::kThreads)
+        ++S;
+    const int64_t nkb_cap = nkb_cap_of(S);
+    if (M * nkb_cap * decode::kGroupsPerBlock > int64_t(ITEMS) * decode::kThreads) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    const int smem = L::smem_bytes(int(nkb_cap));
+    if (smem > 227 * 1024) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    static bool attr_done[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, 227 * 1024, dev, attr_done);
+    if (st != MFP8_OK) return st;
+    CUtensorMap tmW;
+    if ((st = make_map_u8(&tmW, W8, N, K, decode::BW)) != MFP8_OK) return st;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(S), unsigned(tiles));
+    cfg.blockDim = dim3(decode::kThreads);
+    cfg.dynamicSmemBytes = size_t(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tmW, static_cast<const __nv_bfloat16*>(X), s_w,
+                           static_cast<__nv_bfloat16*>(Y), int(M), int(N), int(K), int(nkb_cap),
+                           weights_static ? 1 : 0, static_cast<uint8_t*>(x8_out), sa_out) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
+mfp8_status launch_fused(const void* X, int64_t M, int64_t K, const void* W8, const float* s_w, int64_t N,
+                         void* Y, bool weights_static, void* x8_out, float* sa_out, int dev,
+                         const DeviceInfo& info, cudaStream_t stream) {
+    if (M <= 16)
+        return launch_decode_mp<16, 16>(X, M, K, W8, s_w, N, Y, weights_static, x8_out, sa_out, dev, info, stream);
+    if (M <= 32)
+        return launch_decode_mp<32, 24>(X, M, K, W8, s_w, N, Y, weights_static, x8_out, sa_out, dev, info, stream);
+    if (M <= 64)
+        return launch_decode_mp<64, 24>(X, M, K, W8, s_w, N, Y, weights_static, x8_out, sa_out, dev, info, stream);
+    return MFP8_ERR_UNSUPPORTED_SHAPE;
+}
+
 int choose_path(int64_t M, int64_t N, int64_t K) {
     (void)N;
     (void)K;
-    return M <= 64 ? MFP8_PATH_SPLITK : MFP8_PATH_TILED;
+    return M <= kFusedMaxM ? MFP8_PATH_SPLITK : MFP8_PATH_TILED;
 }
 
 mfp8_status check_gemm_args(int64_t M, int64_t N, int64_t K, const void* W8, const float* s_w, const void* Y) {
@@ -253,6 +391,7 @@ mfp8_status run_gemm(const void* X8, const float* s_a, int64_t M, int64_t K, con
     // The tiled kernel takes M, N, K as 32-bit; tile counts must fit too.
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (path == MFP8_PATH_TILED) return launch_tiled(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    if (path == MFP8_PATH_PAIR) return launch_pair(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
     if (path == MFP8_PATH_SPLITK) {
         if (M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
         return launch_splitk(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
@@ -296,7 +435,7 @@ mfp8_status mfp8_quantize_weight(const void* W_bf16, int64_t N, int64_t K, void*
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
-    return quantize_rows(W_bf16, N, K, W_fp8, w_scale, static_cast<cudaStream_t>(stream));
+    return quantize_weight_rows(W_bf16, N, K, W_fp8, w_scale, static_cast<cudaStream_t>(stream));
 }
 
 mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K, void* X_fp8, float* x_scale,
@@ -306,7 +445,7 @@ mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K, void* X_
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
-    return quantize_rows(X_bf16, M, K, X_fp8, x_scale, static_cast<cudaStream_t>(stream));
+    return quantize_act_rows(X_bf16, M, K, X_fp8, x_scale, static_cast<cudaStream_t>(stream));
 }
 
 size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -316,54 +455,73 @@ size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 
 mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
                            int64_t N, void* Y_bf16, void* workspace, size_t workspace_bytes_given, int path,
-                           void* X_fp8_out, float* x_scale_out, void* stream) {
+                           int flags, void* X_fp8_out, float* x_scale_out, void* stream) {
     mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
     if (st != MFP8_OK) return st;
-    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_SPLITK) return MFP8_ERR_INVALID_ARG;
+    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_PAIR) return MFP8_ERR_INVALID_ARG;
+    if ((flags & ~MFP8_FLAG_STATIC_WEIGHTS) != 0) return MFP8_ERR_INVALID_ARG;
     if (path == MFP8_PATH_SPLITK && M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_bf16) return MFP8_ERR_INVALID_ARG;
     if (!aligned16(X_bf16)) return MFP8_ERR_MISALIGNED;
     if ((X_fp8_out == nullptr) != (x_scale_out == nullptr)) return MFP8_ERR_INVALID_ARG;
     if (ranges_overlap(X_bf16, size_t(M * K * 2), Y_bf16, size_t(M * N * 2))) return MFP8_ERR_INVALID_ARG;
-
-    void* X8;
-    float* s_a;
     if (X_fp8_out) {
         if (!aligned16(X_fp8_out) || !aligned16(x_scale_out)) return MFP8_ERR_MISALIGNED;
-        X8 = X_fp8_out;
-        s_a = x_scale_out;
-    } else {
+        if ((st = check_quant_args(X_bf16, M, K, X_fp8_out, x_scale_out)) != MFP8_OK) return st;
+        if (ranges_overlap(X_fp8_out, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
+            ranges_overlap(x_scale_out, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
+            return MFP8_ERR_INVALID_ARG;
+    }
+    if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
+    const bool fused = path == MFP8_PATH_SPLITK && M <= kFusedMaxM;
+
+    void* X8 = X_fp8_out;
+    float* s_a = x_scale_out;
+    if (!fused && !X8) {
         const size_t need = workspace_bytes(M, K);
         if (!workspace || workspace_bytes_given < need) return MFP8_ERR_WORKSPACE;
         if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
         X8 = workspace;
         s_a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(size_t(M) * size_t(K), 256));
+        if ((st = check_quant_args(X_bf16, M, K, X8, s_a)) != MFP8_OK) return st;
+        if (ranges_overlap(X8, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
+            ranges_overlap(s_a, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
+            return MFP8_ERR_INVALID_ARG;
     }
-    if ((st = check_quant_args(X_bf16, M, K, X8, s_a)) != MFP8_OK) return st;
-    if (ranges_overlap(X8, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
-        ranges_overlap(s_a, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
-        return MFP8_ERR_INVALID_ARG;
 
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((st = quantize_rows(X_bf16, M, K, X8, s_a, s)) != MFP8_OK) return st;
+    if (fused) {
+        st = launch_fused(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, (flags & MFP8_FLAG_STATIC_WEIGHTS) != 0,
+                          X_fp8_out, x_scale_out, dev, info, s);
+        if (st != MFP8_ERR_UNSUPPORTED_SHAPE) return st;
+        // Too large for the on-chip codes: quantize pass + unfused split-K.
+        if (!X8) {
+            const size_t need = workspace_bytes(M, K);
+            if (!workspace || workspace_bytes_given < need) return MFP8_ERR_WORKSPACE;
+            if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
+            X8 = workspace;
+            s_a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(size_t(M) * size_t(K), 256));
+        }
+    }
+    if ((st = quantize_act_rows(X_bf16, M, K, X8, s_a, s)) != MFP8_OK) return st;
     return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, path, /*dependent=*/true, dev, info, s);
 }
 
 mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
                         int64_t N, void* Y_bf16, void* workspace, size_t workspace_bytes_given, void* stream) {
     return mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes_given,
-                          MFP8_PATH_AUTO, nullptr, nullptr, stream);
+                          MFP8_PATH_AUTO, 0, nullptr, nullptr, stream);
 }
 
 mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K, const void* W_fp8,
                       const float* w_scale, int64_t N, void* Y_bf16, int path, void* stream) {
     mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
     if (st != MFP8_OK) return st;
-    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_SPLITK) return MFP8_ERR_INVALID_ARG;
+    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_PAIR) return MFP8_ERR_INVALID_ARG;
     if (path == MFP8_PATH_SPLITK && M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_fp8 || !x_scale) return MFP8_ERR_INVALID_ARG;

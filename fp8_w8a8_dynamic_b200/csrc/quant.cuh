@@ -79,11 +79,15 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red /* [
 
 // One block per row; the row (K/8 16-byte vectors) lives in registers,
 // VPT vectors per thread.  Requires K/8 <= VPT * 256.
-template <int VPT>
+// EARLY_TRIGGER lets the next kernel on the stream start its prologue at
+// once (activation quantization: the GEMM that follows waits for the codes
+// before reading them).  The weight quantizer leaves it off, so nothing that
+// follows starts before the weight codes are complete.
+template <int VPT, bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
                       float* __restrict__ S) {
-    grid_launch_dependents();
+    if (EARLY_TRIGGER) grid_launch_dependents();
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = K >> 3;
@@ -112,10 +116,11 @@ quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict_
 }
 
 // Any K: two passes over the row (the second one is served by L2).
+template <bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_loop_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
                        float* __restrict__ S) {
-    grid_launch_dependents();
+    if (EARLY_TRIGGER) grid_launch_dependents();
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = K >> 3;

@@ -24,6 +24,9 @@ ERR_DEVICE = 7
 PATH_AUTO = 0
 PATH_TILED = 1
 PATH_SPLITK = 2
+PATH_PAIR = 3
+
+FLAG_STATIC_WEIGHTS = 1
 
 
 class Mfp8Error(RuntimeError):
@@ -48,7 +51,7 @@ def lib():
             "mfp8_quantize_act": (i32, [P, i64, i64, P, P, P]),
             "mfp8_linear_workspace_bytes": (sz, [i64, i64, i64]),
             "mfp8_linear": (i32, [P, i64, i64, P, P, i64, P, P, sz, P]),
-            "mfp8_linear_ex": (i32, [P, i64, i64, P, P, i64, P, P, sz, i32, P, P, P]),
+            "mfp8_linear_ex": (i32, [P, i64, i64, P, P, i64, P, P, sz, i32, i32, P, P, P]),
             "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, i32, P]),
             "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
             "mfp8_debug_bounded_wait": (i32, [i64, P]),
@@ -82,10 +85,10 @@ def mfp8_linear(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_by
     return lib().mfp8_linear(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, stream)
 
 
-def mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, path,
+def mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, path, flags,
                    X_fp8_out, x_scale_out, stream=0):
     return lib().mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes,
-                                path, X_fp8_out, x_scale_out, stream)
+                                path, flags, X_fp8_out, x_scale_out, stream)
 
 
 def mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path=PATH_AUTO, stream=0):
@@ -159,7 +162,7 @@ def workspace_for(M, N, K, device):
 
 
 def linear(X, W8, w_scale, out=None, workspace=None, path=PATH_AUTO, x8_out=None, xs_out=None,
-           stream=None):
+           flags=0, stream=None):
     """Y = FP8_DYNAMIC Linear(X) with pre-quantized weights.  X bf16 [M, K]."""
     import torch
     M, K = X.shape
@@ -170,7 +173,7 @@ def linear(X, W8, w_scale, out=None, workspace=None, path=PATH_AUTO, x8_out=None
         workspace = workspace_for(M, N, K, X.device)
     ws_bytes = workspace.numel() if workspace is not None else 0
     _check(mfp8_linear_ex(_ptr(X), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), _ptr(workspace),
-                          ws_bytes, path, _ptr(x8_out), _ptr(xs_out), _stream_handle(stream)),
+                          ws_bytes, path, flags, _ptr(x8_out), _ptr(xs_out), _stream_handle(stream)),
            "mfp8_linear_ex")
     return out
 

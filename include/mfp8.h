@@ -85,9 +85,11 @@ MFP8_API mfp8_status mfp8_quantize_weight(const void* W_bf16, int64_t N, int64_t
 MFP8_API mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K,
                               void* X_fp8, float* x_scale, void* stream);
 
-/* Bytes of device workspace mfp8_linear needs for these sizes (0 when the
- * chosen kernel quantizes X on chip).  Never fails; returns 0 for invalid
- * sizes (mfp8_linear then reports the error). */
+/* Bytes of device workspace that is enough for mfp8_linear and for every
+ * kernel choice of mfp8_linear_ex at these sizes (the activation codes and
+ * scales of the separate quantize pass).  The decode-sized kernel (M <= 64)
+ * quantizes on chip and ignores the workspace.  Never fails; returns 0 for
+ * invalid sizes (mfp8_linear then reports the error). */
 MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* The FP8_DYNAMIC Linear: Y = bf16(  (Xq . Wq^T) * x_scale (x) w_scale  ).
@@ -98,9 +100,10 @@ MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *            mfp8_quantize_weight, read only.
  *   Y_bf16   [M, N] bf16, written.  Must not overlap any input.
  *   workspace / workspace_bytes: device scratch of at least
- *            mfp8_linear_workspace_bytes(M, N, K) bytes (may be NULL when
- *            that is 0).  Its contents on entry do not matter; they are
- *            garbage on exit.  Concurrent calls need separate workspaces.
+ *            mfp8_linear_workspace_bytes(M, N, K) bytes; may be NULL for
+ *            M <= 64, where the kernel keeps the activation codes on chip.
+ *            Its contents on entry do not matter; they are garbage on exit.
+ *            Concurrent calls need separate workspaces.
  * The activation quantization (per-token scale + e4m3 codes) happens inside
  * this call: its codes and scales are bit-identical to mfp8_quantize_act.
  * Outputs are within |y - y_ref| <= 2^-7 |y_ref| + 1e-5 * sum_k |a_k w_k| s_a s_w
@@ -114,19 +117,32 @@ MFP8_API mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K,
 typedef enum {
     MFP8_PATH_AUTO = 0,   /* what mfp8_linear does: chosen from M, N, K */
     MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
-    MFP8_PATH_SPLITK = 2  /* weight-streaming split-K tcgen05 GEMM (M <= 128) */
+    MFP8_PATH_SPLITK = 2, /* weight-streaming split-K tcgen05 GEMM (M <= 128); M <= 64 fuses the quantize step */
+    MFP8_PATH_PAIR = 3    /* quantize pass, then the 256 x 256-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
 } mfp8_path;
 
-/* mfp8_linear with an explicit kernel choice, and optional copies of the
- * activation codes and scales it computed (X_fp8_out [M, K] and
+/* Flags for mfp8_linear_ex. */
+#define MFP8_FLAG_STATIC_WEIGHTS 1
+/* The caller promises that W_fp8 and w_scale are not written by any work
+ * still pending on `stream` (they are a model's static weights, quantized
+ * once).  The decode-sized kernel may then start streaming the weights while
+ * the previous kernel on the stream is still finishing (programmatic
+ * dependent launch); the activations are still read only after that kernel
+ * has completed.  Without the flag every input is read after it. */
+
+/* mfp8_linear with an explicit kernel choice, flags, and optional copies of
+ * the activation codes and scales it computed (X_fp8_out [M, K] and
  * x_scale_out [M]; pass NULL for none).  Used to test each kernel on the
- * same shapes and to check that the activation bytes of every path are
- * bit-identical to mfp8_quantize_act.  Returns MFP8_ERR_UNSUPPORTED_SHAPE if
- * the chosen kernel cannot take these sizes. */
+ * same shapes, to check that the activation bytes of every path are
+ * bit-identical to mfp8_quantize_act, and by callers with static weights.
+ * path MFP8_PATH_SPLITK with M <= 64 quantizes X inside the GEMM kernel (one
+ * launch); with 64 < M <= 128 it runs the quantize pass first.  Returns
+ * MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel cannot take these sizes,
+ * MFP8_ERR_INVALID_ARG for an unknown path or flag. */
 MFP8_API mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K,
                            const void* W_fp8, const float* w_scale, int64_t N,
                            void* Y_bf16, void* workspace, size_t workspace_bytes,
-                           int path, void* X_fp8_out, float* x_scale_out,
+                           int path, int flags, void* X_fp8_out, float* x_scale_out,
                            void* stream);
 
 /* The contraction and epilogue alone, on activations already quantized by

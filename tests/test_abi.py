@@ -78,16 +78,19 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     def call(**kw):
         a = {**args, **kw}
         return L(a["X"], a["M"], a["K"], a["W"], a["sw"], a["N"], a["Y"], a["ws"], a["wsb"],
-                 kw.get("path", 0), kw.get("x8", None), kw.get("xs", None), None)
+                 kw.get("path", 0), kw.get("flags", 0), kw.get("x8", None), kw.get("xs", None), None)
 
     assert call(N=12) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(N=0) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(K=8) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(W=None) == mfp8.ERR_INVALID_ARG
     assert call(Y=FAKE * 4 + 4) == mfp8.ERR_MISALIGNED
-    assert call(ws=None) == mfp8.ERR_WORKSPACE
-    assert call(wsb=100) == mfp8.ERR_WORKSPACE
+    assert call(M=65, ws=None) == mfp8.ERR_WORKSPACE  # quantize pass needs the workspace
+    assert call(M=65, wsb=100) == mfp8.ERR_WORKSPACE
+    assert call(M=4, path=mfp8.PATH_TILED, ws=None) == mfp8.ERR_WORKSPACE
+    assert call(flags=2) == mfp8.ERR_INVALID_ARG
     assert call(path=7) == mfp8.ERR_INVALID_ARG
+    assert call(path=4) == mfp8.ERR_INVALID_ARG
     assert call(path=mfp8.PATH_SPLITK, M=129) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
     assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X

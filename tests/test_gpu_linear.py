@@ -16,13 +16,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def run_case(M, N, K, path, seed=0, kind="normal", rows=None, check_codes=True):
+def run_case(M, N, K, path, seed=0, kind="normal", rows=None, check_codes=True, flags=0):
     x = W.make_x(M, K, seed=seed, stream=M, kind=kind, device=DEV)
     w = W.make_w(N, K, seed=seed, stream=N, device=DEV)
     W8, sw = mfp8.quantize_weight(w)
     x8 = torch.empty((M, K), dtype=torch.uint8, device=DEV)
     xs = torch.empty((M,), dtype=torch.float32, device=DEV)
-    y = mfp8.linear(x, W8, sw, path=path, x8_out=x8, xs_out=xs)
+    y = mfp8.linear(x, W8, sw, path=path, x8_out=x8, xs_out=xs, flags=flags)
     torch.cuda.synchronize()
     assert mfp8.device_status() == mfp8.OK
     w8_h, sw_h = u8(W8), f32(sw)
@@ -45,27 +45,59 @@ TILED_ONLY = [(130, 264, 384), (300, 520, 1040), (256, 1024, 4096), (1000, 2056,
 
 
 @pytest.mark.parametrize("M,N,K", SMALL)
-@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_AUTO])
+@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR, mfp8.PATH_AUTO])
 def test_linear_small(M, N, K, path):
     run_case(M, N, K, path, seed=M * 7 + N)
 
 
-@pytest.mark.parametrize("M,N,K", TILED_ONLY)
-def test_linear_tiled_ragged(M, N, K):
-    run_case(M, N, K, mfp8.PATH_TILED, seed=11, kind="rowscale")
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (8, 12288, 4096), (16, 4096, 12288), (64, 1024, 4096),
+                                   (33, 264, 400)])
+def test_linear_static_weights_flag(M, N, K):
+    run_case(M, N, K, mfp8.PATH_AUTO, seed=M + 3, flags=mfp8.FLAG_STATIC_WEIGHTS)
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 4096, 4096), (130, 264, 384), (64, 1024, 4096)])
-def test_gemm_entry_point_matches_linear(M, N, K):
-    x, W8, sw, y = run_case(M, N, K, mfp8.PATH_AUTO, seed=5, check_codes=False)
+def test_linear_without_codes_out_matches_with():
+    """The decode kernel writes the optional code copy only from its first
+    cluster; the outputs must not depend on whether it is asked for."""
+    for M in (1, 7, 64, 100):
+        x = W.make_x(M, 4096, seed=9, device=DEV)
+        W8, sw = mfp8.quantize_weight(W.make_w(1024, 4096, seed=9, device=DEV))
+        y1 = mfp8.linear(x, W8, sw)
+        x8 = torch.empty((M, 4096), dtype=torch.uint8, device=DEV)
+        xs = torch.empty((M,), dtype=torch.float32, device=DEV)
+        y2 = mfp8.linear(x, W8, sw, x8_out=x8, xs_out=xs)
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K", TILED_ONLY + [(513, 776, 1024), (2048, 1024, 4096)])
+@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_PAIR])
+def test_linear_tiled_ragged(M, N, K, path):
+    run_case(M, N, K, path, seed=11, kind="rowscale")
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 4096, 4096), (130, 264, 384), (64, 1024, 4096), (100, 512, 1024)])
+@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR])
+def test_gemm_entry_point(M, N, K, path):
+    """mfp8_gemm on codes from mfp8_quantize_act: within tolerance of the
+    oracle, and bit-identical to mfp8_linear on the same kernel when that
+    kernel is the same (tiled, or split-K above the fused size)."""
+    if path == mfp8.PATH_SPLITK and M > 128:
+        pytest.skip("split-K takes M <= 128")
+    x = W.make_x(M, K, seed=5, device=DEV)
+    W8, sw = mfp8.quantize_weight(W.make_w(N, K, seed=5, device=DEV))
     x8, xs = mfp8.quantize_act(x)
-    y2 = mfp8.gemm(x8, xs, W8, sw)
+    y2 = mfp8.gemm(x8, xs, W8, sw, path=path)
     torch.cuda.synchronize()
-    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    assert_linear_parity(y2, u8(x8), f32(xs), u8(W8), f32(sw), what="mfp8_gemm")
+    if path != mfp8.PATH_SPLITK or M > 64:
+        y = mfp8.linear(x, W8, sw, path=path)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
 
 
 def test_deterministic():
-    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK):
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR):
         x = W.make_x(16, 4096, seed=0, device=DEV)
         W8, sw = mfp8.quantize_weight(W.make_w(4096, 4096, seed=0, device=DEV))
         ys = [mfp8.linear(x, W8, sw, path=path) for _ in range(3)]
@@ -92,7 +124,7 @@ def test_onehot_weights_exact_product():
     expect = (xd[:, j.numpy()] * wd[np.arange(N), j.numpy()][None, :]
               * f32(xs)[:, None].astype(np.float64) * f32(sw)[None, :].astype(np.float64))
     expect_bf16 = torch.from_numpy(expect).to(torch.bfloat16)
-    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK):
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR):
         y = mfp8.linear(x, W8, sw, path=path).cpu()
         # one product, rounded once: equal unless the kernel's fp32 rounding of
         # the product lands on the other side of a bf16 tie
@@ -108,7 +140,7 @@ def test_zero_activation_rows_give_zero_outputs():
     x[3] = 0
     x[17] = 0
     W8, sw = mfp8.quantize_weight(W.make_w(N, K, seed=4, device=DEV))
-    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK):
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR):
         y = mfp8.linear(x, W8, sw, path=path)
         torch.cuda.synchronize()
         assert (y[3] == 0).all() and (y[17] == 0).all()
