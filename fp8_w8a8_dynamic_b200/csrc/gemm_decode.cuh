@@ -13,7 +13,8 @@
 //      waiting on the previous kernel when the caller declared the weights
 //      static);
 //   2. every thread loads its share of this CTA's K-slice of X (BF16) into
-//      registers and folds it into a per-row absmax in shared memory;
+//      registers (a large slice's remainder is read again in step 4) and
+//      folds it into a per-row absmax in shared memory;
 //   3. the per-row slice maxima are pushed to every CTA of the cluster with
 //      st.async (remote store + transaction count on the receiver's
 //      mbarrier); each CTA then holds all S maxima of every row, takes the
@@ -73,19 +74,21 @@ struct Layout {
     static constexpr int TMEM_COLS = MP < 32 ? 32 : MP;
     static constexpr int NUM_BARS = 2 * STAGES + 4;  // full, empty, tfull, drain, xbar, rbar
     // [X tiles: nkb_cap * X_TILE][recv: 128 rows * MP floats][pmax_all: kMaxCluster * MP]
-    // [pmax_local: MP][sa: MP][bars][tmem holder, abort flag]
+    // [pmax_local: MP][sa: MP][1/sa: MP][s_w of my channels: 128][bars][tmem holder, abort flag]
     __host__ __device__ static int x_off() { return RING_BYTES; }
     __host__ __device__ static int recv_off(int nkb_cap) { return x_off() + nkb_cap * X_TILE; }
     // S * ceil(128 / S) <= 128 + S rows of partials
     __host__ __device__ static int pmax_all_off(int nkb_cap) { return recv_off(nkb_cap) + (BW + kMaxCluster) * MP * 4; }
     __host__ __device__ static int pmax_off(int nkb_cap) { return pmax_all_off(nkb_cap) + kMaxCluster * MP * 4; }
     __host__ __device__ static int sa_off(int nkb_cap) { return pmax_off(nkb_cap) + MP * 4; }
-    __host__ __device__ static int bar_off(int nkb_cap) { return (sa_off(nkb_cap) + MP * 4 + 7) & ~7; }
+    __host__ __device__ static int sw_off(int nkb_cap) { return sa_off(nkb_cap) + 2 * MP * 4; }
+    __host__ __device__ static int bar_off(int nkb_cap) { return (sw_off(nkb_cap) + BW * 4 + 7) & ~7; }
     __host__ __device__ static int misc_off(int nkb_cap) { return bar_off(nkb_cap) + NUM_BARS * 8; }
     __host__ __device__ static int smem_bytes(int nkb_cap) { return misc_off(nkb_cap) + 16 + 1024; }
 };
 
-// ITEMS: 8-element groups of X held per thread (>= M * nkb_cap * 16 / 192).
+// ITEMS: 8-element groups of X a thread keeps in registers between the
+// absmax pass and the codes pass; groups beyond ITEMS * 192 are read twice.
 template <int MP, int STAGES, int ITEMS>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16* __restrict__ X,
@@ -102,6 +105,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16*
     uint32_t* pmax_all = reinterpret_cast<uint32_t*>(smem + L::pmax_all_off(nkb_cap));  // [S][MP]
     uint32_t* pmax = reinterpret_cast<uint32_t*>(smem + L::pmax_off(nkb_cap));          // [MP]
     float* sa_sm = reinterpret_cast<float*>(smem + L::sa_off(nkb_cap));                  // [MP]
+    float* ra_sm = sa_sm + MP;                                                            // [MP] 1/s
+    float* sw_sm = reinterpret_cast<float*>(smem + L::sw_off(nkb_cap));                  // [my_rows]
     const uint32_t bar0 = sbase + L::bar_off(nkb_cap);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -167,8 +172,17 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16*
             tma_load_2d_hint(sW + i * L::W_BYTES, &tmW, full_bar(i), (kb_begin + i) * BK, n0, policy_w);
         }
     }
+    // The channel scales this CTA applies, fetched while the rest proceeds.
+    if (weights_static && threadIdx.x >= 64 && threadIdx.x < 64 + my_rows) {
+        const int n = n0 + c0 + int(threadIdx.x) - 64;
+        sw_sm[threadIdx.x - 64] = n < N ? __ldg(s_w + n) : 0.0f;
+    }
     grid_dependency_wait();  // X comes from earlier work on the stream
     grid_launch_dependents();
+    if (!weights_static && threadIdx.x >= 64 && threadIdx.x < 64 + my_rows) {
+        const int n = n0 + c0 + int(threadIdx.x) - 64;
+        sw_sm[threadIdx.x - 64] = n < N ? __ldg(s_w + n) : 0.0f;
+    }
 
     // 2. This CTA's K-slice of X into registers; per-row slice absmax.
     const int groups_per_row = nkb * kGroupsPerBlock;
@@ -197,6 +211,22 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16*
                 }
             }
         }
+        // Items beyond the register cache (large slices): max only; the
+        // codes pass reads them again (L2-resident by then).
+        for (int e = int(threadIdx.x) + ITEMS * kThreads; e < items; e += kThreads) {
+            const int m = e / groups_per_row;
+            const int k = k_lo + (e % groups_per_row) * 8;
+            if (k < K) {
+                const uint32_t a = absmax_bits_u4(__ldg(reinterpret_cast<const uint4*>(X + int64_t(m) * K + k)), 0u);
+                const uint32_t a16 = max(a & 0xffffu, a >> 16);
+                if (m != run_row) {
+                    if (run_row >= 0) atomicMax(pmax + run_row, run_max);
+                    run_row = m;
+                    run_max = 0;
+                }
+                run_max = max(run_max, a16);
+            }
+        }
         if (run_row >= 0) atomicMax(pmax + run_row, run_max);
     }
     __syncthreads();
@@ -216,6 +246,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16*
             for (uint32_t p = 0; p < S; ++p) amax = max(amax, pmax_all[p * MP + m]);
             const float s = scale_from_absmax_bits(amax);
             sa_sm[m] = s;
+            ra_sm[m] = __frcp_rn(s);
             if (sa_out && blockIdx.y == 0 && rank == 0 && m < M) sa_out[m] = s;
         }
     }
@@ -243,12 +274,25 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16*
                 const int k = k_lo + g * 8;
                 uint2 q = make_uint2(0u, 0u);
                 if (k < K) {
-                    q = quantize8(xv[i], sa_sm[m]);
+                    q = quantize8(xv[i], sa_sm[m], ra_sm[m]);
                     if (write_out) *reinterpret_cast<uint2*>(x8_out + int64_t(m) * K + k) = q;
                 }
                 const int chunk = (kc >> 4) ^ (m & 7);
                 *reinterpret_cast<uint2*>(xtiles + kb_local * L::X_TILE + m * BK + chunk * 16 + (kc & 15)) = q;
             }
+        }
+        for (int e = int(threadIdx.x) + ITEMS * kThreads; e < items; e += kThreads) {
+            const int m = e / groups_per_row;
+            const int g = e % groups_per_row;
+            const int kc = (g % kGroupsPerBlock) * 8;
+            const int k = k_lo + g * 8;
+            uint2 q = make_uint2(0u, 0u);
+            if (k < K) {
+                q = quantize8(__ldg(reinterpret_cast<const uint4*>(X + int64_t(m) * K + k)), sa_sm[m], ra_sm[m]);
+                if (write_out) *reinterpret_cast<uint2*>(x8_out + int64_t(m) * K + k) = q;
+            }
+            const int chunk = (kc >> 4) ^ (m & 7);
+            *reinterpret_cast<uint2*>(xtiles + (g / kGroupsPerBlock) * L::X_TILE + m * BK + chunk * 16 + (kc & 15)) = q;
         }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // codes -> tensor-core reads
@@ -337,7 +381,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16*
             const int n = n0 + c0 + r;
             float acc = 0.0f;
             for (uint32_t p = 0; p < S; ++p) acc += recv[(p * my_rows + r) * MP + m];
-            if (n < N) Y[int64_t(m) * N + n] = __float2bfloat16_rn(acc * sa_sm[m] * __ldg(s_w + n));
+            if (n < N) Y[int64_t(m) * N + n] = __float2bfloat16_rn(acc * sa_sm[m] * sw_sm[r]);
         }
     } else {
         // Give partials still on their way a bounded chance to land before

@@ -1,23 +1,24 @@
 // gemm_pair.cuh — prefill-sized FP8 GEMM on CTA pairs (tcgen05 cta_group::2):
 //     Y[m, n] = bf16( (sum_k dec(X8[m,k]) * dec(W8[n,k])) * s_a[m] * s_w[n] )
 //
-// A cluster of two CTAs computes 256 x 256 output tiles with one MMA stream:
+// A cluster of two CTAs computes 256 x BN output tiles (BN = 256, or 128
+// when that fills the GPU in fewer rounds) with one MMA stream:
 //   - each CTA loads, with plain TMA (no multicast), its own 128 rows of the
-//     X8 tile and its own 128 rows of the W8 tile into the same shared-memory
+//     X8 tile and its own BN/2 rows of the W8 tile into the same shared-memory
 //     offsets; the loads of both CTAs count their bytes on the even CTA's
 //     "full" barrier;
 //   - one thread of the even CTA issues tcgen05.mma.cta_group::2 (M = 256,
-//     N = 256, K = 32 per instruction); the hardware reads the A rows and the
+//     N = BN, K = 32 per instruction); the hardware reads the A rows and the
 //     B columns of both CTAs, and each CTA's TMEM receives its 128 rows of D;
 //   - tcgen05.commit with a two-CTA mask frees the ring slot in both CTAs and
 //     hands each CTA its finished accumulator;
 //   - each CTA's four epilogue warps scale and store their 128 rows and
 //     report back to the even CTA, which then reuses that accumulator.
-// Per CTA and k-block the ring takes 32 KB for 128 x 256 x 128 MACs, two
-// thirds of the bytes a single-CTA 128 x 256 tile needs, so a six-deep ring
-// fits and L2 -> SM traffic drops by a third.  Two fp32 accumulators
-// (2 x 256 TMEM columns) overlap the epilogue of one tile with the main loop
-// of the next.  Tiles are walked n-fastest.
+// With BN = 256, per CTA and k-block the ring takes 32 KB for 128 x 256 x 128
+// MACs, two thirds of the bytes a single-CTA 128 x 256 tile needs, so a
+// six-deep ring fits and L2 -> SM traffic drops by a third.  Two fp32
+// accumulators (2 x BN TMEM columns) overlap the epilogue of one tile with the
+// main loop of the next.  Tiles are walked n-fastest.
 //
 // Every wait is bounded (see gemm_tiled.cuh); both CTAs meet on a cluster
 // barrier before either leaves, so neither exits while the other may still
@@ -33,17 +34,18 @@ namespace mfp8 {
 namespace pair {
 
 constexpr int BM = 256;        // rows of the pair's tile (128 per CTA)
-constexpr int BN = 256;        // columns of the tile (128 W8 rows per CTA)
 constexpr int HALF = 128;
 constexpr int BK = 128;
 constexpr int MMA_K = 32;
 constexpr int kThreads = 192;
-constexpr int TMEM_COLS = 2 * BN;
 
-template <int STAGES>
+// BN: columns of the pair's tile (BN/2 W8 rows per CTA), 256 or 128.
+template <int BN, int STAGES>
 struct Layout {
-    static constexpr int A_BYTES = HALF * BK;  // this CTA's rows of X8
-    static constexpr int B_BYTES = HALF * BK;  // this CTA's rows of W8
+    static_assert(BN == 256 || BN == 128, "pair tile width");
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int A_BYTES = HALF * BK;       // this CTA's rows of X8
+    static constexpr int B_BYTES = (BN / 2) * BK;   // this CTA's rows of W8
     static constexpr int CTA_STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = STAGES * A_BYTES;
@@ -57,12 +59,13 @@ __device__ __forceinline__ __nv_bfloat162 scale2(float a, float b, float sa, flo
     return __floats2bfloat162_rn(a * sa * sw0, b * sa * sw1);
 }
 
-template <int STAGES>
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ s_a, const float* __restrict__ s_w,
                  __nv_bfloat16* __restrict__ Y, int M, int N, int K) {
-    using L = Layout<STAGES>;
+    using L = Layout<BN, STAGES>;
+    constexpr int TMEM_COLS = L::TMEM_COLS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -129,7 +132,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     if (cr == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * L::CTA_STAGE_BYTES);
                     tma_load_2d_pair(sA + stage * L::A_BYTES, &tmX, leader_full, kb * BK, tm * BM + int(cr) * HALF,
                                      policy_x);
-                    tma_load_2d_pair(sB + stage * L::B_BYTES, &tmW, leader_full, kb * BK, tn * BN + int(cr) * HALF,
+                    tma_load_2d_pair(sB + stage * L::B_BYTES, &tmW, leader_full, kb * BK, tn * BN + int(cr) * (BN / 2),
                                      policy_w);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }

@@ -7,14 +7,16 @@
 
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "../../include/mfp8.h"
 #include "status.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "gemm_tiled.cuh"
-#include "gemm_splitk.cuh"
+#include "gemm_skinny.cuh"
 #include "gemm_decode.cuh"
 #include "gemm_pair.cuh"
 
@@ -97,29 +99,32 @@ mfp8_status launch_status() {
 // ------------------------------------------------------------- quantize --
 
 template <bool EARLY_TRIGGER>
-mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
+mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float* S, unsigned int* zero, int nzero,
+                            cudaStream_t stream) {
     if (R == 0) return MFP8_OK;
     const int64_t nvec = K / 8;
     const uint4* x = static_cast<const uint4*>(X);
     uint2* q = static_cast<uint2*>(Q);
     const dim3 grid(static_cast<unsigned>(R)), block(kQuantThreads);
-    if (nvec <= 256) quant_rows_reg_kernel<1, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 512) quant_rows_reg_kernel<2, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 1024) quant_rows_reg_kernel<4, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 1536) quant_rows_reg_kernel<6, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
-    else if (nvec <= 2048) quant_rows_reg_kernel<8, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
-    else quant_rows_loop_kernel<EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S);
+    if (nvec <= 256) quant_rows_reg_kernel<1, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
+    else if (nvec <= 512) quant_rows_reg_kernel<2, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
+    else if (nvec <= 1024) quant_rows_reg_kernel<4, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
+    else if (nvec <= 1536) quant_rows_reg_kernel<6, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
+    else if (nvec <= 2048) quant_rows_reg_kernel<8, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
+    else quant_rows_loop_kernel<EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
     return launch_status();
 }
 
-// Activations: the GEMM launched next may start its prologue early.
-mfp8_status quantize_act_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
-    return quantize_rows_t<true>(X, R, K, Q, S, stream);
+// Activations: the GEMM launched next may start its prologue early.  Block 0
+// also clears the GEMM's split-K counters, if any.
+mfp8_status quantize_act_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream,
+                              unsigned int* zero = nullptr, int nzero = 0) {
+    return quantize_rows_t<true>(X, R, K, Q, S, zero, nzero, stream);
 }
 
 // Weights: no early start for whatever follows.
 mfp8_status quantize_weight_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
-    return quantize_rows_t<false>(X, R, K, Q, S, stream);
+    return quantize_rows_t<false>(X, R, K, Q, S, nullptr, 0, stream);
 }
 
 mfp8_status check_quant_args(const void* X, int64_t R, int64_t K, const void* Q, const float* S) {
@@ -139,7 +144,6 @@ mfp8_status check_quant_args(const void* X, int64_t R, int64_t K, const void* Q,
 
 constexpr int kTiledBN = 256;
 constexpr int kTiledStages = 4;
-constexpr int64_t kSplitKMaxM = 128;
 
 template <class Kern>
 mfp8_status set_smem(Kern kern, int bytes, int dev, bool* done) {
@@ -184,23 +188,19 @@ mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K,
     return MFP8_OK;
 }
 
-int64_t splitk_cluster(int64_t tiles, int64_t kb_total, int per_sm, const DeviceInfo& info);
-
-#ifndef MFP8_PAIR_STAGES
-#define MFP8_PAIR_STAGES 6
-#endif
-
-mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                        int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info, cudaStream_t stream) {
-    using L = pair::Layout<MFP8_PAIR_STAGES>;
-    auto kern = pair::gemm_pair_kernel<MFP8_PAIR_STAGES>;
+template <int BN, int STAGES>
+mfp8_status launch_pair_bn(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+                           int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                           cudaStream_t stream) {
+    using L = pair::Layout<BN, STAGES>;
+    auto kern = pair::gemm_pair_kernel<BN, STAGES>;
     static bool attr_done[kMaxDevices] = {};
     mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
     if (st != MFP8_OK) return st;
     CUtensorMap tmX, tmW;
     if ((st = make_map_u8(&tmX, X8, M, K, pair::HALF)) != MFP8_OK) return st;
-    if ((st = make_map_u8(&tmW, W8, N, K, pair::HALF)) != MFP8_OK) return st;
-    const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN);
+    if ((st = make_map_u8(&tmW, W8, N, K, BN / 2)) != MFP8_OK) return st;
+    const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + BN - 1) / BN);
     const int64_t max_pairs = info.sm_count / 2;
     const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
 
@@ -226,107 +226,100 @@ mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, 
     return MFP8_OK;
 }
 
-template <int MP, int STAGES>
-mfp8_status launch_splitk_mp(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
-                             const float* s_w, int64_t N, void* Y, bool dependent, int dev,
-                             const DeviceInfo& info, cudaStream_t stream) {
-    using L = splitk::Layout<MP, STAGES>;
-    auto kern = splitk::gemm_splitk_kernel<MP, STAGES>;
-    static bool attr_done[kMaxDevices] = {};
-    mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
-    if (st != MFP8_OK) return st;
-    CUtensorMap tmW, tmX;
-    if ((st = make_map_u8(&tmW, W8, N, K, splitk::BW)) != MFP8_OK) return st;
-    if ((st = make_map_u8(&tmX, X8, M, K, MP)) != MFP8_OK) return st;
-
-    const int64_t tiles = (N + splitk::BW - 1) / splitk::BW;
-    const int64_t kb_total = (K + splitk::BK - 1) / splitk::BK;
-    // Split K so that the grid covers the SMs about twice (two CTAs fit per
-    // SM for the small MP), without giving any CTA an empty K range.
-    const int per_sm = (2 * L::SMEM_BYTES <= 227 * 1024) ? 2 : 1;
-    const int64_t S = splitk_cluster(tiles, kb_total, per_sm, info);
-    if (tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(S), unsigned(tiles));
-    cfg.blockDim = dim3(splitk::kThreads);
-    cfg.dynamicSmemBytes = L::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(S);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tmW, tmX, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
-                           int(K)) != cudaSuccess) {
-        cudaGetLastError();
-        return MFP8_ERR_CUDA;
-    }
-    return MFP8_OK;
+// Tile width for the pair kernel: the one that finishes sooner, counting
+// rounds of tiles over the CTA pairs times the time of one tile.  A
+// 256 x 128 tile moves 3/4 of the bytes of a 256 x 256 tile for half the
+// MACs and measured about 1.45x slower per MAC, so it is chosen only when it
+// saves rounds (narrow N, e.g. the k/v projections at M = 2048).
+int pair_tile_width(int64_t M, int64_t N, const DeviceInfo& info) {
+    const int64_t pairs = info.sm_count / 2;
+    const int64_t mt = (M + pair::BM - 1) / pair::BM;
+    const int64_t r256 = (mt * ((N + 255) / 256) + pairs - 1) / pairs;
+    const int64_t r128 = (mt * ((N + 127) / 128) + pairs - 1) / pairs;
+    return double(r128) * 128.0 * 1.45 < double(r256) * 256.0 ? 128 : 256;
 }
 
-mfp8_status launch_splitk(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
-                          const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
-                          cudaStream_t stream) {
-    if (M <= 16) return launch_splitk_mp<16, 5>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-    if (M <= 32) return launch_splitk_mp<32, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-    if (M <= 64) return launch_splitk_mp<64, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-    if (M <= 128) return launch_splitk_mp<128, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-    return MFP8_ERR_UNSUPPORTED_SHAPE;
+mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+                        int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info, cudaStream_t stream) {
+    if (pair_tile_width(M, N, info) == 128)
+        return launch_pair_bn<128, 8>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    return launch_pair_bn<256, 6>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
 }
 
 constexpr int64_t kFusedMaxM = 64;
 
-// Cluster size (K-split) for the weight-streaming kernels: enough CTAs to
-// cover every SM `per_sm` times, at most 8 (portable cluster size), and no
-// CTA with an empty K range.
-int64_t splitk_cluster(int64_t tiles, int64_t kb_total, int per_sm, const DeviceInfo& info) {
-    int64_t S = (int64_t(info.sm_count) * per_sm + tiles - 1) / tiles;
-    if (S > 8) S = 8;
-    if (S > kb_total) S = kb_total;
-    if (S < 1) S = 1;
-    return S;
-}
 
-// Decode kernel sizing: CTAs per SM the grid aims to fill, at most.
-#ifndef MFP8_DECODE_CTAS_PER_SM
-#define MFP8_DECODE_CTAS_PER_SM 2
-#endif
 #ifndef MFP8_DECODE_STAGES
 #define MFP8_DECODE_STAGES 4
 #endif
+
+// Clusters of `S` CTAs of `kern` (with `smem` bytes each) that the device
+// keeps resident at once.  Clusters are placed inside one GPC, so this can
+// be far below (SMs x CTAs per SM) / S.  Cached per device and shape.
+template <class Kern>
+int max_active_clusters(Kern kern, int S, int smem, int threads, int dev) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, const void*, int, int>, int> cache;
+    const auto key = std::make_tuple(dev, reinterpret_cast<const void*>(kern), S, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(S));
+    cfg.blockDim = dim3(unsigned(threads));
+    cfg.dynamicSmemBytes = size_t(smem);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cache[key] = n;
+    return n;
+}
 
 template <int MP, int ITEMS>
 mfp8_status launch_decode_mp(const void* X, int64_t M, int64_t K, const void* W8, const float* s_w, int64_t N,
                              void* Y, bool weights_static, void* x8_out, float* sa_out, int dev,
                              const DeviceInfo& info, cudaStream_t stream) {
+    (void)info;
     constexpr int STAGES = MFP8_DECODE_STAGES;
     using L = decode::Layout<MP, STAGES>;
     auto kern = decode::gemm_decode_kernel<MP, STAGES, ITEMS>;
     const int64_t tiles = (N + decode::BW - 1) / decode::BW;
     const int64_t kb_total = (K + decode::BK - 1) / decode::BK;
     if (tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    // K-split: fill the SMs without a second wave, then split further if one
-    // CTA's slice of X would not fit in its registers.
-    int64_t S = (int64_t(info.sm_count) * MFP8_DECODE_CTAS_PER_SM) / tiles;
-    if (S < 1) S = 1;
-    if (S > decode::kMaxCluster) S = decode::kMaxCluster;
-    if (S > kb_total) S = kb_total;
-    auto nkb_cap_of = [&](int64_t s) { return (kb_total + s - 1) / s; };
-    while (S < decode::kMaxCluster && S < kb_total &&
-           M * nkb_cap_of(S) * decode::kGroupsPerBlock > int64_t(ITEMS) * decode::kThreads)
-        ++S;
-    const int64_t nkb_cap = nkb_cap_of(S);
-    if (M * nkb_cap * decode::kGroupsPerBlock > int64_t(ITEMS) * decode::kThreads) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    const int smem = L::smem_bytes(int(nkb_cap));
-    if (smem > 227 * 1024) return MFP8_ERR_UNSUPPORTED_SHAPE;
     static bool attr_done[kMaxDevices] = {};
     mfp8_status st = set_smem(kern, 227 * 1024, dev, attr_done);
     if (st != MFP8_OK) return st;
+    // K-split S: the largest cluster size whose whole grid (tiles clusters)
+    // is resident in one wave; failing that, the S with the fewest waves.
+    auto nkb_cap_of = [&](int64_t s) { return (kb_total + s - 1) / s; };
+    int64_t best_S = 0, best_waves = INT64_MAX;
+    for (int64_t S = decode::kMaxCluster; S >= 1; --S) {
+        if (S > kb_total) continue;
+        const int64_t nkb_cap = nkb_cap_of(S);
+        const int smem = L::smem_bytes(int(nkb_cap));
+        if (smem > 227 * 1024) continue;
+        const int active = max_active_clusters(kern, int(S), smem, decode::kThreads, dev);
+        if (active <= 0) continue;
+        const int64_t waves = (tiles + active - 1) / active;
+        if (waves < best_waves) {
+            best_waves = waves;
+            best_S = S;
+        }
+        if (waves == 1) break;
+    }
+    if (best_S == 0) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t S = best_S;
+    const int64_t nkb_cap = nkb_cap_of(S);
+    const int smem = L::smem_bytes(int(nkb_cap));
     CUtensorMap tmW;
     if ((st = make_map_u8(&tmW, W8, N, K, decode::BW)) != MFP8_OK) return st;
 
@@ -365,10 +358,15 @@ mfp8_status launch_fused(const void* X, int64_t M, int64_t K, const void* W8, co
     return MFP8_ERR_UNSUPPORTED_SHAPE;
 }
 
+constexpr int64_t kSkinnyMaxM = skinny::kMaxM;
+constexpr int kSkinnyStages = 4;
+
 int choose_path(int64_t M, int64_t N, int64_t K) {
     (void)N;
     (void)K;
-    return M <= kFusedMaxM ? MFP8_PATH_SPLITK : MFP8_PATH_TILED;
+    if (M <= 64) return MFP8_PATH_SPLITK;
+    if (M < 256) return MFP8_PATH_TILED;
+    return MFP8_PATH_PAIR;
 }
 
 mfp8_status check_gemm_args(int64_t M, int64_t N, int64_t K, const void* W8, const float* s_w, const void* Y) {
@@ -384,26 +382,102 @@ mfp8_status check_gemm_args(int64_t M, int64_t N, int64_t K, const void* W8, con
     return MFP8_OK;
 }
 
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// K-splits of the skinny kernel: as many CTAs as SMs, no CTA without k-blocks.
+int64_t skinny_splits(int64_t N, int64_t K, int sm_count) {
+    const int64_t tiles = (N + skinny::BN - 1) / skinny::BN;
+    const int64_t kb_total = (K + skinny::BK - 1) / skinny::BK;
+    int64_t splits = sm_count / tiles;
+    if (splits < 1) splits = 1;
+    if (splits > kb_total) splits = kb_total;
+    return splits;
+}
+
+// How one call uses the caller's workspace: the activation codes and scales
+// of the quantize pass, then (split-K) the fp32 partials [tile][split][M][256]
+// and one counter per tile; each region 256-byte aligned.
+struct Plan {
+    size_t x8_off = 0, sa_off = 0, part_off = 0, cnt_off = 0, total = 0;
+    int64_t tiles = 0, splits = 0;
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, bool codes, bool split_k, int sm_count) {
+    Plan p;
+    size_t off = 0;
+    if (codes) {
+        p.x8_off = off;
+        off += round_up(size_t(M) * size_t(K), 256);
+        p.sa_off = off;
+        off += round_up(size_t(M) * 4, 256);
+    }
+    if (split_k) {
+        p.tiles = (N + skinny::BN - 1) / skinny::BN;
+        p.splits = skinny_splits(N, K, sm_count);
+        p.part_off = off;
+        off += round_up(size_t(p.tiles * p.splits) * size_t(M) * skinny::BN * 4, 256);
+        p.cnt_off = off;
+        off += round_up(size_t(p.tiles) * 4, 256);
+    }
+    p.total = off;
+    return p;
+}
+
+mfp8_status launch_skinny(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+                          int64_t N, void* Y, float* partial, unsigned int* counters, const Plan& plan,
+                          bool weights_static, bool dependent, int dev, cudaStream_t stream) {
+    using L = skinny::Layout<kSkinnyStages>;
+    auto kern = skinny::gemm_skinny_kernel<kSkinnyStages>;
+    static bool attr_done[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
+    if (st != MFP8_OK) return st;
+    CUtensorMap tmX, tmW;
+    if ((st = make_map_u8(&tmX, X8, M, K, skinny::BM)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmW, W8, N, K, skinny::BN)) != MFP8_OK) return st;
+    if (plan.tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(plan.splits), unsigned(plan.tiles));
+    cfg.blockDim = dim3(skinny::kThreads);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, s_a, s_w, static_cast<__nv_bfloat16*>(Y), partial, counters,
+                           int(M), int(N), int(K), weights_static ? 1 : 0) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
+// The GEMM on codes already in memory (tiled, pair, or split-K).
 mfp8_status run_gemm(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                     int64_t N, void* Y, int path, bool dependent, int dev, const DeviceInfo& info,
-                     cudaStream_t stream) {
-    if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
-    // The tiled kernel takes M, N, K as 32-bit; tile counts must fit too.
+                     int64_t N, void* Y, int path, void* ws, const Plan& plan, bool weights_static, bool dependent,
+                     int dev, const DeviceInfo& info, cudaStream_t stream) {
+    // The kernels take M, N, K as 32-bit.
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (path == MFP8_PATH_TILED) return launch_tiled(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
     if (path == MFP8_PATH_PAIR) return launch_pair(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
     if (path == MFP8_PATH_SPLITK) {
-        if (M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
-        return launch_splitk(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+        uint8_t* base = static_cast<uint8_t*>(ws);
+        return launch_skinny(X8, s_a, M, K, W8, s_w, N, Y, reinterpret_cast<float*>(base + plan.part_off),
+                             reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static, dependent,
+                             dev, stream);
     }
     return MFP8_ERR_INVALID_ARG;
 }
 
-size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-// Workspace: X8 [M, K] then s_a [M], each 256-byte aligned.
-size_t workspace_bytes(int64_t M, int64_t K) {
-    return round_up(size_t(M) * size_t(K), 256) + round_up(size_t(M) * 4, 256);
+int sm_count_for_sizing() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+        return sms;
+    cudaGetLastError();
+    return 148;  // B200
 }
 
 __global__ void bounded_wait_kernel(uint64_t limit_ns) {
@@ -449,8 +523,8 @@ mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K, void* X_
 }
 
 size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || K > kMaxDim) return 0;
-    return workspace_bytes(M, K);
+    if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return 0;
+    return make_plan(M, N, K, true, M <= kSkinnyMaxM, sm_count_for_sizing()).total;
 }
 
 mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
@@ -458,9 +532,10 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
                            int flags, void* X_fp8_out, float* x_scale_out, void* stream) {
     mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
     if (st != MFP8_OK) return st;
-    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_PAIR) return MFP8_ERR_INVALID_ARG;
+    if (path < MFP8_PATH_AUTO || path > MFP8_PATH_FUSED) return MFP8_ERR_INVALID_ARG;
     if ((flags & ~MFP8_FLAG_STATIC_WEIGHTS) != 0) return MFP8_ERR_INVALID_ARG;
-    if (path == MFP8_PATH_SPLITK && M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_SPLITK && M > kSkinnyMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_FUSED && M > kFusedMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_bf16) return MFP8_ERR_INVALID_ARG;
     if (!aligned16(X_bf16)) return MFP8_ERR_MISALIGNED;
@@ -474,41 +549,35 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
             return MFP8_ERR_INVALID_ARG;
     }
     if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
-    const bool fused = path == MFP8_PATH_SPLITK && M <= kFusedMaxM;
-
-    void* X8 = X_fp8_out;
-    float* s_a = x_scale_out;
-    if (!fused && !X8) {
-        const size_t need = workspace_bytes(M, K);
-        if (!workspace || workspace_bytes_given < need) return MFP8_ERR_WORKSPACE;
-        if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
-        X8 = workspace;
-        s_a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(size_t(M) * size_t(K), 256));
-        if ((st = check_quant_args(X_bf16, M, K, X8, s_a)) != MFP8_OK) return st;
-        if (ranges_overlap(X8, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
-            ranges_overlap(s_a, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
-            return MFP8_ERR_INVALID_ARG;
+    const bool weights_static = (flags & MFP8_FLAG_STATIC_WEIGHTS) != 0;
+    const bool split_k = path == MFP8_PATH_SPLITK;
+    Plan plan;
+    if (path != MFP8_PATH_FUSED) {
+        plan = make_plan(M, N, K, X_fp8_out == nullptr, split_k, sm_count_for_sizing());
+        if (plan.total > 0) {
+            if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
+            if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
+            if (ranges_overlap(workspace, plan.total, Y_bf16, size_t(M * N * 2)) ||
+                ranges_overlap(workspace, plan.total, X_bf16, size_t(M * K * 2)))
+                return MFP8_ERR_INVALID_ARG;
+        }
     }
 
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (fused) {
-        st = launch_fused(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, (flags & MFP8_FLAG_STATIC_WEIGHTS) != 0,
-                          X_fp8_out, x_scale_out, dev, info, s);
-        if (st != MFP8_ERR_UNSUPPORTED_SHAPE) return st;
-        // Too large for the on-chip codes: quantize pass + unfused split-K.
-        if (!X8) {
-            const size_t need = workspace_bytes(M, K);
-            if (!workspace || workspace_bytes_given < need) return MFP8_ERR_WORKSPACE;
-            if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
-            X8 = workspace;
-            s_a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(size_t(M) * size_t(K), 256));
-        }
-    }
-    if ((st = quantize_act_rows(X_bf16, M, K, X8, s_a, s)) != MFP8_OK) return st;
-    return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, path, /*dependent=*/true, dev, info, s);
+    if (path == MFP8_PATH_FUSED)
+        return launch_fused(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, weights_static, X_fp8_out, x_scale_out, dev,
+                            info, s);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    void* X8 = X_fp8_out ? X_fp8_out : base + plan.x8_off;
+    float* s_a = x_scale_out ? x_scale_out : reinterpret_cast<float*>(base + plan.sa_off);
+    unsigned int* counters = split_k ? reinterpret_cast<unsigned int*>(base + plan.cnt_off) : nullptr;
+    if ((st = quantize_act_rows(X_bf16, M, K, X8, s_a, s, counters, split_k ? int(plan.tiles) : 0)) != MFP8_OK)
+        return st;
+    return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, path, workspace, plan, weights_static,
+                    /*dependent=*/true, dev, info, s);
 }
 
 mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
@@ -517,23 +586,45 @@ mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K, const void* W_
                           MFP8_PATH_AUTO, 0, nullptr, nullptr, stream);
 }
 
+size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return 0;
+    return make_plan(M, N, K, false, M <= kSkinnyMaxM, sm_count_for_sizing()).total;
+}
+
 mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K, const void* W_fp8,
-                      const float* w_scale, int64_t N, void* Y_bf16, int path, void* stream) {
+                      const float* w_scale, int64_t N, void* Y_bf16, void* workspace, size_t workspace_bytes_given,
+                      int path, void* stream) {
     mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
     if (st != MFP8_OK) return st;
     if (path < MFP8_PATH_AUTO || path > MFP8_PATH_PAIR) return MFP8_ERR_INVALID_ARG;
-    if (path == MFP8_PATH_SPLITK && M > kSplitKMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_SPLITK && M > kSkinnyMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_fp8 || !x_scale) return MFP8_ERR_INVALID_ARG;
     if (!aligned16(X_fp8) || !aligned16(x_scale)) return MFP8_ERR_MISALIGNED;
     if (ranges_overlap(X_fp8, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
         ranges_overlap(x_scale, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
         return MFP8_ERR_INVALID_ARG;
+    if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
+    const bool split_k = path == MFP8_PATH_SPLITK;
+    const Plan plan = make_plan(M, N, K, false, split_k, sm_count_for_sizing());
+    if (plan.total > 0) {
+        if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
+        if (ranges_overlap(workspace, plan.total, Y_bf16, size_t(M * N * 2))) return MFP8_ERR_INVALID_ARG;
+    }
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
-    return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, /*dependent=*/false, dev, info,
-                    static_cast<cudaStream_t>(stream));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (plan.total > 0) {
+        if (cudaMemsetAsync(static_cast<uint8_t*>(workspace) + plan.cnt_off, 0, size_t(plan.tiles) * 4, s) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return MFP8_ERR_CUDA;
+        }
+    }
+    return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, workspace, plan,
+                    /*weights_static=*/false, /*dependent=*/false, dev, info, s);
 }
 
 mfp8_status mfp8_e4m3_encode_f32(const float* in, int64_t n, uint8_t* out, void* stream) {

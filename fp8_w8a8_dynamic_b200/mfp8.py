@@ -25,6 +25,7 @@ PATH_AUTO = 0
 PATH_TILED = 1
 PATH_SPLITK = 2
 PATH_PAIR = 3
+PATH_FUSED = 4
 
 FLAG_STATIC_WEIGHTS = 1
 
@@ -52,7 +53,8 @@ def lib():
             "mfp8_linear_workspace_bytes": (sz, [i64, i64, i64]),
             "mfp8_linear": (i32, [P, i64, i64, P, P, i64, P, P, sz, P]),
             "mfp8_linear_ex": (i32, [P, i64, i64, P, P, i64, P, P, sz, i32, i32, P, P, P]),
-            "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, i32, P]),
+            "mfp8_gemm_workspace_bytes": (sz, [i64, i64, i64]),
+            "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, P, sz, i32, P]),
             "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
             "mfp8_debug_bounded_wait": (i32, [i64, P]),
             "mfp8_get_device_status": (i32, [P]),
@@ -91,8 +93,14 @@ def mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace
                                 path, flags, X_fp8_out, x_scale_out, stream)
 
 
-def mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path=PATH_AUTO, stream=0):
-    return lib().mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, stream)
+def mfp8_gemm_workspace_bytes(M, N, K):
+    return lib().mfp8_gemm_workspace_bytes(M, N, K)
+
+
+def mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, path=PATH_AUTO,
+              stream=0):
+    return lib().mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, path,
+                           stream)
 
 
 def mfp8_e4m3_encode_f32(inp, n, out, stream=0):
@@ -169,7 +177,7 @@ def linear(X, W8, w_scale, out=None, workspace=None, path=PATH_AUTO, x8_out=None
     N = W8.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    if workspace is None and x8_out is None:
+    if workspace is None:
         workspace = workspace_for(M, N, K, X.device)
     ws_bytes = workspace.numel() if workspace is not None else 0
     _check(mfp8_linear_ex(_ptr(X), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), _ptr(workspace),
@@ -178,15 +186,18 @@ def linear(X, W8, w_scale, out=None, workspace=None, path=PATH_AUTO, x8_out=None
     return out
 
 
-def gemm(X8, x_scale, W8, w_scale, out=None, path=PATH_AUTO, stream=None):
+def gemm(X8, x_scale, W8, w_scale, out=None, path=PATH_AUTO, workspace=None, stream=None):
     """The contraction alone on pre-quantized activations."""
     import torch
     M, K = X8.shape
     N = W8.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=X8.device)
-    _check(mfp8_gemm(_ptr(X8), _ptr(x_scale), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), path,
-                     _stream_handle(stream)), "mfp8_gemm")
+    if workspace is None:
+        workspace = torch.empty((max(mfp8_gemm_workspace_bytes(M, N, K), 16),), dtype=torch.uint8,
+                                device=X8.device)
+    _check(mfp8_gemm(_ptr(X8), _ptr(x_scale), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), _ptr(workspace),
+                     workspace.numel(), path, _stream_handle(stream)), "mfp8_gemm")
     return out
 
 

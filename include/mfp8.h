@@ -85,10 +85,10 @@ MFP8_API mfp8_status mfp8_quantize_weight(const void* W_bf16, int64_t N, int64_t
 MFP8_API mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K,
                               void* X_fp8, float* x_scale, void* stream);
 
-/* Bytes of device workspace that is enough for mfp8_linear and for every
- * kernel choice of mfp8_linear_ex at these sizes (the activation codes and
- * scales of the separate quantize pass).  The decode-sized kernel (M <= 64)
- * quantizes on chip and ignores the workspace.  Never fails; returns 0 for
+/* Bytes of device workspace that are enough for mfp8_linear and for every
+ * kernel choice of mfp8_linear_ex at these sizes on the current device: the
+ * activation codes and scales of the quantize pass and, for M <= 128, the
+ * fp32 split-K partials and per-tile counters.  Never fails; returns 0 for
  * invalid sizes (mfp8_linear then reports the error). */
 MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -100,10 +100,10 @@ MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *            mfp8_quantize_weight, read only.
  *   Y_bf16   [M, N] bf16, written.  Must not overlap any input.
  *   workspace / workspace_bytes: device scratch of at least
- *            mfp8_linear_workspace_bytes(M, N, K) bytes; may be NULL for
- *            M <= 64, where the kernel keeps the activation codes on chip.
- *            Its contents on entry do not matter; they are garbage on exit.
- *            Concurrent calls need separate workspaces.
+ *            mfp8_linear_workspace_bytes(M, N, K) bytes, 16-byte aligned.
+ *            Its contents on entry do not matter (the call initialises what
+ *            it uses); they are garbage on exit.  Calls that may run at the
+ *            same time need separate workspaces.
  * The activation quantization (per-token scale + e4m3 codes) happens inside
  * this call: its codes and scales are bit-identical to mfp8_quantize_act.
  * Outputs are within |y - y_ref| <= 2^-7 |y_ref| + 1e-5 * sum_k |a_k w_k| s_a s_w
@@ -117,8 +117,9 @@ MFP8_API mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K,
 typedef enum {
     MFP8_PATH_AUTO = 0,   /* what mfp8_linear does: chosen from M, N, K */
     MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
-    MFP8_PATH_SPLITK = 2, /* weight-streaming split-K tcgen05 GEMM (M <= 128); M <= 64 fuses the quantize step */
-    MFP8_PATH_PAIR = 3    /* quantize pass, then the 256 x 256-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
+    MFP8_PATH_SPLITK = 2, /* quantize pass, then the weight-streaming split-K GEMM over all SMs (M <= 128) */
+    MFP8_PATH_PAIR = 3,   /* quantize pass, then the 256-row-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
+    MFP8_PATH_FUSED = 4   /* one kernel: on-chip quantize + cluster split-K GEMM (M <= 64), no workspace */
 } mfp8_path;
 
 /* Flags for mfp8_linear_ex. */
@@ -135,22 +136,30 @@ typedef enum {
  * x_scale_out [M]; pass NULL for none).  Used to test each kernel on the
  * same shapes, to check that the activation bytes of every path are
  * bit-identical to mfp8_quantize_act, and by callers with static weights.
- * path MFP8_PATH_SPLITK with M <= 64 quantizes X inside the GEMM kernel (one
- * launch); with 64 < M <= 128 it runs the quantize pass first.  Returns
- * MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel cannot take these sizes,
- * MFP8_ERR_INVALID_ARG for an unknown path or flag. */
+ * MFP8_PATH_FUSED quantizes X inside the GEMM kernel and needs no workspace.
+ * When X_fp8_out is given, the quantize pass writes the codes there instead
+ * of the workspace.  Returns MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel
+ * cannot take these sizes, MFP8_ERR_INVALID_ARG for an unknown path or flag. */
 MFP8_API mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K,
                            const void* W_fp8, const float* w_scale, int64_t N,
                            void* Y_bf16, void* workspace, size_t workspace_bytes,
                            int path, int flags, void* X_fp8_out, float* x_scale_out,
                            void* stream);
 
+/* Workspace bytes mfp8_gemm needs at these sizes on the current device
+ * (the split-K partials and counters; 0 when no kernel choice needs any). */
+MFP8_API size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
 /* The contraction and epilogue alone, on activations already quantized by
  * mfp8_quantize_act: Y = bf16((X_fp8 . W_fp8^T) * x_scale (x) w_scale).
- * Lets the GEMM be timed and checked without the quantize pass. */
+ * Lets the GEMM be timed and checked without the quantize pass.  path is
+ * AUTO, TILED, SPLITK or PAIR; the split-K kernel takes its partials from
+ * `workspace` (at least mfp8_gemm_workspace_bytes) and clears its counters
+ * with a memset on `stream` first. */
 MFP8_API mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K,
                       const void* W_fp8, const float* w_scale, int64_t N,
-                      void* Y_bf16, int path, void* stream);
+                      void* Y_bf16, void* workspace, size_t workspace_bytes,
+                      int path, void* stream);
 
 /* Diagnostic: encode n fp32 values with the device's e4m3 conversion (the
  * one the quantize kernels use).  in [n] fp32, out [n] codes.  Used to check

@@ -50,9 +50,16 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_bytes(lib):
-    # X8 [M, K] then s_a [M], each rounded up to 256 bytes
-    assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == 65536 + 256
-    assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == 256 + 256
+    # X8 [M, K] then s_a [M], each rounded up to 256 bytes; for M <= 128 also
+    # the split-K partials [tiles][splits][M][256] fp32 and one counter per tile
+    # (sized for 148 SMs when no device is present)
+    assert mfp8.mfp8_linear_workspace_bytes(300, 4096, 4096) == 300 * 4096 + 1280
+    tiles, splits = 16, 9  # N = 4096 in 256-wide tiles; 148 // 16 K-splits
+    assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == 65536 + 256 + tiles * splits * 16 * 1024 + 256
+    assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == tiles * splits * 16 * 1024 + 256
+    assert mfp8.mfp8_gemm_workspace_bytes(300, 4096, 4096) == 0
+    # one K-block only: one split
+    assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == 256 + 256 + 3 * 1024 + 256
     assert mfp8.mfp8_linear_workspace_bytes(0, 8, 48) == 0
     assert mfp8.mfp8_linear_workspace_bytes(4, 8, -1) == 0
 
@@ -90,13 +97,17 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert call(M=4, path=mfp8.PATH_TILED, ws=None) == mfp8.ERR_WORKSPACE
     assert call(flags=2) == mfp8.ERR_INVALID_ARG
     assert call(path=7) == mfp8.ERR_INVALID_ARG
-    assert call(path=4) == mfp8.ERR_INVALID_ARG
+    assert call(path=5) == mfp8.ERR_INVALID_ARG
+    assert call(path=mfp8.PATH_FUSED, M=65) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(ws=None) == mfp8.ERR_WORKSPACE  # split-K partials
     assert call(path=mfp8.PATH_SPLITK, M=129) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
     assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X
     assert call(M=0) == mfp8.OK
     G = mfp8.mfp8_gemm
-    assert G(None, FAKE, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, 0, None) == mfp8.ERR_INVALID_ARG
+    assert G(None, FAKE, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_INVALID_ARG
+    assert G(FAKE, FAKE * 9, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_WORKSPACE
+    assert G(FAKE, FAKE * 9, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, mfp8.PATH_FUSED, None) == mfp8.ERR_INVALID_ARG
     assert mfp8.mfp8_e4m3_encode_f32(FAKE, -1, FAKE * 2, None) == mfp8.ERR_INVALID_ARG
     assert mfp8.mfp8_debug_bounded_wait(0, None) == mfp8.ERR_INVALID_ARG
     assert mfp8.mfp8_debug_bounded_wait(10 ** 6, None) == mfp8.ERR_INVALID_ARG

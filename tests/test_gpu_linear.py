@@ -45,15 +45,19 @@ TILED_ONLY = [(130, 264, 384), (300, 520, 1040), (256, 1024, 4096), (1000, 2056,
 
 
 @pytest.mark.parametrize("M,N,K", SMALL)
-@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR, mfp8.PATH_AUTO])
+@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR, mfp8.PATH_FUSED,
+                                  mfp8.PATH_AUTO])
 def test_linear_small(M, N, K, path):
+    if path == mfp8.PATH_FUSED and M > 64:
+        pytest.skip("the fused decode kernel takes M <= 64")
     run_case(M, N, K, path, seed=M * 7 + N)
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (8, 12288, 4096), (16, 4096, 12288), (64, 1024, 4096),
                                    (33, 264, 400)])
-def test_linear_static_weights_flag(M, N, K):
-    run_case(M, N, K, mfp8.PATH_AUTO, seed=M + 3, flags=mfp8.FLAG_STATIC_WEIGHTS)
+@pytest.mark.parametrize("path", [mfp8.PATH_SPLITK, mfp8.PATH_FUSED])
+def test_linear_static_weights_flag(M, N, K, path):
+    run_case(M, N, K, path, seed=M + 3, flags=mfp8.FLAG_STATIC_WEIGHTS)
 
 
 def test_linear_without_codes_out_matches_with():
@@ -80,8 +84,7 @@ def test_linear_tiled_ragged(M, N, K, path):
 @pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR])
 def test_gemm_entry_point(M, N, K, path):
     """mfp8_gemm on codes from mfp8_quantize_act: within tolerance of the
-    oracle, and bit-identical to mfp8_linear on the same kernel when that
-    kernel is the same (tiled, or split-K above the fused size)."""
+    oracle, and bit-identical to mfp8_linear through the same kernel."""
     if path == mfp8.PATH_SPLITK and M > 128:
         pytest.skip("split-K takes M <= 128")
     x = W.make_x(M, K, seed=5, device=DEV)
@@ -90,14 +93,14 @@ def test_gemm_entry_point(M, N, K, path):
     y2 = mfp8.gemm(x8, xs, W8, sw, path=path)
     torch.cuda.synchronize()
     assert_linear_parity(y2, u8(x8), f32(xs), u8(W8), f32(sw), what="mfp8_gemm")
-    if path != mfp8.PATH_SPLITK or M > 64:
+    if True:
         y = mfp8.linear(x, W8, sw, path=path)
         torch.cuda.synchronize()
         assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
 
 
 def test_deterministic():
-    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR):
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR, mfp8.PATH_FUSED):
         x = W.make_x(16, 4096, seed=0, device=DEV)
         W8, sw = mfp8.quantize_weight(W.make_w(4096, 4096, seed=0, device=DEV))
         ys = [mfp8.linear(x, W8, sw, path=path) for _ in range(3)]
@@ -124,7 +127,7 @@ def test_onehot_weights_exact_product():
     expect = (xd[:, j.numpy()] * wd[np.arange(N), j.numpy()][None, :]
               * f32(xs)[:, None].astype(np.float64) * f32(sw)[None, :].astype(np.float64))
     expect_bf16 = torch.from_numpy(expect).to(torch.bfloat16)
-    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR):
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR, mfp8.PATH_FUSED):
         y = mfp8.linear(x, W8, sw, path=path).cpu()
         # one product, rounded once: equal unless the kernel's fp32 rounding of
         # the product lands on the other side of a bf16 tie
@@ -140,7 +143,7 @@ def test_zero_activation_rows_give_zero_outputs():
     x[3] = 0
     x[17] = 0
     W8, sw = mfp8.quantize_weight(W.make_w(N, K, seed=4, device=DEV))
-    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR):
+    for path in (mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR, mfp8.PATH_FUSED):
         y = mfp8.linear(x, W8, sw, path=path)
         torch.cuda.synchronize()
         assert (y[3] == 0).all() and (y[17] == 0).all()
@@ -162,10 +165,11 @@ def sampled_rows(M, n=48, seed=0):
 
 
 @pytest.mark.parametrize("lin", W.LAYER_LINEARS, ids=lambda l: l.name)
-def test_decode_layer_full_size(lin):
+@pytest.mark.parametrize("path", [mfp8.PATH_AUTO, mfp8.PATH_FUSED])
+def test_decode_layer_full_size(lin, path):
     """Decode: the 7 Linears of one layer at M in {1, 4, 8}, every output."""
     for M in (1, 4, 8):
-        run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=1, kind="normal")
+        run_case(M, lin.N, lin.K, path, seed=1, kind="normal", flags=mfp8.FLAG_STATIC_WEIGHTS)
 
 
 @pytest.mark.parametrize("lin", W.LAYER_LINEARS, ids=lambda l: l.name)

@@ -97,3 +97,49 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     q, s = mfp8.quantize_act(x)
     torch.cuda.synchronize()
     assert (u8(q) == 0x7E).all()
+
+
+def _magnitude_sweep_rows(n_rows, seed):
+    """Rows holding every finite bf16 magnitude up to the row's absmax, with
+    random signs, under n_rows different absmax values spread over the whole
+    bf16 range (including ones whose scale is raised to FLT_MIN)."""
+    rng = np.random.default_rng(seed)
+    mags = np.arange(0, 0x7F80, dtype=np.uint16)  # every finite non-negative bf16
+    fixed = [0x7F7F, 0x43E0, 0x3F80, 0x0080, 0x0001, 0x0C00, 0x3C00, 0x4780]  # max, 448, 1, tiny, ...
+    tops = np.array(fixed + list(rng.integers(0x0001, 0x7F80, n_rows - len(fixed))), dtype=np.uint16)
+    K = 0x7F80 + 16
+    rows = np.zeros((n_rows, K), dtype=np.uint16)
+    for i, top in enumerate(tops):
+        r = mags[mags <= top].copy()
+        r = r | (rng.integers(0, 2, r.size, dtype=np.uint16) << 15)  # random signs
+        rng.shuffle(r)
+        rows[i, : r.size] = r
+        rows[i, r.size] = top  # the row's absmax, positive
+    return rows
+
+
+def test_every_bf16_magnitude_under_many_scales():
+    """The multiply-with-boundary-check quantizer against the oracle's
+    division on every bf16 magnitude, under 256 row scales."""
+    rows = _magnitude_sweep_rows(256, seed=21)
+    x = torch.from_numpy(rows.view(np.int16)).view(torch.bfloat16).to(DEV)
+    check_rows(x)
+
+
+@pytest.mark.parametrize("path", [mfp8.PATH_SPLITK, mfp8.PATH_FUSED])
+def test_decode_kernel_codes_every_bf16_magnitude(path):
+    """The same sweep through the decode paths (the fused kernel quantizes on
+    chip and can write its codes out), four tokens per call."""
+    rows = _magnitude_sweep_rows(32, seed=22)
+    K = rows.shape[1]
+    W8, sw = mfp8.quantize_weight(W.make_w(128, K, seed=5, device=DEV))
+    for i in range(0, rows.shape[0], 4):
+        blk = rows[i:i + 4]
+        x = torch.from_numpy(blk.view(np.int16)).view(torch.bfloat16).to(DEV)
+        x8 = torch.empty((4, K), dtype=torch.uint8, device=DEV)
+        xs = torch.empty((4,), dtype=torch.float32, device=DEV)
+        mfp8.linear(x, W8, sw, path=path, x8_out=x8, xs_out=xs)
+        torch.cuda.synchronize()
+        q_ref, s_ref = oracle.quantize_rows(blk)
+        assert np.array_equal(f32(xs).view(np.uint32), s_ref.view(np.uint32))
+        assert np.array_equal(u8(x8), q_ref)
