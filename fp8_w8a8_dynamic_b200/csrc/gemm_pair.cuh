@@ -116,6 +116,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     cluster_wait_acquire();  // both CTAs' barriers exist before any cross-CTA signal
     const uint32_t tmem_base = *tmem_holder;
 
+    // The next call's quantize kernel may start launching; it waits for this
+    // grid to finish before it touches memory.
+    grid_launch_dependents();
     grid_dependency_wait();  // X8 and s_a may come from the kernel launched just before
 
     if (warp == 0) {

@@ -1,4 +1,4 @@
-// gemm_skinny.cuh — decode-sized FP8 GEMM (M <= 128 tokens) without
+// gemm_skinny.cuh — decode-sized FP8_DYNAMIC GEMM (M <= 128 tokens) without
 // clusters: split-K over the whole GPU with a last-arriver reduction.
 //
 //   Y[m, n] = bf16( (sum_k dec(X8[m,k]) * dec(W8[n,k])) * s_a[m] * s_w[n] )
@@ -8,23 +8,28 @@
 // consumes: a tcgen05.mma takes about the same time whether its N is 16 or
 // 256, so the weights are the MMA's B operand (N = 256 output channels per
 // instruction, 8 KB of W8) and the tokens its A operand (M = 128 rows, of
-// which only the first M are real; the TMA load fills the rest with zeros
-// and reads nothing for them).
+// which only the first M are real; the rest are zeros).
 //
 // Grid: tiles (256 channels each) x splits (K ranges), at most one CTA per
 // SM, no clusters.  Each CTA
 //   1. streams its W8 K-range into a 4-stage TMA ring straight away (the
 //      weights do not depend on the kernel before it when declared static);
-//   2. waits for the activation codes of the quantize kernel launched just
-//      before (programmatic dependent launch), and loads them per stage;
+//   2. gets the activation codes of its K-range:
+//        QUANT = false: loads them, per stage, from the codes the quantize
+//                       kernel launched just before wrote (TMA; rows >= M
+//                       are filled with zeros and cost no reads);
+//        QUANT = true (M <= 16): reads the whole rows of X (BF16) itself,
+//                       takes each token's absmax and scale (the same rule
+//                       and device functions as the quantize kernel), and
+//                       its four otherwise idle warps write the codes of each
+//                       k-block into the ring, next to the weights;
 //   3. issues 4 MMAs per 128-byte k-block into one fp32 TMEM accumulator;
 //   4. writes rows 0..M-1 of the accumulator (fp32) to the workspace
-//      ([tile][split][M][256]),
-//      fences, and counts itself on the tile's counter;
+//      ([tile][split][M][256]), fences, and counts itself on the tile's
+//      counter (atomicInc with wrap-around: the last arrival puts it back to
+//      zero, so the counters stay zero between calls);
 //   5. the last CTA of a tile to arrive sums the split partials in split
 //      order (deterministic), applies s_a[m] * s_w[n] and writes BF16.
-// The tile counters live in the workspace and are zeroed by the quantize
-// kernel of the same call, so no state carries over between calls.
 //
 // Every wait is bounded; see gemm_tiled.cuh.
 #pragma once
@@ -33,6 +38,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace mfp8 {
 namespace skinny {
@@ -43,6 +49,8 @@ constexpr int BK = 128;
 constexpr int MMA_K = 32;
 constexpr int kThreads = 192;
 constexpr int kMaxM = 128;    // all four epilogue warps read their TMEM lanes
+constexpr int kMaxFusedM = 16;
+constexpr int kMaxSplits = 16;
 
 template <int STAGES>
 struct Layout {
@@ -54,18 +62,28 @@ struct Layout {
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 2;  // full, empty, tfull, drain
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem holder, abort, last flag
-    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+    static constexpr int SCALE_OFF = MISC_OFF + 16;          // amax bits, s, 1/s  [kMaxFusedM] each
+    static constexpr int SMEM_BYTES = SCALE_OFF + 3 * kMaxFusedM * 4 + 1024;
     static constexpr int TMEM_COLS = BN;
 };
 
-// A stage's transaction count is the whole box, rows filled with zeros
-// included.
-template <int STAGES>
+struct Args {
+    const __nv_bfloat16* X;  // QUANT: activations [M, K]
+    const float* s_a;        // !QUANT: scales from the quantize kernel
+    const float* s_w;
+    __nv_bfloat16* Y;
+    float* partial;
+    unsigned int* counters;
+    uint8_t* x8_out;         // QUANT: optional copy of the codes (tile 0 writes them)
+    float* sa_out;           // QUANT: optional copy of the scales
+    int M, N, K;
+    int weights_static;
+};
+
+template <int STAGES, bool QUANT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                   const float* __restrict__ s_a, const float* __restrict__ s_w,
-                   __nv_bfloat16* __restrict__ Y, float* __restrict__ partial, unsigned int* __restrict__ counters,
-                   int M, int N, int K, int weights_static) {
+                   const Args args) {
     using L = Layout<STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -80,7 +98,11 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+    uint32_t* amax_sm = reinterpret_cast<uint32_t*>(smem + L::SCALE_OFF);
+    float* s_sm = reinterpret_cast<float*>(amax_sm + kMaxFusedM);
+    float* r_sm = s_sm + kMaxFusedM;
 
+    const int M = args.M, N = args.N, K = args.K;
     const uint32_t warp = warp_id_sync();
     const uint32_t lane = lane_id();
     const int splits = int(gridDim.x);
@@ -91,10 +113,12 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     const int kb_begin = int((int64_t(kb_total) * split) / splits);
     const int kb_end = int((int64_t(kb_total) * (split + 1)) / splits);
     const int nkb = kb_end - kb_begin;  // >= 1 (host keeps splits <= kb_total)
+    const int prologue = nkb < STAGES ? nkb : STAGES;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
+            // QUANT: the four code-writing warps arrive too.
+            mbar_init(full_bar(s), QUANT ? 5 : 1);
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(tfull_bar, 1);
@@ -102,8 +126,22 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tmX);
+        if (!QUANT) tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
+    }
+    if (QUANT) {
+        // Code rows >= M stay zero in every ring slot; rows < M are rewritten
+        // for each k-block.  The row absmax starts at zero.
+        const int pad_chunks = (BM - M) * (BK / 16);
+        for (int i = int(threadIdx.x); i < STAGES * pad_chunks; i += kThreads) {
+            const int s = i / pad_chunks;
+            const int rem = i % pad_chunks;
+            const int row = M + rem / (BK / 16), chunk = rem % (BK / 16);
+            *reinterpret_cast<uint4*>(smem + L::A_OFF + s * L::A_BYTES + row * BK + chunk * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (threadIdx.x < kMaxFusedM) amax_sm[threadIdx.x] = 0u;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zero rows -> tensor-core reads
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), L::TMEM_COLS);
@@ -113,36 +151,77 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    // The next call's quantize kernel may start launching; it waits for this
+    // grid to finish before it touches memory.
+    grid_launch_dependents();
+
+    if (QUANT) {
+        // Weights first (static weights do not depend on the previous kernel).
+        if (threadIdx.x == 0) {
+            const uint64_t policy_w = l2_policy_evict_first();
+            if (!args.weights_static) grid_dependency_wait();
+            for (int i = 0; i < prologue; ++i) {
+                mbar_arrive_expect_tx(full_bar(i), L::B_BYTES);
+                tma_load_2d_hint(sB + i * L::B_BYTES, &tmW, full_bar(i), (kb_begin + i) * BK, n0, policy_w);
+            }
+        }
+        // X comes from earlier work on the stream.  Row absmax over all of K.
+        grid_dependency_wait();
+        const int groups = K / 8;
+        uint32_t run_max = 0;
+        int run_row = -1;
+        for (int e = int(threadIdx.x); e < M * groups; e += kThreads) {
+            const int m = e / groups;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(args.X + int64_t(m) * K) + (e % groups));
+            const uint32_t a = absmax_bits_u4(v, 0u);
+            const uint32_t a16 = max(a & 0xffffu, a >> 16);
+            if (m != run_row) {
+                if (run_row >= 0) atomicMax(amax_sm + run_row, run_max);
+                run_row = m;
+                run_max = 0;
+            }
+            run_max = max(run_max, a16);
+        }
+        if (run_row >= 0) atomicMax(amax_sm + run_row, run_max);
+        __syncthreads();
+        if (int(threadIdx.x) < M) {
+            const float s = scale_from_absmax_bits(amax_sm[threadIdx.x]);
+            s_sm[threadIdx.x] = s;
+            r_sm[threadIdx.x] = __frcp_rn(s);
+            if (args.sa_out && tile == 0 && split == 0) args.sa_out[threadIdx.x] = s;
+        }
+        __syncthreads();
+    }
 
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t policy_w = l2_policy_evict_first();
-            uint32_t issued_mask = 0, issued_parity = 0;
-            const int prologue = nkb < STAGES ? nkb : STAGES;
-            // Weights first: they do not depend on the previous kernel when
-            // the caller declared them static.
-            if (!weights_static) grid_dependency_wait();
-            for (int i = 0; i < prologue; ++i) {
-                mbar_arrive_expect_tx(full_bar(i), L::STAGE_BYTES);
-                tma_load_2d_hint(sB + i * L::B_BYTES, &tmW, full_bar(i), (kb_begin + i) * BK, n0, policy_w);
+            uint32_t issued_parity = 0;
+            if (!QUANT) {
+                if (!args.weights_static) grid_dependency_wait();
+                for (int i = 0; i < prologue; ++i) {
+                    mbar_arrive_expect_tx(full_bar(i), L::STAGE_BYTES);
+                    tma_load_2d_hint(sB + i * L::B_BYTES, &tmW, full_bar(i), (kb_begin + i) * BK, n0, policy_w);
+                }
+                grid_dependency_wait();  // the codes come from the quantize kernel
+                for (int i = 0; i < prologue; ++i)
+                    tma_load_2d(sA + i * L::A_BYTES, &tmX, full_bar(i), (kb_begin + i) * BK, 0);
             }
-            grid_dependency_wait();  // the codes come from the quantize kernel
-            for (int i = 0; i < prologue; ++i) {
-                tma_load_2d(sA + i * L::A_BYTES, &tmX, full_bar(i), (kb_begin + i) * BK, 0);
-                issued_mask |= 1u << i;
-            }
+            uint32_t issued_mask = (1u << prologue) - 1u;
             int stage = prologue % STAGES;
             uint32_t phase = prologue == STAGES ? 1u : 0u;
             for (int i = prologue; i < nkb; ++i) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) break;
-                mbar_arrive_expect_tx(full_bar(stage), L::STAGE_BYTES);
+                mbar_arrive_expect_tx(full_bar(stage), QUANT ? L::B_BYTES : L::STAGE_BYTES);
                 tma_load_2d_hint(sB + stage * L::B_BYTES, &tmW, full_bar(stage), (kb_begin + i) * BK, n0, policy_w);
-                tma_load_2d(sA + stage * L::A_BYTES, &tmX, full_bar(stage), (kb_begin + i) * BK, 0);
+                if (!QUANT) tma_load_2d(sA + stage * L::A_BYTES, &tmX, full_bar(stage), (kb_begin + i) * BK, 0);
                 issued_mask |= 1u << stage;
                 issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (*abort_flag) {
+                // Only the weight copies' bytes are outstanding; a slot whose
+                // code writers gave up simply never completes its phase.
                 volatile int no_abort = 0;
                 for (int s = 0; s < STAGES; ++s)
                     if (issued_mask & (1u << s))
@@ -177,12 +256,42 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             }
         }
     } else {
-        // Warp w reads TMEM lanes [32 (w % 4), 32 (w % 4) + 32): token rows.
         const uint32_t q = warp & 3u;
+        if (QUANT) {
+            // Warps 2-5 write the codes of each k-block into the ring slot the
+            // weights of that k-block land in: M rows x 16 groups of 8.
+            const int t = int(threadIdx.x) - 64;  // 0..127
+            const bool write_out = args.x8_out != nullptr && tile == 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int i = 0; i < nkb; ++i) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) break;
+                uint8_t* a_tile = smem + L::A_OFF + stage * L::A_BYTES;
+                const int kb = kb_begin + i;
+                for (int e = t; e < M * (BK / 8); e += 128) {
+                    const int m = e / (BK / 8);
+                    const int kc = (e % (BK / 8)) * 8;  // column within the k-block
+                    const int k = kb * BK + kc;
+                    uint2 code = make_uint2(0u, 0u);
+                    if (k < K) {
+                        code = quantize8(__ldg(reinterpret_cast<const uint4*>(args.X + int64_t(m) * K + k)), s_sm[m],
+                                         r_sm[m]);
+                        if (write_out) *reinterpret_cast<uint2*>(args.x8_out + int64_t(m) * K + k) = code;
+                    }
+                    const int chunk = (kc >> 4) ^ (m & 7);
+                    *reinterpret_cast<uint2*>(a_tile + m * BK + chunk * 16 + (kc & 15)) = code;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // codes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full_bar(stage));
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        // Warp w reads TMEM lanes [32 (w % 4), 32 (w % 4) + 32): token rows.
         const int m = int(q * 32 + lane);
         if (int(q * 32) < M && mbar_wait(tfull_bar, 0, abort_flag)) {
             tc_fence_after();
-            float* dst = partial + ((int64_t(tile) * splits + split) * M + m) * BN;
+            float* dst = args.partial + ((int64_t(tile) * splits + split) * M + m) * BN;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
                 uint32_t r[32];
@@ -205,22 +314,56 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     __syncthreads();
     if (threadIdx.x == 0 && !*abort_flag) {
         __threadfence();
-        const unsigned int prev = atomicAdd(counters + tile, 1u);
+        // Wraps back to zero on the last arrival.
+        const unsigned int prev = atomicInc(args.counters + tile, unsigned(splits - 1));
         *last_flag = (prev == unsigned(splits - 1)) ? 1 : 0;
     }
     __syncthreads();
     if (*last_flag) {
         __threadfence();
-        grid_dependency_wait();  // s_a comes from the quantize kernel
-        const int cols = min(BN, N - n0);
-        for (int e = int(threadIdx.x); e < M * cols; e += kThreads) {
-            const int m = e / cols;
-            const int c = e % cols;
-            const float* src = partial + (int64_t(tile) * splits * M + m) * BN + c;
-            float acc = 0.0f;
-            for (int p = 0; p < splits; ++p) acc += __ldcg(src + int64_t(p) * M * BN);
-            const int n = n0 + c;
-            Y[int64_t(m) * N + n] = __float2bfloat16_rn(acc * __ldcg(s_a + m) * __ldg(s_w + n));
+        if (!QUANT) grid_dependency_wait();  // s_a comes from the quantize kernel
+        // Every (row, 4 columns) item loads its splits' float4s at once, two
+        // items per round, so the reads overlap; sums keep split order.
+        const int cols = min(BN, N - n0);  // a multiple of 8
+        const int c4 = cols / 4;
+        const int items = M * c4;
+        const int64_t stride4 = int64_t(M) * BN / 4;
+        const float4* base4 = reinterpret_cast<const float4*>(args.partial + int64_t(tile) * splits * M * BN);
+        for (int e0 = int(threadIdx.x); e0 < items; e0 += 2 * kThreads) {
+            float4 v[2][kMaxSplits];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * kThreads;
+                const int m = e / c4, c = (e % c4) * 4;
+                const float4* src = base4 + (int64_t(m) * BN + c) / 4;
+#pragma unroll
+                for (int j = 0; j < kMaxSplits; ++j)
+                    v[u][j] = (e < items && j < splits) ? __ldcg(src + j * stride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * kThreads;
+                if (e >= items) continue;
+                const int m = e / c4, c = (e % c4) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < kMaxSplits; ++j)
+                    if (j < splits) {
+                        acc.x += v[u][j].x;
+                        acc.y += v[u][j].y;
+                        acc.z += v[u][j].z;
+                        acc.w += v[u][j].w;
+                    }
+                const int n = n0 + c;
+                const float sa = QUANT ? s_sm[m] : __ldcg(args.s_a + m);
+                const float4 sw = __ldg(reinterpret_cast<const float4*>(args.s_w + n));
+                __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * sa * sw.x, acc.y * sa * sw.y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * sa * sw.z, acc.w * sa * sw.w);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t*>(&lo);
+                pk.y = *reinterpret_cast<uint32_t*>(&hi);
+                *reinterpret_cast<uint2*>(args.Y + int64_t(m) * N + n) = pk;
+            }
         }
     }
 

@@ -109,6 +109,9 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
+    // The next call's quantize kernel may start launching; it waits for this
+    // grid to finish before it touches memory.
+    grid_launch_dependents();
     // X8 and s_a may come from the quantize kernel launched just before.
     grid_dependency_wait();
 

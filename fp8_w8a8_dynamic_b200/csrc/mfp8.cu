@@ -17,7 +17,6 @@
 #include "quant.cuh"
 #include "gemm_tiled.cuh"
 #include "gemm_skinny.cuh"
-#include "gemm_decode.cuh"
 #include "gemm_pair.cuh"
 
 namespace mfp8 {
@@ -98,6 +97,25 @@ mfp8_status launch_status() {
 
 // ------------------------------------------------------------- quantize --
 
+template <class Kern>
+mfp8_status launch_quant(Kern kern, bool dependent, int64_t R, const uint4* x, int64_t K, uint2* q, float* S,
+                         unsigned int* zero, int nzero, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(R));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, x, K, q, S, zero, nzero) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
 template <bool EARLY_TRIGGER>
 mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float* S, unsigned int* zero, int nzero,
                             cudaStream_t stream) {
@@ -105,14 +123,12 @@ mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float*
     const int64_t nvec = K / 8;
     const uint4* x = static_cast<const uint4*>(X);
     uint2* q = static_cast<uint2*>(Q);
-    const dim3 grid(static_cast<unsigned>(R)), block(kQuantThreads);
-    if (nvec <= 256) quant_rows_reg_kernel<1, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
-    else if (nvec <= 512) quant_rows_reg_kernel<2, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
-    else if (nvec <= 1024) quant_rows_reg_kernel<4, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
-    else if (nvec <= 1536) quant_rows_reg_kernel<6, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
-    else if (nvec <= 2048) quant_rows_reg_kernel<8, EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
-    else quant_rows_loop_kernel<EARLY_TRIGGER><<<grid, block, 0, stream>>>(x, K, q, S, zero, nzero);
-    return launch_status();
+    if (nvec <= 256) return launch_quant(quant_rows_reg_kernel<1, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
+    if (nvec <= 512) return launch_quant(quant_rows_reg_kernel<2, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
+    if (nvec <= 1024) return launch_quant(quant_rows_reg_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
+    if (nvec <= 1536) return launch_quant(quant_rows_reg_kernel<6, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
+    if (nvec <= 2048) return launch_quant(quant_rows_reg_kernel<8, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
+    return launch_quant(quant_rows_loop_kernel<EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
 }
 
 // Activations: the GEMM launched next may start its prologue early.  Block 0
@@ -188,6 +204,37 @@ mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K,
     return MFP8_OK;
 }
 
+// Clusters of `S` CTAs of `kern` (with `smem` bytes each) that the device
+// keeps resident at once.  Clusters are placed inside one GPC, so this can be
+// below (SMs x CTAs per SM) / S.  Cached per device and kernel.
+template <class Kern>
+int max_active_clusters(Kern kern, int S, int smem, int threads, int dev) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, const void*, int, int>, int> cache;
+    const auto key = std::make_tuple(dev, reinterpret_cast<const void*>(kern), S, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(S));
+    cfg.blockDim = dim3(unsigned(threads));
+    cfg.dynamicSmemBytes = size_t(smem);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cache[key] = n;
+    return n;
+}
+
 template <int BN, int STAGES>
 mfp8_status launch_pair_bn(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
                            int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
@@ -201,7 +248,9 @@ mfp8_status launch_pair_bn(const void* X8, const float* s_a, int64_t M, int64_t 
     if ((st = make_map_u8(&tmX, X8, M, K, pair::HALF)) != MFP8_OK) return st;
     if ((st = make_map_u8(&tmW, W8, N, K, BN / 2)) != MFP8_OK) return st;
     const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + BN - 1) / BN);
-    const int64_t max_pairs = info.sm_count / 2;
+    // The grid is persistent: only as many pairs as can be resident at once.
+    int64_t max_pairs = max_active_clusters(kern, 2, L::SMEM_BYTES, pair::kThreads, dev);
+    if (max_pairs <= 0 || max_pairs > info.sm_count / 2) max_pairs = info.sm_count / 2;
     const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
 
     cudaLaunchConfig_t cfg = {};
@@ -246,125 +295,13 @@ mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, 
     return launch_pair_bn<256, 6>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
 }
 
-constexpr int64_t kFusedMaxM = 64;
-
-
-#ifndef MFP8_DECODE_STAGES
-#define MFP8_DECODE_STAGES 4
-#endif
-
-// Clusters of `S` CTAs of `kern` (with `smem` bytes each) that the device
-// keeps resident at once.  Clusters are placed inside one GPC, so this can
-// be far below (SMs x CTAs per SM) / S.  Cached per device and shape.
-template <class Kern>
-int max_active_clusters(Kern kern, int S, int smem, int threads, int dev) {
-    static std::mutex mu;
-    static std::map<std::tuple<int, const void*, int, int>, int> cache;
-    const auto key = std::make_tuple(dev, reinterpret_cast<const void*>(kern), S, smem);
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(S));
-    cfg.blockDim = dim3(unsigned(threads));
-    cfg.dynamicSmemBytes = size_t(smem);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(S);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        n = 0;
-    }
-    cache[key] = n;
-    return n;
-}
-
-template <int MP, int ITEMS>
-mfp8_status launch_decode_mp(const void* X, int64_t M, int64_t K, const void* W8, const float* s_w, int64_t N,
-                             void* Y, bool weights_static, void* x8_out, float* sa_out, int dev,
-                             const DeviceInfo& info, cudaStream_t stream) {
-    (void)info;
-    constexpr int STAGES = MFP8_DECODE_STAGES;
-    using L = decode::Layout<MP, STAGES>;
-    auto kern = decode::gemm_decode_kernel<MP, STAGES, ITEMS>;
-    const int64_t tiles = (N + decode::BW - 1) / decode::BW;
-    const int64_t kb_total = (K + decode::BK - 1) / decode::BK;
-    if (tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    static bool attr_done[kMaxDevices] = {};
-    mfp8_status st = set_smem(kern, 227 * 1024, dev, attr_done);
-    if (st != MFP8_OK) return st;
-    // K-split S: the largest cluster size whose whole grid (tiles clusters)
-    // is resident in one wave; failing that, the S with the fewest waves.
-    auto nkb_cap_of = [&](int64_t s) { return (kb_total + s - 1) / s; };
-    int64_t best_S = 0, best_waves = INT64_MAX;
-    for (int64_t S = decode::kMaxCluster; S >= 1; --S) {
-        if (S > kb_total) continue;
-        const int64_t nkb_cap = nkb_cap_of(S);
-        const int smem = L::smem_bytes(int(nkb_cap));
-        if (smem > 227 * 1024) continue;
-        const int active = max_active_clusters(kern, int(S), smem, decode::kThreads, dev);
-        if (active <= 0) continue;
-        const int64_t waves = (tiles + active - 1) / active;
-        if (waves < best_waves) {
-            best_waves = waves;
-            best_S = S;
-        }
-        if (waves == 1) break;
-    }
-    if (best_S == 0) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    const int64_t S = best_S;
-    const int64_t nkb_cap = nkb_cap_of(S);
-    const int smem = L::smem_bytes(int(nkb_cap));
-    CUtensorMap tmW;
-    if ((st = make_map_u8(&tmW, W8, N, K, decode::BW)) != MFP8_OK) return st;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(S), unsigned(tiles));
-    cfg.blockDim = dim3(decode::kThreads);
-    cfg.dynamicSmemBytes = size_t(smem);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(S);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tmW, static_cast<const __nv_bfloat16*>(X), s_w,
-                           static_cast<__nv_bfloat16*>(Y), int(M), int(N), int(K), int(nkb_cap),
-                           weights_static ? 1 : 0, static_cast<uint8_t*>(x8_out), sa_out) != cudaSuccess) {
-        cudaGetLastError();
-        return MFP8_ERR_CUDA;
-    }
-    return MFP8_OK;
-}
-
-mfp8_status launch_fused(const void* X, int64_t M, int64_t K, const void* W8, const float* s_w, int64_t N,
-                         void* Y, bool weights_static, void* x8_out, float* sa_out, int dev,
-                         const DeviceInfo& info, cudaStream_t stream) {
-    if (M <= 16)
-        return launch_decode_mp<16, 16>(X, M, K, W8, s_w, N, Y, weights_static, x8_out, sa_out, dev, info, stream);
-    if (M <= 32)
-        return launch_decode_mp<32, 24>(X, M, K, W8, s_w, N, Y, weights_static, x8_out, sa_out, dev, info, stream);
-    if (M <= 64)
-        return launch_decode_mp<64, 24>(X, M, K, W8, s_w, N, Y, weights_static, x8_out, sa_out, dev, info, stream);
-    return MFP8_ERR_UNSUPPORTED_SHAPE;
-}
-
 constexpr int64_t kSkinnyMaxM = skinny::kMaxM;
+constexpr int64_t kFusedMaxM = skinny::kMaxFusedM;
 constexpr int kSkinnyStages = 4;
 
 int choose_path(int64_t M, int64_t N, int64_t K) {
-    (void)N;
     (void)K;
-    if (M <= 64) return MFP8_PATH_SPLITK;
+    if (M <= 64 && (N + 255) / 256 <= 4096) return MFP8_PATH_SPLITK;
     if (M < 256) return MFP8_PATH_TILED;
     return MFP8_PATH_PAIR;
 }
@@ -384,19 +321,26 @@ mfp8_status check_gemm_args(int64_t M, int64_t N, int64_t K, const void* W8, con
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// K-splits of the skinny kernel: as many CTAs as SMs, no CTA without k-blocks.
+// K-splits of the skinny kernel: as many CTAs as SMs, no CTA without
+// k-blocks, and at most 16 partials for the last CTA of a tile to add up.
 int64_t skinny_splits(int64_t N, int64_t K, int sm_count) {
     const int64_t tiles = (N + skinny::BN - 1) / skinny::BN;
     const int64_t kb_total = (K + skinny::BK - 1) / skinny::BK;
     int64_t splits = sm_count / tiles;
+    if (splits > 16) splits = 16;
     if (splits < 1) splits = 1;
     if (splits > kb_total) splits = kb_total;
     return splits;
 }
 
-// How one call uses the caller's workspace: the activation codes and scales
-// of the quantize pass, then (split-K) the fp32 partials [tile][split][M][256]
-// and one counter per tile; each region 256-byte aligned.
+// How one call uses the caller's workspace.  The split-K tile counters sit
+// at a fixed place, the first kCounterBytes, in every layout: they must stay
+// zero between calls whatever shapes and paths share the workspace.  Then
+// the activation codes and scales of the quantize pass, then the split-K
+// fp32 partials [tile][split][M][256]; each region 256-byte aligned.
+constexpr int64_t kMaxSplitKTiles = 4096;  // N <= 1M for the split-K path
+constexpr size_t kCounterBytes = size_t(kMaxSplitKTiles) * 4;
+
 struct Plan {
     size_t x8_off = 0, sa_off = 0, part_off = 0, cnt_off = 0, total = 0;
     int64_t tiles = 0, splits = 0;
@@ -404,7 +348,9 @@ struct Plan {
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, bool codes, bool split_k, int sm_count) {
     Plan p;
-    size_t off = 0;
+    if (!codes && !split_k) return p;  // nothing to keep: no workspace needed
+    size_t off = kCounterBytes;
+    p.cnt_off = 0;
     if (codes) {
         p.x8_off = off;
         off += round_up(size_t(M) * size_t(K), 256);
@@ -416,25 +362,42 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool codes, bool split_k, int sm
         p.splits = skinny_splits(N, K, sm_count);
         p.part_off = off;
         off += round_up(size_t(p.tiles * p.splits) * size_t(M) * skinny::BN * 4, 256);
-        p.cnt_off = off;
-        off += round_up(size_t(p.tiles) * 4, 256);
     }
     p.total = off;
     return p;
 }
 
-mfp8_status launch_skinny(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+// QUANT: X is BF16 and the kernel quantizes it (M <= 16); otherwise X8/s_a
+// are the codes of the quantize pass.
+template <bool QUANT>
+mfp8_status launch_skinny(const void* X, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
                           int64_t N, void* Y, float* partial, unsigned int* counters, const Plan& plan,
-                          bool weights_static, bool dependent, int dev, cudaStream_t stream) {
+                          bool weights_static, bool dependent, void* x8_out, float* sa_out, int dev,
+                          cudaStream_t stream) {
     using L = skinny::Layout<kSkinnyStages>;
-    auto kern = skinny::gemm_skinny_kernel<kSkinnyStages>;
+    auto kern = skinny::gemm_skinny_kernel<kSkinnyStages, QUANT>;
     static bool attr_done[kMaxDevices] = {};
     mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
     if (st != MFP8_OK) return st;
     CUtensorMap tmX, tmW;
-    if ((st = make_map_u8(&tmX, X8, M, K, skinny::BM)) != MFP8_OK) return st;
     if ((st = make_map_u8(&tmW, W8, N, K, skinny::BN)) != MFP8_OK) return st;
+    if (QUANT) tmX = tmW;  // unused
+    else if ((st = make_map_u8(&tmX, X, M, K, skinny::BM)) != MFP8_OK) return st;
     if (plan.tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
+
+    skinny::Args args;
+    args.X = static_cast<const __nv_bfloat16*>(X);
+    args.s_a = s_a;
+    args.s_w = s_w;
+    args.Y = static_cast<__nv_bfloat16*>(Y);
+    args.partial = partial;
+    args.counters = counters;
+    args.x8_out = static_cast<uint8_t*>(x8_out);
+    args.sa_out = sa_out;
+    args.M = int(M);
+    args.N = int(N);
+    args.K = int(K);
+    args.weights_static = weights_static ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(plan.splits), unsigned(plan.tiles));
@@ -446,8 +409,7 @@ mfp8_status launch_skinny(const void* X8, const float* s_a, int64_t M, int64_t K
     attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, s_a, s_w, static_cast<__nv_bfloat16*>(Y), partial, counters,
-                           int(M), int(N), int(K), weights_static ? 1 : 0) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, args) != cudaSuccess) {
         cudaGetLastError();
         return MFP8_ERR_CUDA;
     }
@@ -464,9 +426,9 @@ mfp8_status run_gemm(const void* X8, const float* s_a, int64_t M, int64_t K, con
     if (path == MFP8_PATH_PAIR) return launch_pair(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
     if (path == MFP8_PATH_SPLITK) {
         uint8_t* base = static_cast<uint8_t*>(ws);
-        return launch_skinny(X8, s_a, M, K, W8, s_w, N, Y, reinterpret_cast<float*>(base + plan.part_off),
-                             reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static, dependent,
-                             dev, stream);
+        return launch_skinny<false>(X8, s_a, M, K, W8, s_w, N, Y, reinterpret_cast<float*>(base + plan.part_off),
+                                    reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static,
+                                    dependent, nullptr, nullptr, dev, stream);
     }
     return MFP8_ERR_INVALID_ARG;
 }
@@ -534,6 +496,8 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     if (st != MFP8_OK) return st;
     if (path < MFP8_PATH_AUTO || path > MFP8_PATH_FUSED) return MFP8_ERR_INVALID_ARG;
     if ((flags & ~MFP8_FLAG_STATIC_WEIGHTS) != 0) return MFP8_ERR_INVALID_ARG;
+    if ((path == MFP8_PATH_SPLITK || path == MFP8_PATH_FUSED) && (N + 255) / 256 > 4096)
+        return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (path == MFP8_PATH_SPLITK && M > kSkinnyMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (path == MFP8_PATH_FUSED && M > kFusedMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
@@ -550,27 +514,29 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     }
     if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
     const bool weights_static = (flags & MFP8_FLAG_STATIC_WEIGHTS) != 0;
-    const bool split_k = path == MFP8_PATH_SPLITK;
-    Plan plan;
-    if (path != MFP8_PATH_FUSED) {
-        plan = make_plan(M, N, K, X_fp8_out == nullptr, split_k, sm_count_for_sizing());
-        if (plan.total > 0) {
-            if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
-            if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
-            if (ranges_overlap(workspace, plan.total, Y_bf16, size_t(M * N * 2)) ||
-                ranges_overlap(workspace, plan.total, X_bf16, size_t(M * K * 2)))
-                return MFP8_ERR_INVALID_ARG;
-        }
+    // Split-K with the quantize pass, or (FUSED, M <= 16) the split-K kernel
+    // that quantizes X itself: no codes in the workspace, no extra launch.
+    const bool fused = path == MFP8_PATH_FUSED;
+    const bool split_k = path == MFP8_PATH_SPLITK || fused;
+    const Plan plan = make_plan(M, N, K, X_fp8_out == nullptr && !fused, split_k, sm_count_for_sizing());
+    if (plan.total > 0) {
+        if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
+        if (ranges_overlap(workspace, plan.total, Y_bf16, size_t(M * N * 2)) ||
+            ranges_overlap(workspace, plan.total, X_bf16, size_t(M * K * 2)))
+            return MFP8_ERR_INVALID_ARG;
     }
 
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (path == MFP8_PATH_FUSED)
-        return launch_fused(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, weights_static, X_fp8_out, x_scale_out, dev,
-                            info, s);
     uint8_t* base = static_cast<uint8_t*>(workspace);
+    if (fused)
+        return launch_skinny<true>(X_bf16, nullptr, M, K, W_fp8, w_scale, N, Y_bf16,
+                                   reinterpret_cast<float*>(base + plan.part_off),
+                                   reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static,
+                                   /*dependent=*/true, X_fp8_out, x_scale_out, dev, s);
     void* X8 = X_fp8_out ? X_fp8_out : base + plan.x8_off;
     float* s_a = x_scale_out ? x_scale_out : reinterpret_cast<float*>(base + plan.sa_off);
     unsigned int* counters = split_k ? reinterpret_cast<unsigned int*>(base + plan.cnt_off) : nullptr;
@@ -597,7 +563,7 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
     mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
     if (st != MFP8_OK) return st;
     if (path < MFP8_PATH_AUTO || path > MFP8_PATH_PAIR) return MFP8_ERR_INVALID_ARG;
-    if (path == MFP8_PATH_SPLITK && M > kSkinnyMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_SPLITK && (M > kSkinnyMaxM || (N + 255) / 256 > 4096)) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_fp8 || !x_scale) return MFP8_ERR_INVALID_ARG;
     if (!aligned16(X_fp8) || !aligned16(x_scale)) return MFP8_ERR_MISALIGNED;
@@ -616,7 +582,7 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (plan.total > 0) {
+    if (split_k) {
         if (cudaMemsetAsync(static_cast<uint8_t*>(workspace) + plan.cnt_off, 0, size_t(plan.tiles) * 4, s) !=
             cudaSuccess) {
             cudaGetLastError();

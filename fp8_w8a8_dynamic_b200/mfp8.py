@@ -164,9 +164,11 @@ def quantize_act(X, stream=None):
 
 
 def workspace_for(M, N, K, device):
+    """A zero-filled workspace for mfp8_linear at these sizes (the split-K
+    counters in it must start at zero; every call leaves them zero)."""
     import torch
     nbytes = mfp8_linear_workspace_bytes(M, N, K)
-    return torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=device)
+    return torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=device)
 
 
 def linear(X, W8, w_scale, out=None, workspace=None, path=PATH_AUTO, x8_out=None, xs_out=None,
@@ -194,7 +196,7 @@ def gemm(X8, x_scale, W8, w_scale, out=None, path=PATH_AUTO, workspace=None, str
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=X8.device)
     if workspace is None:
-        workspace = torch.empty((max(mfp8_gemm_workspace_bytes(M, N, K), 16),), dtype=torch.uint8,
+        workspace = torch.zeros((max(mfp8_gemm_workspace_bytes(M, N, K), 16),), dtype=torch.uint8,
                                 device=X8.device)
     _check(mfp8_gemm(_ptr(X8), _ptr(x_scale), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), _ptr(workspace),
                      workspace.numel(), path, _stream_handle(stream)), "mfp8_gemm")

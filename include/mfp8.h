@@ -100,10 +100,13 @@ MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *            mfp8_quantize_weight, read only.
  *   Y_bf16   [M, N] bf16, written.  Must not overlap any input.
  *   workspace / workspace_bytes: device scratch of at least
- *            mfp8_linear_workspace_bytes(M, N, K) bytes, 16-byte aligned.
- *            Its contents on entry do not matter (the call initialises what
- *            it uses); they are garbage on exit.  Calls that may run at the
- *            same time need separate workspaces.
+ *            mfp8_linear_workspace_bytes(M, N, K) bytes, 16-byte aligned,
+ *            ZERO-FILLED before its first use (e.g. one cudaMemset).  It
+ *            holds the activation codes and, for decode sizes, the split-K
+ *            partials and one counter per output tile; every call leaves the
+ *            counters at zero, so the zero-fill is needed once, and again
+ *            only after a call reported MFP8_ERR_TIMEOUT.  Calls that may run
+ *            at the same time need separate workspaces.
  * The activation quantization (per-token scale + e4m3 codes) happens inside
  * this call: its codes and scales are bit-identical to mfp8_quantize_act.
  * Outputs are within |y - y_ref| <= 2^-7 |y_ref| + 1e-5 * sum_k |a_k w_k| s_a s_w
@@ -119,7 +122,7 @@ typedef enum {
     MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
     MFP8_PATH_SPLITK = 2, /* quantize pass, then the weight-streaming split-K GEMM over all SMs (M <= 128) */
     MFP8_PATH_PAIR = 3,   /* quantize pass, then the 256-row-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
-    MFP8_PATH_FUSED = 4   /* one kernel: on-chip quantize + cluster split-K GEMM (M <= 64), no workspace */
+    MFP8_PATH_FUSED = 4   /* one kernel: split-K GEMM that quantizes X on chip (M <= 16) */
 } mfp8_path;
 
 /* Flags for mfp8_linear_ex. */
@@ -136,9 +139,10 @@ typedef enum {
  * x_scale_out [M]; pass NULL for none).  Used to test each kernel on the
  * same shapes, to check that the activation bytes of every path are
  * bit-identical to mfp8_quantize_act, and by callers with static weights.
- * MFP8_PATH_FUSED quantizes X inside the GEMM kernel and needs no workspace.
- * When X_fp8_out is given, the quantize pass writes the codes there instead
- * of the workspace.  Returns MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel
+ * MFP8_PATH_FUSED quantizes X inside the split-K kernel (every CTA takes the
+ * row scales itself): one launch, and no codes in the workspace.  When
+ * X_fp8_out is given, the codes are written there as well (the quantize
+ * pass writes them there instead of the workspace).  Returns MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel
  * cannot take these sizes, MFP8_ERR_INVALID_ARG for an unknown path or flag. */
 MFP8_API mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K,
                            const void* W_fp8, const float* w_scale, int64_t N,

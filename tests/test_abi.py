@@ -50,16 +50,18 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_bytes(lib):
-    # X8 [M, K] then s_a [M], each rounded up to 256 bytes; for M <= 128 also
-    # the split-K partials [tiles][splits][M][256] fp32 and one counter per tile
-    # (sized for 148 SMs when no device is present)
-    assert mfp8.mfp8_linear_workspace_bytes(300, 4096, 4096) == 300 * 4096 + 1280
+    # 16 KB of split-K counters first (a fixed place in every layout), then X8
+    # [M, K] and s_a [M], each rounded up to 256 bytes, then for M <= 128 the
+    # split-K partials [tiles][splits][M][256] fp32 (sized for 148 SMs when no
+    # device is present)
+    C = 16384
+    assert mfp8.mfp8_linear_workspace_bytes(300, 4096, 4096) == C + 300 * 4096 + 1280
     tiles, splits = 16, 9  # N = 4096 in 256-wide tiles; 148 // 16 K-splits
-    assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == 65536 + 256 + tiles * splits * 16 * 1024 + 256
-    assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == tiles * splits * 16 * 1024 + 256
+    assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == C + 65536 + 256 + tiles * splits * 16 * 1024
+    assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == C + tiles * splits * 16 * 1024
     assert mfp8.mfp8_gemm_workspace_bytes(300, 4096, 4096) == 0
     # one K-block only: one split
-    assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == 256 + 256 + 3 * 1024 + 256
+    assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == C + 256 + 256 + 3 * 1024
     assert mfp8.mfp8_linear_workspace_bytes(0, 8, 48) == 0
     assert mfp8.mfp8_linear_workspace_bytes(4, 8, -1) == 0
 
@@ -98,7 +100,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert call(flags=2) == mfp8.ERR_INVALID_ARG
     assert call(path=7) == mfp8.ERR_INVALID_ARG
     assert call(path=5) == mfp8.ERR_INVALID_ARG
-    assert call(path=mfp8.PATH_FUSED, M=65) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(path=mfp8.PATH_FUSED, M=17) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(ws=None) == mfp8.ERR_WORKSPACE  # split-K partials
     assert call(path=mfp8.PATH_SPLITK, M=129) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
