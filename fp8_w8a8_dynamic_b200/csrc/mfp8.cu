@@ -442,6 +442,40 @@ int sm_count_for_sizing() {
     return 148;  // B200
 }
 
+// Scratch of mfp8_linear_noalloc: one fixed array per device, part of the
+// module's own global memory, so that entry point allocates nothing.  It is
+// for callers that cannot call an allocator where they call the Linear: a C
+// host with no device allocator of its own, or one whose memory is planned
+// in full up front (a fixed budget per GPU).  Every call on a device uses
+// the same bytes, so two calls that can be in flight at once race.
+constexpr size_t kStaticWsBytes = MFP8_STATIC_WORKSPACE_BYTES;
+static_assert(kStaticWsBytes >= kCounterBytes + 256, "static scratch must hold the split-K counters");
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+// Once per device: the array's device address, and its split-K counters set
+// to zero (later calls leave them at zero).  The memset runs on the legacy
+// stream and is waited for here, so it is ordered before every later call on
+// any stream.  This is the only place the entry point synchronises.
+mfp8_status static_workspace(int dev, void** out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_static_ws_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return MFP8_ERR_CUDA;
+        }
+        if (cudaMemset(p, 0, kCounterBytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+            cudaGetLastError();
+            return MFP8_ERR_CUDA;
+        }
+        g_static_ws_ptr[dev] = p;
+    }
+    *out = g_static_ws_ptr[dev];
+    return MFP8_OK;
+}
+
 __global__ void bounded_wait_kernel(uint64_t limit_ns) {
     __shared__ __align__(8) uint64_t bar;
     __shared__ int abort_flag;
@@ -550,6 +584,20 @@ mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K, const void* W_
                         int64_t N, void* Y_bf16, void* workspace, size_t workspace_bytes_given, void* stream) {
     return mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes_given,
                           MFP8_PATH_AUTO, 0, nullptr, nullptr, stream);
+}
+
+mfp8_status mfp8_linear_noalloc(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
+                               int64_t N, void* Y_bf16, void* stream) {
+    mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
+    if (st != MFP8_OK || M == 0) return st;
+    if (mfp8_linear_workspace_bytes(M, N, K) > kStaticWsBytes) return MFP8_ERR_WORKSPACE;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
+    void* ws = nullptr;
+    if ((st = static_workspace(dev, &ws)) != MFP8_OK) return st;
+    return mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, ws, kStaticWsBytes, MFP8_PATH_AUTO, 0,
+                          nullptr, nullptr, stream);
 }
 
 size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {

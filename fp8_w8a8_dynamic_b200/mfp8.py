@@ -53,6 +53,7 @@ def lib():
             "mfp8_linear_workspace_bytes": (sz, [i64, i64, i64]),
             "mfp8_linear": (i32, [P, i64, i64, P, P, i64, P, P, sz, P]),
             "mfp8_linear_ex": (i32, [P, i64, i64, P, P, i64, P, P, sz, i32, i32, P, P, P]),
+            "mfp8_linear_noalloc": (i32, [P, i64, i64, P, P, i64, P, P]),
             "mfp8_gemm_workspace_bytes": (sz, [i64, i64, i64]),
             "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, P, sz, i32, P]),
             "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
@@ -91,6 +92,13 @@ def mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace
                    X_fp8_out, x_scale_out, stream=0):
     return lib().mfp8_linear_ex(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes,
                                 path, flags, X_fp8_out, x_scale_out, stream)
+
+
+def mfp8_linear_noalloc(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, stream=0):
+    return lib().mfp8_linear_noalloc(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, stream)
+
+
+STATIC_WORKSPACE_BYTES = 16 << 20  # MFP8_STATIC_WORKSPACE_BYTES
 
 
 def mfp8_gemm_workspace_bytes(M, N, K):

@@ -150,6 +150,32 @@ MFP8_API mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K,
                            int path, int flags, void* X_fp8_out, float* x_scale_out,
                            void* stream);
 
+/* Size of the library's own scratch for mfp8_linear_noalloc: 16 MiB per device. */
+#define MFP8_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/* mfp8_linear without a caller workspace: the scratch is a fixed array of
+ * MFP8_STATIC_WORKSPACE_BYTES in the library's device memory, one per
+ * device.  The pages describe no counterpart: this serves callers that
+ * cannot allocate at the call site (a C host without its own device
+ * allocator, or one that plans all device memory up front).  The call
+ * allocates no memory.
+ *   Arguments, results and tolerance: as mfp8_linear (kernel choice AUTO).
+ *   Sizes whose mfp8_linear_workspace_bytes(M, N, K) exceeds
+ *   MFP8_STATIC_WORKSPACE_BYTES are rejected with MFP8_ERR_WORKSPACE before
+ *   any device work (e.g. M <= 64 fits every projection up to N, K = 12288;
+ *   the quantized activations of larger M need M * K bytes).
+ *   Set-up: the first call on each device looks up the array's address and
+ *   zeroes its counters, then waits for the device (cudaDeviceSynchronize).
+ *   Make that first call before any stream capture begins.
+ *   Concurrency: every call on a device shares the one scratch array.  Calls
+ *   that may be in flight at the same time (different streams, or host
+ *   threads) race and give wrong results; serialise them, e.g. on one stream.
+ *   After a call reported MFP8_ERR_TIMEOUT the next call still starts from
+ *   zeroed counters (the quantize pass clears them). */
+MFP8_API mfp8_status mfp8_linear_noalloc(const void* X_bf16, int64_t M, int64_t K,
+                                const void* W_fp8, const float* w_scale, int64_t N,
+                                void* Y_bf16, void* stream);
+
 /* Workspace bytes mfp8_gemm needs at these sizes on the current device
  * (the split-K partials and counters; 0 when no kernel choice needs any). */
 MFP8_API size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);

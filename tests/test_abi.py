@@ -36,6 +36,12 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(raw, name), f"{name} declared in mfp8.h but not exported"
 
 
+def test_static_workspace_size_matches_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define MFP8_STATIC_WORKSPACE_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == mfp8.STATIC_WORKSPACE_BYTES
+
+
 def test_library_does_not_need_libcuda():
     # The driver is reached through cudaGetDriverEntryPoint at run time.
     out = os.popen(f"ldd {mfp8.LIB_PATH}").read()
@@ -106,6 +112,11 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
     assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X
     assert call(M=0) == mfp8.OK
+    NA = mfp8.mfp8_linear_noalloc
+    assert NA(FAKE, 4, 64, FAKE * 2, FAKE * 3, 12, FAKE * 4, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert NA(FAKE, 0, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None) == mfp8.OK
+    # more than the library's fixed scratch: codes alone are 4096 * 8192 bytes
+    assert NA(FAKE, 4096, 8192, FAKE * 2, FAKE * 3, 64, FAKE * 4, None) == mfp8.ERR_WORKSPACE
     G = mfp8.mfp8_gemm
     assert G(None, FAKE, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_INVALID_ARG
     assert G(FAKE, FAKE * 9, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_WORKSPACE
