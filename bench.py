@@ -176,7 +176,8 @@ def time_graph(torch, fn, steps, warmup, dist_ctx):
     for _ in range(warmup):
         g.replay()
     torch.cuda.synchronize()
-    dist_ctx.barrier()
+    if dist_ctx is not None:
+        dist_ctx.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -184,62 +185,56 @@ def time_graph(torch, fn, steps, warmup, dist_ctx):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
-    dist_ctx.barrier()
     ms = e0.elapsed_time(e1)
     del g
+    if dist_ctx is None:
+        return ms
+    dist_ctx.barrier()
     return dist_ctx.max(ms)
 
 
-def kernel_times(torch, mfp8, layer, reps):
-    """Per-launch CUDA-event times of the GEMM kernel and of the quantize
-    kernel.  Each launch sits between two event-record nodes of one CUDA
-    graph, so the host's launch latency never shows up as a gap between the
-    events."""
-    x8 = {}
-    for mi, M in enumerate(layer.Ms):
-        for i, lin in enumerate(layer.lins):
-            x8[(M, i)] = mfp8.quantize_act(layer.x[(M, i)])
-    torch.cuda.synchronize()
+def kernel_times(torch, mfp8, layer, steps, warmup):
+    """Average launch duration of the GEMM kernel and of the quantize kernel
+    over the step's Linears.  Each is a CUDA graph of that kernel's launches
+    alone, one per Linear with nothing between them, timed with CUDA events
+    around `steps` replays on the launching stream; the average includes the
+    gaps between graph nodes, so it is an upper bound on a launch's own time.
+    The split-K workspaces are zero-filled once (every call leaves their
+    counters at zero)."""
     keys = [(mi, M, i, lin) for mi, M in enumerate(layer.Ms) for i, lin in enumerate(layer.lins)]
-    gws_of = {(M, i): torch.empty((max(16, mfp8.mfp8_gemm_workspace_bytes(M, lin.N, lin.K)),), dtype=torch.uint8,
+    x8 = {(M, i): mfp8.quantize_act(layer.x[(M, i)]) for (mi, M, i, lin) in keys}
+    gws_of = {(M, i): torch.zeros((max(16, mfp8.mfp8_gemm_workspace_bytes(M, lin.N, lin.K)),), dtype=torch.uint8,
                                   device=layer.x[(M, i)].device) for (mi, M, i, lin) in keys}
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in keys]
+    torch.cuda.synchronize()
 
-    def body(h):
-        for (mi, M, i, lin), e in zip(keys, ev):
+    def gemms(h):
+        for (mi, M, i, lin) in keys:
             s = layer.weight_set(mi)
             q8, qs = x8[(M, i)]
-            e[0].record()
-            st = mfp8.mfp8_quantize_act(layer.x[(M, i)].data_ptr(), M, lin.K, q8.data_ptr(), qs.data_ptr(), h)
-            e[1].record()
-            e[2].record()
             gws = gws_of[(M, i)]
-            st2 = mfp8.mfp8_gemm(q8.data_ptr(), qs.data_ptr(), M, lin.K, layer.w8[s][i].data_ptr(),
-                                 layer.sw[s][i].data_ptr(), lin.N, layer.y[(M, i)].data_ptr(),
-                                 gws.data_ptr(), gws.numel(), 0, h)
-            e[3].record()
-            if st != mfp8.OK or st2 != mfp8.OK:
-                raise mfp8.Mfp8Error(st or st2, "kernel timing")
+            st = mfp8.mfp8_gemm(q8.data_ptr(), qs.data_ptr(), M, lin.K, layer.w8[s][i].data_ptr(),
+                                layer.sw[s][i].data_ptr(), lin.N, layer.y[(M, i)].data_ptr(),
+                                gws.data_ptr(), gws.numel(), mfp8.PATH_AUTO, h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_gemm")
 
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        body(torch.cuda.current_stream().cuda_stream)
-    out = dict(gemm_ms=0.0, gemm_bytes=0, gemm_flops=0, gemm_n=0, quant_ms=0.0, quant_bytes=0, quant_n=0)
-    g.replay()
-    torch.cuda.synchronize()
-    for _ in range(reps):
-        g.replay()
-        torch.cuda.synchronize()
-        for (mi, M, i, lin), e in zip(keys, ev):
-            out["quant_ms"] += e[0].elapsed_time(e[1])
-            out["gemm_ms"] += e[2].elapsed_time(e[3])
-            out["quant_bytes"] += 3 * M * lin.K + 4 * M
-            out["gemm_bytes"] += lin.N * lin.K + 4 * lin.N + M * lin.K + 4 * M + 2 * M * lin.N
-            out["gemm_flops"] += 2 * M * lin.N * lin.K
-            out["gemm_n"] += 1
-            out["quant_n"] += 1
-    del g
-    return out
+    def quants(h):
+        for (mi, M, i, lin) in keys:
+            q8, qs = x8[(M, i)]
+            st = mfp8.mfp8_quantize_act(layer.x[(M, i)].data_ptr(), M, lin.K, q8.data_ptr(), qs.data_ptr(), h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_quantize_act")
+
+    n = len(keys)
+    gemm_ms = time_graph(torch, gemms, steps, warmup, None)
+    quant_ms = time_graph(torch, quants, steps, warmup, None)
+    paths = sorted({mfp8.mfp8_choose_path(M, lin.N, lin.K) for (mi, M, i, lin) in keys})
+    return dict(gemm_us=gemm_ms * 1e3 / (steps * n), quant_us=quant_ms * 1e3 / (steps * n), launches=steps * n,
+                gemm_bytes=sum(lin.N * lin.K + 4 * lin.N + M * lin.K + 4 * M + 2 * M * lin.N
+                               for (mi, M, i, lin) in keys) / n,
+                gemm_flops=sum(2 * M * lin.N * lin.K for (mi, M, i, lin) in keys) / n,
+                quant_bytes=sum(3 * M * lin.K + 4 * M for (mi, M, i, lin) in keys) / n,
+                kernel="+".join(mfp8.KERNEL_OF_PATH[p] for p in paths))
 
 
 def e2e_time(torch, mfp8, layer, steps, warmup, dist_ctx):
@@ -410,9 +405,9 @@ def main():
     step_ms = ms / args.steps
     value = wbytes * ctx.world * args.steps / (ms * 1e-3) / 1e9
 
-    kt = kernel_times(torch, mfp8, layer, reps=max(3, min(args.steps, 10)))
-    gemm_gbs = kt["gemm_bytes"] / (kt["gemm_ms"] * 1e-3) / 1e9
-    quant_gbs = kt["quant_bytes"] / (kt["quant_ms"] * 1e-3) / 1e9
+    kt = kernel_times(torch, mfp8, layer, steps=max(5, min(args.steps, 20)), warmup=args.warmup)
+    gemm_gbs = kt["gemm_bytes"] / (kt["gemm_us"] * 1e-6) / 1e9
+    quant_gbs = kt["quant_bytes"] / (kt["quant_us"] * 1e-6) / 1e9
 
     e2e_ms, h2d, d2h = e2e_time(torch, mfp8, layer, max(3, args.steps // 5), 3, ctx)
     e2e_val = wbytes * ctx.world * max(3, args.steps // 5) / (e2e_ms * 1e-3) / 1e9
@@ -430,15 +425,16 @@ def main():
         psteps = max(5, args.steps // 2)
         pms = time_graph(torch, lambda h: pl.step(mfp8, h), psteps, args.warmup, ctx)
         tflops = pl.flops_per_step() * psteps / (pms * 1e-3) / 1e12
-        pk = kernel_times(torch, mfp8, pl, reps=3)
-        g_tf = pk["gemm_flops"] / (pk["gemm_ms"] * 1e-3) / 1e12
+        pk = kernel_times(torch, mfp8, pl, steps=5, warmup=args.warmup)
+        g_tf = pk["gemm_flops"] / (pk["gemm_us"] * 1e-6) / 1e12
         fp8_peak = 2.0 * peaks["bf16_tflops"]
         prefill = {"metric": "FP8-dynamic Linear TFLOPS (M=2048, 7 Linears, quantize included)",
                    "value": round(tflops, 1), "unit": "TFLOP/s", "ms_per_step": round(pms / psteps, 4),
                    "frac_of_fp8_peak": round(tflops / fp8_peak, 4),
                    "roofline": {"bound": "tensor", "achieved": round(g_tf, 1), "peak": round(fp8_peak, 1),
                                 "unit": "TFLOP/s", "frac": round(g_tf / fp8_peak, 4), "traffic": None,
-                                "kernel": "gemm_tiled_kernel", "peak_source": f"{peaks['source']} bf16 x 2 (fp8/bf16 nominal ratio)"}}
+                                "kernel": pk["kernel"], "avg_launch_us": round(pk["gemm_us"], 3),
+                                "peak_source": f"{peaks['source']} bf16 x 2 (fp8/bf16 nominal ratio)"}}
         del pl
         torch.cuda.empty_cache()
 
@@ -456,10 +452,11 @@ def main():
         "frac_of_hbm": round(value / ctx.world / peaks["hbm_gbs"], 4),
         "roofline": {"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": None,
-                     "kernel": "gemm_skinny_kernel", "launches_timed": kt["gemm_n"],
-                     "avg_launch_us": round(kt["gemm_ms"] * 1e3 / kt["gemm_n"], 3),
+                     "kernel": kt["kernel"], "launches_timed": kt["launches"],
+                     "avg_launch_us": round(kt["gemm_us"], 3),
+                     "bytes_per_launch": round(kt["gemm_bytes"]),
                      "peak_source": peaks["source"]},
-        "quantize_act": {"GB/s": round(quant_gbs, 1), "avg_launch_us": round(kt["quant_ms"] * 1e3 / kt["quant_n"], 3)},
+        "quantize_act": {"GB/s": round(quant_gbs, 1), "avg_launch_us": round(kt["quant_us"], 3)},
         "weight_quant": wq,
         "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": layer_launches(args.steps),

@@ -28,8 +28,10 @@
 //      ([tile][split][M][256]), fences, and counts itself on the tile's
 //      counter (atomicInc with wrap-around: the last arrival puts it back to
 //      zero, so the counters stay zero between calls);
-//   5. the last CTA of a tile to arrive sums the split partials in split
-//      order (deterministic), applies s_a[m] * s_w[n] and writes BF16.
+//   5. the last CTA of a tile to arrive pulls the tile's partials into its
+//      (by then idle) ring with bulk copies, one round trip for all splits,
+//      sums them in split order (deterministic), applies s_a[m] * s_w[n]
+//      (staged in shared memory while the weights streamed) and writes BF16.
 //
 // Every wait is bounded; see gemm_tiled.cuh.
 #pragma once
@@ -60,10 +62,14 @@ struct Layout {
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = STAGES * A_BYTES;
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 2;  // full, empty, tfull, drain
+    static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 3;  // full, empty, tfull, drain, reduce
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem holder, abort, last flag
-    static constexpr int SCALE_OFF = MISC_OFF + 16;          // amax bits, s, 1/s  [kMaxFusedM] each
-    static constexpr int SMEM_BYTES = SCALE_OFF + 3 * kMaxFusedM * 4 + 1024;
+    static constexpr int SCALE_OFF = (MISC_OFF + 16 + 15) / 16 * 16;               // amax bits, s, 1/s [kMaxFusedM]
+    static constexpr int SW_OFF = (SCALE_OFF + 3 * kMaxFusedM * 4 + 15) / 16 * 16;  // s_w of the tile [BN], read as float4
+    static constexpr int SA_OFF = SW_OFF + BN * 4;                                 // s_a [kMaxM]
+    static constexpr int SMEM_BYTES = SA_OFF + kMaxM * 4 + 1024;
+    static_assert(SW_OFF % 16 == 0 && BAR_OFF % 8 == 0 && RING_BYTES % 1024 == 0, "shared-memory alignment");
     static constexpr int TMEM_COLS = BN;
 };
 
@@ -95,12 +101,15 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     const uint32_t tfull_bar = bar0 + 8u * (2 * STAGES);
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 1);
+    const uint32_t red_bar = bar0 + 8u * (2 * STAGES + 2);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
     uint32_t* amax_sm = reinterpret_cast<uint32_t*>(smem + L::SCALE_OFF);
     float* s_sm = reinterpret_cast<float*>(amax_sm + kMaxFusedM);
     float* r_sm = s_sm + kMaxFusedM;
+    float* sw_sm = reinterpret_cast<float*>(smem + L::SW_OFF);
+    float* sa_sm = reinterpret_cast<float*>(smem + L::SA_OFF);
 
     const int M = args.M, N = args.N, K = args.K;
     const uint32_t warp = warp_id_sync();
@@ -123,6 +132,7 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         }
         mbar_init(tfull_bar, 1);
         mbar_init(drain_bar, 1);
+        mbar_init(red_bar, 1);
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -257,6 +267,14 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         }
     } else {
         const uint32_t q = warp & 3u;
+        {
+            // The scales the last arriver applies, staged while the weights
+            // stream (s_a comes from the quantize kernel: wait for it).
+            if (!QUANT) grid_dependency_wait();
+            const int t = int(threadIdx.x) - 64;  // 0..127
+            for (int c = t; c < BN; c += 128) sw_sm[c] = (n0 + c < N) ? __ldcg(args.s_w + n0 + c) : 0.f;
+            for (int m = t; m < M; m += 128) sa_sm[m] = QUANT ? s_sm[m] : __ldcg(args.s_a + m);
+        }
         if (QUANT) {
             // Warps 2-5 write the codes of each k-block into the ring slot the
             // weights of that k-block land in: M rows x 16 groups of 8.
@@ -320,50 +338,59 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     }
     __syncthreads();
     if (*last_flag) {
-        __threadfence();
-        if (!QUANT) grid_dependency_wait();  // s_a comes from the quantize kernel
-        // Every (row, 4 columns) item loads its splits' float4s at once, two
-        // items per round, so the reads overlap; sums keep split order.
+        __threadfence();  // the other splits' partials, published before their count
+        // The tile's partials [splits][M][BN] go into the ring (every MMA
+        // has completed, so it is idle), rows_per rows of every split per
+        // round: normally one round, one copy per split.
         const int cols = min(BN, N - n0);  // a multiple of 8
         const int c4 = cols / 4;
-        const int items = M * c4;
-        const int64_t stride4 = int64_t(M) * BN / 4;
-        const float4* base4 = reinterpret_cast<const float4*>(args.partial + int64_t(tile) * splits * M * BN);
-        for (int e0 = int(threadIdx.x); e0 < items; e0 += 2 * kThreads) {
-            float4 v[2][kMaxSplits];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int e = e0 + u * kThreads;
-                const int m = e / c4, c = (e % c4) * 4;
-                const float4* src = base4 + (int64_t(m) * BN + c) / 4;
-#pragma unroll
-                for (int j = 0; j < kMaxSplits; ++j)
-                    v[u][j] = (e < items && j < splits) ? __ldcg(src + j * stride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int rows_per = min(M, (L::RING_BYTES / (BN * 4)) / splits);
+        const float* tile_part = args.partial + int64_t(tile) * splits * M * BN;
+        uint32_t red_phase = 0;
+        for (int r0 = 0; r0 < M; r0 += rows_per) {
+            const int rows = min(rows_per, M - r0);
+            const uint32_t bytes = uint32_t(rows) * BN * 4;
+            if (threadIdx.x == 0) {
+                fence_proxy_async_global();  // partials: generic stores -> bulk-copy reads
+                mbar_arrive_expect_tx(red_bar, bytes * uint32_t(splits));
+                for (int j = 0; j < splits; ++j)
+                    bulk_load(sbase + uint32_t(j) * bytes, tile_part + (int64_t(j) * M + r0) * BN, bytes, red_bar);
             }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int e = e0 + u * kThreads;
-                if (e >= items) continue;
-                const int m = e / c4, c = (e % c4) * 4;
+            // One decision for the whole CTA, so that every thread meets the
+            // same barriers even when a wait gives up.
+            if (!__syncthreads_and(mbar_wait(red_bar, red_phase, abort_flag))) {
+                if (threadIdx.x == 0) {
+                    // Let the copies in flight land before the CTA exits.
+                    volatile int no_abort = 0;
+                    mbar_wait(red_bar, red_phase, &no_abort, 10000000ull);
+                }
+                break;
+            }
+            red_phase ^= 1u;
+            const int items = rows * c4;
+            for (int e = int(threadIdx.x); e < items; e += kThreads) {
+                const int mr = e / c4, c = (e % c4) * 4;
+                const float* src = reinterpret_cast<const float*>(smem) + mr * BN + c;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int j = 0; j < kMaxSplits; ++j)
-                    if (j < splits) {
-                        acc.x += v[u][j].x;
-                        acc.y += v[u][j].y;
-                        acc.z += v[u][j].z;
-                        acc.w += v[u][j].w;
-                    }
-                const int n = n0 + c;
-                const float sa = QUANT ? s_sm[m] : __ldcg(args.s_a + m);
-                const float4 sw = __ldg(reinterpret_cast<const float4*>(args.s_w + n));
+                for (int j = 0; j < splits; ++j) {
+                    const float4 v = *reinterpret_cast<const float4*>(src + j * (bytes / 4));
+                    acc.x += v.x;
+                    acc.y += v.y;
+                    acc.z += v.z;
+                    acc.w += v.w;
+                }
+                const int m = r0 + mr;
+                const float sa = sa_sm[m];
+                const float4 sw = *reinterpret_cast<const float4*>(sw_sm + c);
                 __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * sa * sw.x, acc.y * sa * sw.y);
                 __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * sa * sw.z, acc.w * sa * sw.w);
                 uint2 pk;
                 pk.x = *reinterpret_cast<uint32_t*>(&lo);
                 pk.y = *reinterpret_cast<uint32_t*>(&hi);
-                *reinterpret_cast<uint2*>(args.Y + int64_t(m) * N + n) = pk;
+                *reinterpret_cast<uint2*>(args.Y + int64_t(m) * N + n0 + c) = pk;
             }
+            fence_proxy_async_smem();  // ring: these generic reads -> the next round's bulk-copy writes
+            __syncthreads();
         }
     }
 

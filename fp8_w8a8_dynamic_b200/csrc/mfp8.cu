@@ -600,6 +600,11 @@ mfp8_status mfp8_linear_noalloc(const void* X_bf16, int64_t M, int64_t K, const 
                           nullptr, nullptr, stream);
 }
 
+int mfp8_choose_path(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return MFP8_PATH_AUTO;
+    return choose_path(M, N, K);
+}
+
 size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return 0;
     return make_plan(M, N, K, false, M <= kSkinnyMaxM, sm_count_for_sizing()).total;
@@ -630,13 +635,6 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (split_k) {
-        if (cudaMemsetAsync(static_cast<uint8_t*>(workspace) + plan.cnt_off, 0, size_t(plan.tiles) * 4, s) !=
-            cudaSuccess) {
-            cudaGetLastError();
-            return MFP8_ERR_CUDA;
-        }
-    }
     return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, workspace, plan,
                     /*weights_static=*/false, /*dependent=*/false, dev, info, s);
 }

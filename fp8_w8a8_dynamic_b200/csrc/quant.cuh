@@ -134,9 +134,9 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red /* [
 // One block per row; the row (K/8 16-byte vectors) lives in registers,
 // VPT vectors per thread.  Requires K/8 <= VPT * 256.
 // EARLY_TRIGGER (activation quantization) is the programmatic-dependent
-// form: the kernel waits for the grid before it, then lets the GEMM that
-// follows begin its prologue at once (that GEMM waits for the codes before
-// reading them).  The weight quantizer leaves it off, so nothing that
+// form: the kernel lets the GEMM that follows begin its prologue at once
+// (that GEMM waits for the codes before reading them), then waits for the
+// grid before it.  The weight quantizer leaves it off, so nothing that
 // follows starts before the weight codes are complete.
 // Block 0 also clears `nzero` words at `zero` (the split-K counters of the
 // GEMM that follows in the same call).
@@ -144,12 +144,15 @@ template <int VPT, bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
                       float* __restrict__ S, unsigned int* __restrict__ zero, int nzero) {
-    // Launched as a programmatic dependent of the previous kernel: wait for
-    // it (X may be its output, and it may still read this call's buffers)
-    // before touching memory, then let the GEMM that follows start.
+    // Launched as a programmatic dependent of the previous kernel.  The GEMM
+    // that follows may start launching at once: before its own wait it only
+    // sets itself up and (static weights) reads W, and one of its CTAs and
+    // one of these always fit on an SM together.  This kernel then waits for
+    // the previous one (X may be its output, and it may still read this
+    // call's buffers) before touching memory.
     if (EARLY_TRIGGER) {
-        grid_dependency_wait();
         grid_launch_dependents();
+        grid_dependency_wait();
     }
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < nzero; i += kQuantThreads) zero[i] = 0u;
@@ -186,9 +189,9 @@ template <bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_loop_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
                        float* __restrict__ S, unsigned int* __restrict__ zero, int nzero) {
-    if (EARLY_TRIGGER) {
-        grid_dependency_wait();
+    if (EARLY_TRIGGER) {  // as in quant_rows_reg_kernel
         grid_launch_dependents();
+        grid_dependency_wait();
     }
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < nzero; i += kQuantThreads) zero[i] = 0u;

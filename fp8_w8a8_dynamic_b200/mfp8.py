@@ -54,6 +54,7 @@ def lib():
             "mfp8_linear": (i32, [P, i64, i64, P, P, i64, P, P, sz, P]),
             "mfp8_linear_ex": (i32, [P, i64, i64, P, P, i64, P, P, sz, i32, i32, P, P, P]),
             "mfp8_linear_noalloc": (i32, [P, i64, i64, P, P, i64, P, P]),
+            "mfp8_choose_path": (i32, [i64, i64, i64]),
             "mfp8_gemm_workspace_bytes": (sz, [i64, i64, i64]),
             "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, P, sz, i32, P]),
             "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
@@ -99,6 +100,14 @@ def mfp8_linear_noalloc(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, stream=0):
 
 
 STATIC_WORKSPACE_BYTES = 16 << 20  # MFP8_STATIC_WORKSPACE_BYTES
+
+
+def mfp8_choose_path(M, N, K):
+    return lib().mfp8_choose_path(M, N, K)
+
+
+KERNEL_OF_PATH = {PATH_TILED: "gemm_tiled_kernel", PATH_SPLITK: "gemm_skinny_kernel",
+                  PATH_PAIR: "gemm_pair_kernel", PATH_FUSED: "gemm_skinny_kernel"}
 
 
 def mfp8_gemm_workspace_bytes(M, N, K):

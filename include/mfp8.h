@@ -125,6 +125,10 @@ typedef enum {
     MFP8_PATH_FUSED = 4   /* one kernel: split-K GEMM that quantizes X on chip (M <= 16) */
 } mfp8_path;
 
+/* The kernel MFP8_PATH_AUTO takes at these sizes (TILED, SPLITK or PAIR);
+ * MFP8_PATH_AUTO itself for sizes no kernel takes. */
+MFP8_API int mfp8_choose_path(int64_t M, int64_t N, int64_t K);
+
 /* Flags for mfp8_linear_ex. */
 #define MFP8_FLAG_STATIC_WEIGHTS 1
 /* The caller promises that W_fp8 and w_scale are not written by any work
@@ -183,9 +187,10 @@ MFP8_API size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 /* The contraction and epilogue alone, on activations already quantized by
  * mfp8_quantize_act: Y = bf16((X_fp8 . W_fp8^T) * x_scale (x) w_scale).
  * Lets the GEMM be timed and checked without the quantize pass.  path is
- * AUTO, TILED, SPLITK or PAIR; the split-K kernel takes its partials from
- * `workspace` (at least mfp8_gemm_workspace_bytes) and clears its counters
- * with a memset on `stream` first. */
+ * AUTO, TILED, SPLITK or PAIR; the split-K kernel takes its partials and
+ * tile counters from `workspace` (at least mfp8_gemm_workspace_bytes), under
+ * the same contract as mfp8_linear: zero-filled before its first use, the
+ * counters left at zero by every call. */
 MFP8_API mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K,
                       const void* W_fp8, const float* w_scale, int64_t N,
                       void* Y_bf16, void* workspace, size_t workspace_bytes,

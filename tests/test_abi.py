@@ -66,6 +66,11 @@ def test_workspace_bytes(lib):
     assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == C + 65536 + 256 + tiles * splits * 16 * 1024
     assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == C + tiles * splits * 16 * 1024
     assert mfp8.mfp8_gemm_workspace_bytes(300, 4096, 4096) == 0
+    # the AUTO choice: split-K for decode sizes, 128-row tiles for mid M, pairs above
+    assert mfp8.mfp8_choose_path(8, 12288, 4096) == mfp8.PATH_SPLITK
+    assert mfp8.mfp8_choose_path(200, 4096, 4096) == mfp8.PATH_TILED
+    assert mfp8.mfp8_choose_path(2048, 4096, 4096) == mfp8.PATH_PAIR
+    assert mfp8.mfp8_choose_path(0, 4096, 4096) == mfp8.PATH_AUTO
     # one K-block only: one split
     assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == C + 256 + 256 + 3 * 1024
     assert mfp8.mfp8_linear_workspace_bytes(0, 8, 48) == 0
