@@ -158,8 +158,11 @@ class Layer:
     def flops_per_step(self):
         return sum(2 * M * lin.N * lin.K for M in self.Ms for lin in self.lins)
 
-    def launches_per_step(self):
-        return 2 * len(self.Ms) * len(self.lins)
+    def launches_per_step(self, mfp8):
+        """Library kernels one step launches: one per Linear on the
+        one-kernel decode path, a quantize pass and a GEMM otherwise."""
+        return sum(1 if mfp8.mfp8_choose_path(M, lin.N, lin.K) == mfp8.PATH_FUSED else 2
+                   for M in self.Ms for lin in self.lins)
 
 
 def time_graph(torch, fn, steps, warmup, dist_ctx):
@@ -194,14 +197,27 @@ def time_graph(torch, fn, steps, warmup, dist_ctx):
 
 
 def kernel_times(torch, mfp8, layer, steps, warmup):
-    """Average launch duration of the GEMM kernel and of the quantize kernel
-    over the step's Linears.  Each is a CUDA graph of that kernel's launches
-    alone, one per Linear with nothing between them, timed with CUDA events
-    around `steps` replays on the launching stream; the average includes the
-    gaps between graph nodes, so it is an upper bound on a launch's own time.
-    The split-K workspaces are zero-filled once (every call leaves their
-    counters at zero)."""
+    """Average launch duration of the step's GEMM kernel (and of the quantize
+    kernel where it is a launch of its own) over the step's Linears.  Each is
+    a CUDA graph of that kernel's launches alone, one per Linear with nothing
+    between them, timed with CUDA events around `steps` replays on the
+    launching stream; the average includes the gaps between graph nodes, so
+    it is an upper bound on a launch's own time.  Where every Linear takes
+    the one-kernel decode path (quantization on chip), the graph of the
+    step's launches is that kernel's graph.  The split-K workspaces are
+    zero-filled once (every call leaves their counters at zero)."""
     keys = [(mi, M, i, lin) for mi, M in enumerate(layer.Ms) for i, lin in enumerate(layer.lins)]
+    paths = sorted({mfp8.mfp8_choose_path(M, lin.N, lin.K) for (mi, M, i, lin) in keys})
+    n = len(keys)
+    out = dict(launches=steps * n, kernel="+".join(mfp8.KERNEL_OF_PATH[p] for p in paths),
+               gemm_bytes=sum(lin.N * lin.K + 4 * lin.N + 2 * M * lin.K + 2 * M * lin.N
+                              for (mi, M, i, lin) in keys) / n,
+               gemm_flops=sum(2 * M * lin.N * lin.K for (mi, M, i, lin) in keys) / n,
+               quant_us=None, quant_bytes=None)
+    if paths == [mfp8.PATH_FUSED]:
+        out["gemm_us"] = time_graph(torch, lambda h: layer.step(mfp8, h), steps, warmup, None) * 1e3 / (steps * n)
+        return out
+
     x8 = {(M, i): mfp8.quantize_act(layer.x[(M, i)]) for (mi, M, i, lin) in keys}
     gws_of = {(M, i): torch.zeros((max(16, mfp8.mfp8_gemm_workspace_bytes(M, lin.N, lin.K)),), dtype=torch.uint8,
                                   device=layer.x[(M, i)].device) for (mi, M, i, lin) in keys}
@@ -225,16 +241,12 @@ def kernel_times(torch, mfp8, layer, steps, warmup):
             if st != mfp8.OK:
                 raise mfp8.Mfp8Error(st, "mfp8_quantize_act")
 
-    n = len(keys)
-    gemm_ms = time_graph(torch, gemms, steps, warmup, None)
-    quant_ms = time_graph(torch, quants, steps, warmup, None)
-    paths = sorted({mfp8.mfp8_choose_path(M, lin.N, lin.K) for (mi, M, i, lin) in keys})
-    return dict(gemm_us=gemm_ms * 1e3 / (steps * n), quant_us=quant_ms * 1e3 / (steps * n), launches=steps * n,
-                gemm_bytes=sum(lin.N * lin.K + 4 * lin.N + M * lin.K + 4 * M + 2 * M * lin.N
-                               for (mi, M, i, lin) in keys) / n,
-                gemm_flops=sum(2 * M * lin.N * lin.K for (mi, M, i, lin) in keys) / n,
-                quant_bytes=sum(3 * M * lin.K + 4 * M for (mi, M, i, lin) in keys) / n,
-                kernel="+".join(mfp8.KERNEL_OF_PATH[p] for p in paths))
+    out["gemm_us"] = time_graph(torch, gemms, steps, warmup, None) * 1e3 / (steps * n)
+    out["quant_us"] = time_graph(torch, quants, steps, warmup, None) * 1e3 / (steps * n)
+    out["gemm_bytes"] = sum(lin.N * lin.K + 4 * lin.N + M * lin.K + 4 * M + 2 * M * lin.N
+                            for (mi, M, i, lin) in keys) / n
+    out["quant_bytes"] = sum(3 * M * lin.K + 4 * M for (mi, M, i, lin) in keys) / n
+    return out
 
 
 def e2e_time(torch, mfp8, layer, steps, warmup, dist_ctx):
@@ -407,7 +419,12 @@ def main():
 
     kt = kernel_times(torch, mfp8, layer, steps=max(5, min(args.steps, 20)), warmup=args.warmup)
     gemm_gbs = kt["gemm_bytes"] / (kt["gemm_us"] * 1e-6) / 1e9
-    quant_gbs = kt["quant_bytes"] / (kt["quant_us"] * 1e-6) / 1e9
+    if kt["quant_us"] is None:
+        quant = "fused into " + kt["kernel"]
+    else:
+        quant = {"GB/s": round(kt["quant_bytes"] / (kt["quant_us"] * 1e-6) / 1e9, 1),
+                 "avg_launch_us": round(kt["quant_us"], 3)}
+    launches = layer.launches_per_step(mfp8) * args.steps
 
     e2e_ms, h2d, d2h = e2e_time(torch, mfp8, layer, max(3, args.steps // 5), 3, ctx)
     e2e_val = wbytes * ctx.world * max(3, args.steps // 5) / (e2e_ms * 1e-3) / 1e9
@@ -456,10 +473,10 @@ def main():
                      "avg_launch_us": round(kt["gemm_us"], 3),
                      "bytes_per_launch": round(kt["gemm_bytes"]),
                      "peak_source": peaks["source"]},
-        "quantize_act": {"GB/s": round(quant_gbs, 1), "avg_launch_us": round(kt["quant_us"], 3)},
+        "quantize_act": quant,
         "weight_quant": wq,
         "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": layer_launches(args.steps),
+        "gpu_launches": launches,
         "clocks": clocks.summary(),
         "prefill": prefill,
         "cpu_baseline": cpu,
@@ -468,9 +485,6 @@ def main():
         print(json.dumps(out))
     ctx.close()
 
-
-def layer_launches(steps):
-    return 2 * len(DECODE_MS) * 7 * steps
 
 
 if __name__ == "__main__":

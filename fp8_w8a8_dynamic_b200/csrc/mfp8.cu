@@ -18,6 +18,7 @@
 #include "gemm_tiled.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_stream.cuh"
 
 namespace mfp8 {
 namespace {
@@ -296,11 +297,12 @@ mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, 
 }
 
 constexpr int64_t kSkinnyMaxM = skinny::kMaxM;
-constexpr int64_t kFusedMaxM = skinny::kMaxFusedM;
+constexpr int64_t kStreamMaxM = stream::kMaxM;
 constexpr int kSkinnyStages = 4;
 
 int choose_path(int64_t M, int64_t N, int64_t K) {
     (void)K;
+    if (M <= kStreamMaxM) return MFP8_PATH_FUSED;
     if (M <= 64 && (N + 255) / 256 <= 4096) return MFP8_PATH_SPLITK;
     if (M < 256) return MFP8_PATH_TILED;
     return MFP8_PATH_PAIR;
@@ -410,6 +412,84 @@ mfp8_status launch_skinny(const void* X, const float* s_a, int64_t M, int64_t K,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, args) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
+// ------------------------------------------- decode: one-kernel Linear --
+
+// Cluster size S (K split) of the one-kernel decode path: the largest power
+// of two up to 8 that keeps tiles * S within 1.5 CTAs per SM (two fit on an
+// SM; more CTAs keep more weight copies in flight), no more
+// than the K blocks, and raised (up to 8) until the codes of one CTA's K
+// range fit its code store.  Weight ring: what is left of the shared region.
+// Returns false when no S fits (K too long for this path).
+bool stream_geometry(int64_t M, int64_t N, int64_t K, int sm_count, stream::Geometry* g) {
+    const int64_t tiles = (N + stream::TILE - 1) / stream::TILE;
+    const int64_t kb = (K + stream::SUB - 1) / stream::SUB;
+    const int mpad = M <= 8 ? 8 : 16;
+    int S = 1;
+    while (S < stream::kMaxCluster && tiles * S * 2 <= sm_count * 3 / 2 && S * 2 <= kb) S *= 2;
+    auto code_bytes = [&](int s_) {
+        const int64_t kbs = (kb + s_ - 1) / s_;
+        return (kbs * mpad * stream::SUB + 1023) / 1024 * 1024;
+    };
+    while (code_bytes(S) > stream::kMaxCodeBytes && S < stream::kMaxCluster && S * 2 <= kb) S *= 2;
+    if (code_bytes(S) > stream::kMaxCodeBytes) return false;
+    g->S = S;
+    g->mpad = mpad;
+    g->code_bytes = int(code_bytes(S));
+    const int st = (stream::kShared - g->code_bytes) / stream::kWStageBytes;
+    g->stages = st > stream::kMaxStages ? stream::kMaxStages : st;
+    return g->stages >= stream::kMinStages;
+}
+
+mfp8_status launch_stream(const void* X, int64_t M, int64_t K, const void* W8, const float* s_w, int64_t N,
+                          void* Y, bool weights_static, bool dependent, void* x8_out, float* sa_out, int dev,
+                          const DeviceInfo& info, cudaStream_t stream) {
+    if (M < 1 || M > kStreamMaxM || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
+        return MFP8_ERR_UNSUPPORTED_SHAPE;
+    stream::Geometry g;
+    if (!stream_geometry(M, N, K, info.sm_count, &g)) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    auto kern = stream::gemm_stream_kernel;
+    static bool attr_done[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, stream::Smem::BYTES, dev, attr_done);
+    if (st != MFP8_OK) return st;
+    const int64_t tiles = (N + stream::TILE - 1) / stream::TILE;
+    const int64_t grid = tiles * g.S;
+    if (grid > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    CUtensorMap tmW;
+    if ((st = make_map_u8(&tmW, W8, N, K, stream::TILE)) != MFP8_OK) return st;
+
+    stream::Args args;
+    args.X = static_cast<const __nv_bfloat16*>(X);
+    args.s_w = s_w;
+    args.Y = static_cast<__nv_bfloat16*>(Y);
+    args.x8_out = static_cast<uint8_t*>(x8_out);
+    args.sa_out = sa_out;
+    args.M = int(M);
+    args.N = int(N);
+    args.K = int(K);
+    args.weights_static = weights_static ? 1 : 0;
+    args.g = g;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(stream::kThreads);
+    cfg.dynamicSmemBytes = stream::Smem::BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = unsigned(g.S);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tmW, args) != cudaSuccess) {
         cudaGetLastError();
         return MFP8_ERR_CUDA;
     }
@@ -530,10 +610,9 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     if (st != MFP8_OK) return st;
     if (path < MFP8_PATH_AUTO || path > MFP8_PATH_FUSED) return MFP8_ERR_INVALID_ARG;
     if ((flags & ~MFP8_FLAG_STATIC_WEIGHTS) != 0) return MFP8_ERR_INVALID_ARG;
-    if ((path == MFP8_PATH_SPLITK || path == MFP8_PATH_FUSED) && (N + 255) / 256 > 4096)
-        return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_SPLITK && (N + 255) / 256 > 4096) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (path == MFP8_PATH_SPLITK && M > kSkinnyMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    if (path == MFP8_PATH_FUSED && M > kFusedMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_FUSED && M > kStreamMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_bf16) return MFP8_ERR_INVALID_ARG;
     if (!aligned16(X_bf16)) return MFP8_ERR_MISALIGNED;
@@ -548,11 +627,11 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     }
     if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
     const bool weights_static = (flags & MFP8_FLAG_STATIC_WEIGHTS) != 0;
-    // Split-K with the quantize pass, or (FUSED, M <= 16) the split-K kernel
-    // that quantizes X itself: no codes in the workspace, no extra launch.
+    // FUSED (M <= 16): one kernel quantizes X on chip and streams the
+    // weights; it keeps nothing in the workspace.
     const bool fused = path == MFP8_PATH_FUSED;
-    const bool split_k = path == MFP8_PATH_SPLITK || fused;
-    const Plan plan = make_plan(M, N, K, X_fp8_out == nullptr && !fused, split_k, sm_count_for_sizing());
+    const bool split_k = path == MFP8_PATH_SPLITK;
+    const Plan plan = fused ? Plan() : make_plan(M, N, K, X_fp8_out == nullptr, split_k, sm_count_for_sizing());
     if (plan.total > 0) {
         if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
         if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
@@ -567,10 +646,8 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* base = static_cast<uint8_t*>(workspace);
     if (fused)
-        return launch_skinny<true>(X_bf16, nullptr, M, K, W_fp8, w_scale, N, Y_bf16,
-                                   reinterpret_cast<float*>(base + plan.part_off),
-                                   reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static,
-                                   /*dependent=*/true, X_fp8_out, x_scale_out, dev, s);
+        return launch_stream(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, weights_static, /*dependent=*/true,
+                             X_fp8_out, x_scale_out, dev, info, s);
     void* X8 = X_fp8_out ? X_fp8_out : base + plan.x8_off;
     float* s_a = x_scale_out ? x_scale_out : reinterpret_cast<float*>(base + plan.sa_off);
     unsigned int* counters = split_k ? reinterpret_cast<unsigned int*>(base + plan.cnt_off) : nullptr;
@@ -624,6 +701,7 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
         ranges_overlap(x_scale, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
         return MFP8_ERR_INVALID_ARG;
     if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
+    if (path == MFP8_PATH_FUSED) path = MFP8_PATH_SPLITK;  // codes given: the split-K kernel streams them
     const bool split_k = path == MFP8_PATH_SPLITK;
     const Plan plan = make_plan(M, N, K, false, split_k, sm_count_for_sizing());
     if (plan.total > 0) {
@@ -653,6 +731,22 @@ mfp8_status mfp8_e4m3_encode_f32(const float* in, int64_t n, uint8_t* out, void*
     const int64_t cap = int64_t(info.sm_count) * 16;
     if (blocks > cap) blocks = cap;
     e4m3_encode_kernel<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(in, n, out);
+    return launch_status();
+}
+
+mfp8_status mfp8_debug_quantize_check(void* out_u64x2, void* stream) {
+    if (!out_u64x2) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(out_u64x2)) return MFP8_ERR_MISALIGNED;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(out_u64x2, 0, 16, s) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    quantize_check_kernel<<<0x7f80u, 256, 0, s>>>(static_cast<unsigned long long*>(out_u64x2));
     return launch_status();
 }
 

@@ -8,9 +8,9 @@
 //   s    = fl32(max_k |x_k| / 448), raised to FLT_MIN when smaller
 //   q_k  = e4m3_rn_satfinite(fl32(x_k / s))
 // The codes are those of an IEEE round-to-nearest division x / s, so they
-// are bit-identical to the CPU oracle's; quantize8 reaches them with one
-// multiply per element and an exact divide only near e4m3 rounding
-// boundaries (see there).
+// are bit-identical to the CPU oracle's; quantize8 reaches them with a
+// multiply by the reciprocal and two fused multiply-adds per element (see
+// div_rn_by_recip), checked against the divide on every bf16 pair.
 //
 // Memory-bound: each row is read once (16-byte loads, 8 bf16 per load),
 // held in registers while the block reduces its absmax, then converted and
@@ -46,66 +46,29 @@ __device__ __forceinline__ uint32_t absmax_bits_u4(uint4 v, uint32_t acc) {
     return acc;
 }
 
-__device__ __forceinline__ float scale_from_absmax_bits(uint32_t amax16) {
+__device__ __forceinline__ float scale_from_absmax_bits_div(uint32_t amax16) {
     const float amax = __uint_as_float(amax16 << 16);
     float s = __fdiv_rn(amax, kE4m3Max);
     return s < kFltMin ? kFltMin : s;
 }
 
+// The same scale without a divide.  448 = 7 * 2^6, so fl32(a / 448) is
+// fl32(a / 7) * 2^-6 (scaling by a power of two is exact while the result
+// is normal; below FLT_MIN both forms are raised to FLT_MIN).  fl32(a / 7)
+// is Markstein's corrected quotient with the correctly rounded reciprocal
+// 1/7 = 0x3E124925.  Checked against the divide for every bf16 absmax
+// (mfp8_debug_quantize_check).
+__device__ __forceinline__ float scale_from_absmax_bits(uint32_t amax16) {
+    const float a = __uint_as_float(amax16 << 16);
+    const float r7 = __uint_as_float(0x3E124925u);
+    const float q0 = __fmul_rn(a, r7);
+    const float e = __fmaf_rn(-q0, 7.0f, a);
+    const float s = __fmul_rn(__fmaf_rn(e, r7, q0), 0.015625f);
+    return s < kFltMin ? kFltMin : s;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-// Exact quantization without a divide per element.
-//
-// The code of x is e4m3(fl32(x / s)).  With r = fl32(1 / s) (one correctly
-// rounded reciprocal per row), q = fl32(x * r) differs from x / s by at most
-// 2^-23 |x / s|, so from fl32(x / s) by at most about 3 units in the last
-// place of q.  e4m3 rounding is a step function of its input whose steps
-// sit at the midpoints between neighbouring codes; if q is more than 8 ulps
-// away from every such midpoint, q and fl32(x / s) lie on the same step and
-// encode to the same code.  Only values closer than that (rare) are divided
-// exactly.  The midpoints in fp32 bits:
-//   - |q| >= 432 encodes to 448 whatever the rounding (saturation above
-//     464), so nothing from 440 up needs a check;
-//   - e4m3 normals (|q| >= 2^-6): 3 mantissa bits, so a midpoint is an fp32
-//     whose low 20 mantissa bits are exactly 1 << 19;
-//   - e4m3 subnormals (|q| < 2^-6): steps of 2^-9, midpoints at odd
-//     multiples of 2^-10; in fixed point with 2^-34 units (exact for
-//     |q| >= 2^-11) a midpoint is 2^24 modulo 2^25.  Below 2^-11 everything
-//     encodes to zero (the first midpoint is 2^-10).
-__device__ __forceinline__ bool near_e4m3_midpoint(float q) {
-    const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
-    if (b >= 0x43dc0000u) return false;                    // |q| >= 440
-    if (b >= 0x3c800000u) {                                // |q| >= 2^-6
-        const int32_t d = int32_t(b & 0xfffffu) - 0x80000;
-        return d >= -8 && d <= 8;
-    }
-    if (b < 0x3a000000u) return false;                     // |q| < 2^-11
-    const uint32_t a = uint32_t(__uint_as_float(b) * 17179869184.0f);  // |q| * 2^34, exact
-    const int32_t d = int32_t(a & 0x1ffffffu) - 0x1000000;
-    return d >= -128 && d <= 128;                          // 8 ulps of the largest binade here
-}
-
-// 8 bf16 values -> 8 e4m3 codes (byte i = value i).  r must be fl32(1 / s).
-__device__ __forceinline__ uint2 quantize8(uint4 v, float s, float r) {
-    float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-    float q[8];
-    bool slow = false;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        q[i] = x[i] * r;
-        slow |= near_e4m3_midpoint(q[i]);
-    }
-    if (slow) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], s);
-    }
-    uint2 out;
-    out.x = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
-    out.y = e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16);
-    return out;
-}
 
 // The reference form: one IEEE divide per element.
 __device__ __forceinline__ uint2 quantize8_div(uint4 v, float s) {
@@ -115,6 +78,51 @@ __device__ __forceinline__ uint2 quantize8_div(uint4 v, float s) {
     q.y = e4m3x2(__fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s)) |
           (e4m3x2(__fdiv_rn(bf16_lo(v.w), s), __fdiv_rn(bf16_hi(v.w), s)) << 16);
     return q;
+}
+
+// fl32(a / s) for a >= 0 without a divide: r = fl32(1 / s) (correctly
+// rounded), q0 = fl32(a * r) is within one unit in the last place of a / s,
+// the residual a - q0 * s is exact in one fused multiply-add, and one more
+// fused multiply-add q0 + (a - q0 s) * r rounds to the correctly rounded
+// quotient (Markstein's theorem on division by reciprocal with a corrected
+// quotient).  Working on |x| keeps the sign of zero out of the arithmetic;
+// the code's sign bit is taken from x.  Checked against the IEEE divide on
+// every pair of bf16 values with |x| <= absmax (mfp8_debug_quantize_check).
+__device__ __forceinline__ float div_rn_by_recip(float a, float s, float r) {
+    const float q0 = __fmul_rn(a, r);
+    const float e = __fmaf_rn(-q0, s, a);
+    return __fmaf_rn(e, r, q0);
+}
+
+// Two bf16 values (one 32-bit word) -> two e4m3 codes (16 bits, low value in
+// the low byte).
+__device__ __forceinline__ uint32_t quantize2_fma(uint32_t w, float s, float r) {
+    const float lo = div_rn_by_recip(__uint_as_float((w & 0x7fffu) << 16), s, r);
+    const float hi = div_rn_by_recip(__uint_as_float(w & 0x7fff0000u), s, r);
+    const uint32_t sign = ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
+    return e4m3x2(lo, hi) | sign;
+}
+
+// 8 bf16 values -> 8 e4m3 codes, same codes as quantize8_div.  The
+// corrected quotient needs an exact residual a - q0 s; when s is tiny that
+// residual falls below the normal fp32 range and loses bits, so rows with
+// s < 2^-64 (absmax below about 2.4e-17) take the divide.
+constexpr float kFmaMinScale = 5.42101086242752217004e-20f;  // 2^-64
+
+// For s >= kFmaMinScale only (callers that check the scale once per row).
+__device__ __forceinline__ uint2 quantize8_fast(uint4 v, float s, float r) {
+    uint2 out;
+    out.x = quantize2_fma(v.x, s, r) | (quantize2_fma(v.y, s, r) << 16);
+    out.y = quantize2_fma(v.z, s, r) | (quantize2_fma(v.w, s, r) << 16);
+    return out;
+}
+
+// The divide form out of line, for the rare rows with a tiny scale inside
+// unrolled loops.
+__device__ __noinline__ uint2 quantize8_div_call(uint4 v, float s) { return quantize8_div(v, s); }
+
+__device__ __forceinline__ uint2 quantize8(uint4 v, float s, float r) {
+    return s < kFmaMinScale ? quantize8_div(v, s) : quantize8_fast(v, s, r);
 }
 
 constexpr int kQuantThreads = 256;
@@ -207,6 +215,50 @@ quant_rows_loop_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict
     if (threadIdx.x == 0) S[row] = s;
     uint2* qr = Q + row * nvec;
     for (int64_t j = threadIdx.x; j < nvec; j += kQuantThreads) qr[j] = quantize8(__ldg(xr + j), s, r);
+}
+
+// Diagnostic: for every absmax a (a positive finite bf16, or zero) the
+// divide-free scale against fl32(a / 448), and for every bf16 x with
+// |x| <= a the codes of quantize8 against those of the IEEE-divide form.  Block b takes absmax bits b; out[0] counts mismatching
+// values, out[1] keeps one of them as (a << 16) | x.
+__global__ void quantize_check_kernel(unsigned long long* __restrict__ out) {
+    const uint32_t a = blockIdx.x;  // 0 .. 0x7f7f
+    const float s = scale_from_absmax_bits(a);
+    const float r = __frcp_rn(s);
+    unsigned long long bad = 0;
+    uint32_t witness = 0;
+    if (threadIdx.x == 0 && __float_as_uint(s) != __float_as_uint(scale_from_absmax_bits_div(a))) {
+        ++bad;  // the scale itself differs from the divide's
+        witness = (a << 16) | 0xffffu;
+    }
+    // x magnitudes 0..a, both signs: 2 (a + 1) values, 8 per step
+    const uint32_t n = 2u * (a + 1u);
+    for (uint32_t base = threadIdx.x * 8u; base < n; base += blockDim.x * 8u) {
+        uint32_t h[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t j = base + uint32_t(i);
+            const uint32_t mag = j < n ? (j >> 1) : 0u;
+            h[i] = mag | ((j & 1u) << 15);
+        }
+        const uint4 v = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
+                                   h[6] | (h[7] << 16));
+        const uint2 f = quantize8(v, s, r);
+        const uint2 d = quantize8_div(v, s);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t cf = ((i < 4 ? f.x : f.y) >> (8 * (i & 3))) & 0xffu;
+            const uint32_t cd = ((i < 4 ? d.x : d.y) >> (8 * (i & 3))) & 0xffu;
+            if (base + uint32_t(i) < n && cf != cd) {
+                ++bad;
+                witness = (a << 16) | h[i];
+            }
+        }
+    }
+    if (bad) {
+        atomicAdd(out, bad);
+        atomicExch(out + 1, (unsigned long long)witness);
+    }
 }
 
 // Diagnostic: the e4m3 conversion alone, on arbitrary fp32 values.

@@ -58,6 +58,7 @@ def lib():
             "mfp8_gemm_workspace_bytes": (sz, [i64, i64, i64]),
             "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, P, sz, i32, P]),
             "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
+            "mfp8_debug_quantize_check": (i32, [P, P]),
             "mfp8_debug_bounded_wait": (i32, [i64, P]),
             "mfp8_get_device_status": (i32, [P]),
             "mfp8_status_string": (ctypes.c_char_p, [i32]),
@@ -107,7 +108,7 @@ def mfp8_choose_path(M, N, K):
 
 
 KERNEL_OF_PATH = {PATH_TILED: "gemm_tiled_kernel", PATH_SPLITK: "gemm_skinny_kernel",
-                  PATH_PAIR: "gemm_pair_kernel", PATH_FUSED: "gemm_skinny_kernel"}
+                  PATH_PAIR: "gemm_pair_kernel", PATH_FUSED: "gemm_stream_kernel"}
 
 
 def mfp8_gemm_workspace_bytes(M, N, K):
@@ -122,6 +123,10 @@ def mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, workspace, worksp
 
 def mfp8_e4m3_encode_f32(inp, n, out, stream=0):
     return lib().mfp8_e4m3_encode_f32(inp, n, out, stream)
+
+
+def mfp8_debug_quantize_check(out, stream=0):
+    return lib().mfp8_debug_quantize_check(out, stream)
 
 
 def mfp8_debug_bounded_wait(timeout_us, stream=0):

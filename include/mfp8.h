@@ -122,11 +122,12 @@ typedef enum {
     MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
     MFP8_PATH_SPLITK = 2, /* quantize pass, then the weight-streaming split-K GEMM over all SMs (M <= 128) */
     MFP8_PATH_PAIR = 3,   /* quantize pass, then the 256-row-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
-    MFP8_PATH_FUSED = 4   /* one kernel: split-K GEMM that quantizes X on chip (M <= 16) */
+    MFP8_PATH_FUSED = 4   /* one kernel: quantizes X on chip and streams the weights, whole K per CTA (M <= 16) */
 } mfp8_path;
 
-/* The kernel MFP8_PATH_AUTO takes at these sizes (TILED, SPLITK or PAIR);
- * MFP8_PATH_AUTO itself for sizes no kernel takes. */
+/* The kernel MFP8_PATH_AUTO takes at these sizes (FUSED for M <= 16, SPLITK
+ * up to 64, TILED below 256, PAIR above); MFP8_PATH_AUTO itself for sizes no
+ * kernel takes. */
 MFP8_API int mfp8_choose_path(int64_t M, int64_t N, int64_t K);
 
 /* Flags for mfp8_linear_ex. */
@@ -143,8 +144,9 @@ MFP8_API int mfp8_choose_path(int64_t M, int64_t N, int64_t K);
  * x_scale_out [M]; pass NULL for none).  Used to test each kernel on the
  * same shapes, to check that the activation bytes of every path are
  * bit-identical to mfp8_quantize_act, and by callers with static weights.
- * MFP8_PATH_FUSED quantizes X inside the split-K kernel (every CTA takes the
- * row scales itself): one launch, and no codes in the workspace.  When
+ * MFP8_PATH_FUSED is one launch that quantizes X on chip (every CTA takes
+ * the row scales itself) and owns whole output channels, so it keeps
+ * nothing in the workspace (it may be NULL with 0 bytes).  When
  * X_fp8_out is given, the codes are written there as well (the quantize
  * pass writes them there instead of the workspace).  Returns MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel
  * cannot take these sizes, MFP8_ERR_INVALID_ARG for an unknown path or flag. */
@@ -195,6 +197,18 @@ MFP8_API mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t 
                       const void* W_fp8, const float* w_scale, int64_t N,
                       void* Y_bf16, void* workspace, size_t workspace_bytes,
                       int path, void* stream);
+
+/* Diagnostic: checks the quantizer's divide-free arithmetic against IEEE
+ * divides.  The scale fl32(absmax / 448) of every absmax (0 and each positive
+ * finite bf16) is computed as a corrected quotient by 7 times 2^-6, and each
+ * code rounds x / s with one multiply by the correctly rounded reciprocal,
+ * one fused multiply-add for the residual and one for the corrected quotient;
+ * both are compared with the divide for every bf16 x with |x| <= absmax,
+ * both signs.  out_u64x2 [2] device uint64, written: [0] the number of
+ * scales and codes that differ (0 when the arithmetic is exact), [1] one of
+ * them as (absmax_bits << 16) | x_bits (x_bits 0xffff: the scale).  Read it
+ * after synchronising `stream`. */
+MFP8_API mfp8_status mfp8_debug_quantize_check(void* out_u64x2, void* stream);
 
 /* Diagnostic: encode n fp32 values with the device's e4m3 conversion (the
  * one the quantize kernels use).  in [n] fp32, out [n] codes.  Used to check

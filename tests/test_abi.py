@@ -66,8 +66,11 @@ def test_workspace_bytes(lib):
     assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == C + 65536 + 256 + tiles * splits * 16 * 1024
     assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == C + tiles * splits * 16 * 1024
     assert mfp8.mfp8_gemm_workspace_bytes(300, 4096, 4096) == 0
-    # the AUTO choice: split-K for decode sizes, 128-row tiles for mid M, pairs above
-    assert mfp8.mfp8_choose_path(8, 12288, 4096) == mfp8.PATH_SPLITK
+    # the AUTO choice: the one-kernel path up to 16 tokens, split-K to 64,
+    # 128-row tiles for mid M, pairs above
+    assert mfp8.mfp8_choose_path(8, 12288, 4096) == mfp8.PATH_FUSED
+    assert mfp8.mfp8_choose_path(16, 4096, 12288) == mfp8.PATH_FUSED
+    assert mfp8.mfp8_choose_path(17, 4096, 4096) == mfp8.PATH_SPLITK
     assert mfp8.mfp8_choose_path(200, 4096, 4096) == mfp8.PATH_TILED
     assert mfp8.mfp8_choose_path(2048, 4096, 4096) == mfp8.PATH_PAIR
     assert mfp8.mfp8_choose_path(0, 4096, 4096) == mfp8.PATH_AUTO
@@ -112,7 +115,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert call(path=7) == mfp8.ERR_INVALID_ARG
     assert call(path=5) == mfp8.ERR_INVALID_ARG
     assert call(path=mfp8.PATH_FUSED, M=17) == mfp8.ERR_UNSUPPORTED_SHAPE
-    assert call(ws=None) == mfp8.ERR_WORKSPACE  # split-K partials
+    assert call(ws=None, path=mfp8.PATH_SPLITK) == mfp8.ERR_WORKSPACE  # split-K partials
     assert call(path=mfp8.PATH_SPLITK, M=129) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
     assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X

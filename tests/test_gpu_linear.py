@@ -76,6 +76,53 @@ def test_linear_without_codes_out_matches_with():
         assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
+# The one-kernel decode path: channel groups of 16..256 per CTA, one or
+# several 32 KB code windows along K (8 or 16 code rows per K block), a
+# ragged last K block, a partial last channel group (N % 16 == 8), grids
+# above one CTA per SM, and every M from 1 to 16.
+STREAM = [
+    (1, 8, 16), (2, 24, 144), (7, 1032, 4112), (8, 1024, 12288), (9, 6144, 4096), (12, 264, 4992),
+    (16, 24576, 4096), (4, 40960, 256), (13, 520, 1040), (16, 12296, 2064), (5, 4096, 8320),
+]
+
+
+@pytest.mark.parametrize("M,N,K", STREAM)
+def test_fused_stream_geometry(M, N, K):
+    run_case(M, N, K, mfp8.PATH_FUSED, seed=M * 5 + K, flags=mfp8.FLAG_STATIC_WEIGHTS if M % 2 else 0)
+
+
+@pytest.mark.parametrize("M", list(range(1, 17)))
+def test_fused_every_m(M):
+    run_case(M, 4096, 4096, mfp8.PATH_FUSED, seed=100 + M, kind="rowscale" if M > 2 else "normal")
+
+
+def test_fused_back_to_back_on_one_stream():
+    """Consecutive decode kernels overlap on the GPU (the next one starts its
+    weight stream while this one finishes); each reads its activations only
+    after the previous kernel completed.  A chain where each Linear's input is
+    the previous Linear's output must equal the same chain run one call at a
+    time with a synchronisation in between."""
+    M, H = 8, 4096
+    Ws = [mfp8.quantize_weight(W.make_w(H, H, seed=60 + i, device=DEV)) for i in range(6)]
+    x0 = W.make_x(M, H, seed=61, device=DEV)
+    ws = torch.zeros((16,), dtype=torch.uint8, device=DEV)  # the path keeps nothing there
+    torch.cuda.synchronize()
+
+    def chain(sync):
+        x = x0
+        for W8, sw in Ws:
+            x = mfp8.linear(x, W8, sw, workspace=ws, path=mfp8.PATH_FUSED, flags=mfp8.FLAG_STATIC_WEIGHTS)
+            if sync:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return x
+
+    a, b = chain(False), chain(True)
+    assert mfp8.device_status() == mfp8.OK
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.isfinite(a.float()).all()
+
+
 @pytest.mark.parametrize("M,N,K", TILED_ONLY + [(513, 776, 1024), (2048, 1024, 4096)])
 @pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_PAIR])
 def test_linear_tiled_ragged(M, N, K, path):

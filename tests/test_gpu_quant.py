@@ -143,3 +143,15 @@ def test_decode_kernel_codes_every_bf16_magnitude(path):
         q_ref, s_ref = oracle.quantize_rows(blk)
         assert np.array_equal(f32(xs).view(np.uint32), s_ref.view(np.uint32))
         assert np.array_equal(u8(x8), q_ref)
+
+
+def test_divide_free_rounding_matches_ieee_divide_on_every_bf16_pair():
+    """The quantizers round x / s with a multiply by the correctly rounded
+    reciprocal and two fused multiply-adds.  On every absmax a (zero and each
+    positive finite bf16, i.e. every scale a row can have) and every bf16 x
+    with |x| <= a, both signs, the codes equal those of an IEEE divide."""
+    out = torch.zeros(2, dtype=torch.int64, device=DEV)
+    assert mfp8.mfp8_debug_quantize_check(out.data_ptr(), torch.cuda.current_stream().cuda_stream) == mfp8.OK
+    torch.cuda.synchronize()
+    bad, witness = (int(v) for v in out.cpu())
+    assert bad == 0, f"{bad} codes differ; e.g. absmax bits {witness >> 16:#06x}, x bits {witness & 0xffff:#06x}"
