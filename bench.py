@@ -36,6 +36,17 @@ DECODE_MS = (1, 4, 8)
 PREFILL_M = 2048
 
 
+def load_traffic(kernel):
+    """DRAM bytes per launch of `kernel` on the bench's workload, from the
+    committed ncu summary (profiles/roofline_traffic.json), or None."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "roofline_traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f).get(kernel, {}).get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -468,7 +479,7 @@ def main():
         "data": "synthetic", "config": decode_config(),
         "frac_of_hbm": round(value / ctx.world / peaks["hbm_gbs"], 4),
         "roofline": {"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": load_traffic(kt["kernel"]),
                      "kernel": kt["kernel"], "launches_timed": kt["launches"],
                      "avg_launch_us": round(kt["gemm_us"], 3),
                      "bytes_per_launch": round(kt["gemm_bytes"]),

@@ -269,7 +269,9 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
                     mma_f8(tmem_base, sw128_kmajor_desc(a0 + kk * MMA_K), sw128_kmajor_desc(b0 + kk * MMA_K), idesc,
                            (i | kk) != 0);
                 issued_any = true;
-                mma_commit(wempty_bar(stage));
+                // A commit holds up this thread for a few hundred cycles:
+                // release a ring slot only if the producer will refill it.
+                if (i + STAGES < nkb) mma_commit(wempty_bar(stage));
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (ok) {
