@@ -102,7 +102,7 @@ template <class Kern>
 mfp8_status launch_quant(Kern kern, bool dependent, int64_t R, const uint4* x, int64_t K, uint2* q, float* S,
                          unsigned int* zero, int nzero, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(R));
+    cfg.gridDim = dim3(static_cast<unsigned>(R));  // one block per row
     cfg.blockDim = dim3(kQuantThreads);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -117,6 +117,26 @@ mfp8_status launch_quant(Kern kern, bool dependent, int64_t R, const uint4* x, i
     return MFP8_OK;
 }
 
+// The warp-per-row kernel: `blocks` blocks of 8 rows, R rows in all.
+template <class Kern>
+mfp8_status launch_quant(Kern kern, bool dependent, int64_t blocks, int64_t R, const uint4* x, int64_t K, uint2* q,
+                         float* S, unsigned int* zero, int nzero, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, x, R, K, q, S, zero, nzero) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
 template <bool EARLY_TRIGGER>
 mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float* S, unsigned int* zero, int nzero,
                             cudaStream_t stream) {
@@ -124,6 +144,20 @@ mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float*
     const int64_t nvec = K / 8;
     const uint4* x = static_cast<const uint4*>(X);
     uint2* q = static_cast<uint2*>(Q);
+    // Many rows: one warp per row (8 rows per block) while a row fits in a
+    // warp's registers.
+    const int64_t rows_per_block = kQuantThreads / 32;
+    const int64_t wblocks = (R + rows_per_block - 1) / rows_per_block;
+    if (R >= 256 && nvec <= 32 * 16 && wblocks <= INT32_MAX) {
+        if (nvec <= 32 * 4)
+            return launch_quant(quant_rows_warp_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, zero,
+                                nzero, stream);
+        if (nvec <= 32 * 8)
+            return launch_quant(quant_rows_warp_kernel<8, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, zero,
+                                nzero, stream);
+        return launch_quant(quant_rows_warp_kernel<16, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, zero,
+                            nzero, stream);
+    }
     if (nvec <= 256) return launch_quant(quant_rows_reg_kernel<1, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
     if (nvec <= 512) return launch_quant(quant_rows_reg_kernel<2, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
     if (nvec <= 1024) return launch_quant(quant_rows_reg_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
@@ -159,8 +193,6 @@ mfp8_status check_quant_args(const void* X, int64_t R, int64_t K, const void* Q,
 
 // ----------------------------------------------------------------- GEMM --
 
-constexpr int kTiledBN = 256;
-constexpr int kTiledStages = 4;
 
 template <class Kern>
 mfp8_status set_smem(Kern kern, int bytes, int dev, bool* done) {
@@ -173,18 +205,19 @@ mfp8_status set_smem(Kern kern, int bytes, int dev, bool* done) {
     return MFP8_OK;
 }
 
-mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
-                         const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
-                         cudaStream_t stream) {
-    using L = tiled::Layout<kTiledBN, kTiledStages>;
-    auto kern = tiled::gemm_tiled_kernel<kTiledBN, kTiledStages>;
+template <int BN, int STAGES>
+mfp8_status launch_tiled_bn(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
+                            const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                            cudaStream_t stream) {
+    using L = tiled::Layout<BN, STAGES>;
+    auto kern = tiled::gemm_tiled_kernel<BN, STAGES>;
     static bool attr_done[kMaxDevices] = {};
     mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
     if (st != MFP8_OK) return st;
     CUtensorMap tmX, tmW;
     if ((st = make_map_u8(&tmX, X8, M, K, tiled::BM)) != MFP8_OK) return st;
-    if ((st = make_map_u8(&tmW, W8, N, K, kTiledBN)) != MFP8_OK) return st;
-    const int64_t tiles = ((M + tiled::BM - 1) / tiled::BM) * ((N + kTiledBN - 1) / kTiledBN);
+    if ((st = make_map_u8(&tmW, W8, N, K, BN)) != MFP8_OK) return st;
+    const int64_t tiles = ((M + tiled::BM - 1) / tiled::BM) * ((N + BN - 1) / BN);
     const unsigned grid = static_cast<unsigned>(tiles < info.sm_count ? tiles : info.sm_count);
 
     cudaLaunchConfig_t cfg = {};
@@ -203,6 +236,28 @@ mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K,
         return MFP8_ERR_CUDA;
     }
     return MFP8_OK;
+}
+
+// The 1-CTA kernel's tile width: 256 when that already gives a CTA to most
+// SMs, else the widest of 128, 64, 32 that does (narrower tiles re-read the
+// X8 row panel more often from L2, but a mid-sized M with 256-wide tiles
+// leaves most SMs idle: M = 128, N = 4096 is 16 tiles).
+int tiled_tile_width(int64_t M, int64_t N, const DeviceInfo& info) {
+    const int64_t mt = (M + tiled::BM - 1) / tiled::BM;
+    for (int bn : {256, 128, 64})
+        if (mt * ((N + bn - 1) / bn) * 4 >= int64_t(info.sm_count) * 3) return bn;
+    return 32;
+}
+
+mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
+                         const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                         cudaStream_t stream) {
+    switch (tiled_tile_width(M, N, info)) {
+        case 256: return launch_tiled_bn<256, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+        case 128: return launch_tiled_bn<128, 6>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+        case 64: return launch_tiled_bn<64, 8>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+        default: return launch_tiled_bn<32, 10>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    }
 }
 
 // Clusters of `S` CTAs of `kern` (with `smem` bytes each) that the device
@@ -300,11 +355,18 @@ constexpr int64_t kSkinnyMaxM = skinny::kMaxM;
 constexpr int64_t kStreamMaxM = stream::kMaxM;
 constexpr int kSkinnyStages = 4;
 
+int sm_count_for_sizing();
+
 int choose_path(int64_t M, int64_t N, int64_t K) {
     (void)K;
     if (M <= kStreamMaxM) return MFP8_PATH_FUSED;
     if (M <= 64 && (N + 255) / 256 <= 4096) return MFP8_PATH_SPLITK;
     if (M < 256) return MFP8_PATH_TILED;
+    // Too few 256 x 256 pair tiles to occupy half the CTA pairs (the k/v
+    // projections at M = 2048 make 32): narrower single-CTA tiles fill the
+    // GPU instead.
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    if (pair_tiles * 4 < sm_count_for_sizing()) return MFP8_PATH_TILED;
     return MFP8_PATH_PAIR;
 }
 

@@ -192,6 +192,53 @@ quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict_
     }
 }
 
+// One warp per row, 8 rows per block, for rows of at most 32 * VPL 16-byte
+// vectors (K <= 256 * VPL): the row stays in registers, the absmax is a warp
+// reduction, and no block barrier holds up the other rows.  Loads and stores
+// are lane-contiguous (512 and 256 bytes per instruction).  EARLY_TRIGGER,
+// `zero` and `nzero` as in quant_rows_reg_kernel.
+template <int VPL, bool EARLY_TRIGGER>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_rows_warp_kernel(const uint4* __restrict__ X, int64_t R, int64_t K, uint2* __restrict__ Q,
+                       float* __restrict__ S, unsigned int* __restrict__ zero, int nzero) {
+    if (EARLY_TRIGGER) {
+        grid_launch_dependents();
+        grid_dependency_wait();
+    }
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < nzero; i += kQuantThreads) zero[i] = 0u;
+    const int64_t row = int64_t(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5);
+    if (row >= R) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t nvec = K >> 3;
+    const uint4* xr = X + row * nvec;
+    uint4 v[VPL];
+    uint32_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int64_t j = lane + 32 * i;
+        v[i] = j < nvec ? __ldg(xr + j) : make_uint4(0, 0, 0, 0);
+        acc = absmax_bits_u4(v[i], acc);
+    }
+    const uint32_t amax = __reduce_max_sync(0xffffffffu, max(acc & 0xffffu, acc >> 16));
+    const float s = scale_from_absmax_bits(amax);
+    const float r = __frcp_rn(s);
+    if (lane == 0) S[row] = s;
+    uint2* qr = Q + row * nvec;
+    if (s < kFmaMinScale) {
+        for (int i = 0; i < VPL; ++i) {
+            const int64_t j = lane + 32 * i;
+            if (j < nvec) qr[j] = quantize8_div_call(v[i], s);
+        }
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int64_t j = lane + 32 * i;
+        if (j < nvec) qr[j] = quantize8_fast(v[i], s, r);
+    }
+}
+
 // Any K: two passes over the row (the second one is served by L2).
 template <bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)

@@ -55,6 +55,16 @@ LAYER_LINEARS = (
 )
 MLP_LINEARS = LAYER_LINEARS[4:]
 
+# The same layer with the projections that read the same input packed into
+# one Linear, as the README's packed modules do (qkv_proj, gate_up_proj):
+# output channels concatenate, and so do their per-channel scales.
+PACKED_LAYER_LINEARS = (
+    LinearShape("qkv_proj", HIDDEN, HIDDEN + 2 * KV_WIDTH),
+    LinearShape("o_proj", HIDDEN, HIDDEN),
+    LinearShape("gate_up_proj", HIDDEN, 2 * INTERMEDIATE),
+    LinearShape("down_proj", INTERMEDIATE, HIDDEN),
+)
+
 
 def generator(seed: int, stream: int, device) -> torch.Generator:
     g = torch.Generator(device=device)

@@ -60,6 +60,26 @@ def test_quantize_edge_rows():
     check_rows(x)
 
 
+@pytest.mark.parametrize("K", [64, 1040, 2048, 4096])
+def test_quantize_edge_rows_warp_kernel(K):
+    """Many rows (the warp-per-row kernel): the edge rows above spread among
+    ordinary ones, with ragged K, plus rows whose scale is below 2^-64 (the
+    quantizer's divide branch) and a row whose absmax is a bf16 subnormal."""
+    g = torch.Generator().manual_seed(K)
+    x = torch.randn(300, K, generator=g)
+    x[3] = 0
+    x[17] = -0.0
+    x[40] = 0
+    x[40, 5] = 1e-40
+    x[41] *= 1e-30                      # scale about 1e-32: divide branch
+    x[42] = 0
+    x[42, K - 1] = -3e-25
+    x[99] = 448.0
+    x[100, : K // 2] = 3.0e38
+    x[299] *= 1e4
+    check_rows(x.to(torch.bfloat16).to(DEV))
+
+
 @pytest.mark.parametrize("N,K", [(4096, 4096), (12288, 4096), (4096, 12288), (1024, 4096), (8, 16)])
 def test_quantize_weight_bitexact(N, K):
     check_rows(W.make_w(N, K, seed=1, stream=N + K, device=DEV), which="weight")
