@@ -12,8 +12,10 @@
 //     B columns of both CTAs, and each CTA's TMEM receives its 128 rows of D;
 //   - tcgen05.commit with a two-CTA mask frees the ring slot in both CTAs and
 //     hands each CTA its finished accumulator;
-//   - each CTA's four epilogue warps scale and store their 128 rows and
-//     report back to the even CTA, which then reuses that accumulator.
+//   - each CTA's four epilogue warps scale their 128 rows, stage 32 x 32
+//     bf16 blocks in shared memory and store them with TMA (coalesced,
+//     asynchronous), and report back to the even CTA, which then reuses
+//     that accumulator.
 // With BN = 256, per CTA and k-block the ring takes 32 KB for 128 x 256 x 128
 // MACs, two thirds of the bytes a single-CTA 128 x 256 tile needs, so a
 // six-deep ring fits and L2 -> SM traffic drops by a third.  Two fp32
@@ -49,20 +51,17 @@ struct Layout {
     static constexpr int CTA_STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = STAGES * A_BYTES;
-    static constexpr int BAR_OFF = STAGES * CTA_STAGE_BYTES;
+    static constexpr int STG_OFF = STAGES * CTA_STAGE_BYTES;     // epilogue staging: 4 warps x 2 x 2 KB
+    static constexpr int BAR_OFF = STG_OFF + 4 * 4096;
     static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
 };
 
-__device__ __forceinline__ __nv_bfloat162 scale2(float a, float b, float sa, float sw0, float sw1) {
-    return __floats2bfloat162_rn(a * sa * sw0, b * sa * sw1);
-}
-
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                 const float* __restrict__ s_a, const float* __restrict__ s_w,
+                 const __grid_constant__ CUtensorMap tmY, const float* __restrict__ s_a, const float* __restrict__ s_w,
                  __nv_bfloat16* __restrict__ Y, int M, int N, int K) {
     using L = Layout<BN, STAGES>;
     constexpr int TMEM_COLS = L::TMEM_COLS;
@@ -104,6 +103,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         fence_mbar_init();
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
@@ -181,6 +181,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const uint32_t q = warp & 3u;
         const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0);
         const uint32_t leader_tempty1 = mapa_shared(tempty_bar(1), 0);
+        TmaEpilogue ep{&tmY, sbase + uint32_t(L::STG_OFF) + q * 4096u};
         int local = 0;
         for (int tile = pair_id; tile < num_tiles; tile += num_pairs, ++local) {
             const int acc = local & 1;
@@ -188,41 +189,21 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) break;
             tc_fence_after();
             const int tm = tile / n_tiles, tn = tile % n_tiles;
-            const int row = tm * BM + int(cr) * HALF + int(q * 32 + lane);
-            const bool row_ok = row < M;
-            const float sa = row_ok ? __ldcg(s_a + row) : 0.0f;  // written by the previous kernel
-            __nv_bfloat16* yrow = Y + int64_t(row) * N;
+            const int row0 = tm * BM + int(cr) * HALF + int(q * 32);
+            const int row = row0 + int(lane);
+            const float sa = row < M ? __ldcg(s_a + row) : 0.0f;  // written by the previous kernel
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + ((q * 32u) << 16) + uint32_t(acc * BN + c * 32), r);
                 tmem_wait_ld();
-                const int col0 = tn * BN + c * 32;
-                if (row_ok) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        const int col = col0 + j;
-                        if (col < N) {  // N % 8 == 0
-                            const float4 w0 = __ldg(reinterpret_cast<const float4*>(s_w + col));
-                            const float4 w1 = __ldg(reinterpret_cast<const float4*>(s_w + col + 4));
-                            __nv_bfloat162 o0 = scale2(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]), sa, w0.x, w0.y);
-                            __nv_bfloat162 o1 = scale2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), sa, w0.z, w0.w);
-                            __nv_bfloat162 o2 = scale2(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]), sa, w1.x, w1.y);
-                            __nv_bfloat162 o3 = scale2(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]), sa, w1.z, w1.w);
-                            uint4 pk;
-                            pk.x = *reinterpret_cast<uint32_t*>(&o0);
-                            pk.y = *reinterpret_cast<uint32_t*>(&o1);
-                            pk.z = *reinterpret_cast<uint32_t*>(&o2);
-                            pk.w = *reinterpret_cast<uint32_t*>(&o3);
-                            *reinterpret_cast<uint4*>(yrow + col) = pk;
-                        }
-                    }
-                }
+                ep.put(r, sa, s_w, tn * BN + c * 32, row0, M, N, lane);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0);
         }
+        ep.drain(lane);
     }
 
     tc_fence_before();

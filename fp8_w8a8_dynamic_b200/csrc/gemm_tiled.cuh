@@ -14,7 +14,8 @@
 //              tcgen05.commit releases ring slots and hands finished
 //              accumulators to the epilogue;
 //   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter of the
-//              accumulator, scale by s_a[m] * s_w[n], round to bf16, store.
+//              accumulator, scale by s_a[m] * s_w[n], round to bf16, stage
+//              32 x 32 blocks in shared memory and store them with TMA.
 // The two accumulators let the epilogue of tile i overlap the main loop of
 // tile i+1.  Tiles are walked n-fastest so that one wave of CTAs shares
 // a few X8 row panels and the whole W8 stays L2-resident.
@@ -43,7 +44,8 @@ struct Layout {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = STAGES * A_BYTES;
-    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+    static constexpr int STG_OFF = STAGES * STAGE_BYTES;  // epilogue staging: 4 warps x 2 x 2 KB
+    static constexpr int BAR_OFF = STG_OFF + 4 * 4096;
     // full[S], empty[S], tfull[2], tempty[2], drain
     static constexpr int NUM_BARS = 2 * STAGES + 5;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem base, abort flag
@@ -54,13 +56,10 @@ struct Layout {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "MMA N for M=128");
 };
 
-__device__ __forceinline__ __nv_bfloat162 scale2(float a, float b, float sa, float sw0, float sw1) {
-    return __floats2bfloat162_rn(a * sa * sw0, b * sa * sw1);
-}
-
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                  const __grid_constant__ CUtensorMap tmY,
                   const float* __restrict__ s_a, const float* __restrict__ s_w,
                   __nv_bfloat16* __restrict__ Y, int M, int N, int K) {
     using L = Layout<BN, STAGES>;
@@ -180,8 +179,10 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
         }
     } else {
-        // Epilogue: warp w may read TMEM lanes [32*(w%4), 32*(w%4)+32).
+        // Epilogue: warp w may read TMEM lanes [32*(w%4), 32*(w%4)+32); the
+        // rows go out through shared memory and TMA stores (TmaEpilogue).
         const uint32_t q = warp & 3u;
+        TmaEpilogue ep{&tmY, sbase + uint32_t(L::STG_OFF) + q * 4096u};
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int acc = local & 1;
@@ -189,41 +190,21 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) break;
             tc_fence_after();
             const int tm = tile / n_tiles, tn = tile % n_tiles;
-            const int row = tm * BM + int(q * 32 + lane);
-            const bool row_ok = row < M;
-            const float sa = row_ok ? __ldcg(s_a + row) : 0.0f;  // written by the previous kernel
-            __nv_bfloat16* yrow = Y + int64_t(row) * N;
+            const int row0 = tm * BM + int(q * 32);
+            const int row = row0 + int(lane);
+            const float sa = row < M ? __ldcg(s_a + row) : 0.0f;  // written by the previous kernel
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + ((q * 32u) << 16) + uint32_t(acc * BN + c * 32), r);
                 tmem_wait_ld();
-                const int col0 = tn * BN + c * 32;
-                if (row_ok) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        const int col = col0 + j;
-                        if (col < N) {  // N % 8 == 0: a group of 8 is all in or all out
-                            const float4 w0 = __ldg(reinterpret_cast<const float4*>(s_w + col));
-                            const float4 w1 = __ldg(reinterpret_cast<const float4*>(s_w + col + 4));
-                            __nv_bfloat162 o0 = scale2(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]), sa, w0.x, w0.y);
-                            __nv_bfloat162 o1 = scale2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), sa, w0.z, w0.w);
-                            __nv_bfloat162 o2 = scale2(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]), sa, w1.x, w1.y);
-                            __nv_bfloat162 o3 = scale2(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]), sa, w1.z, w1.w);
-                            uint4 pk;
-                            pk.x = *reinterpret_cast<uint32_t*>(&o0);
-                            pk.y = *reinterpret_cast<uint32_t*>(&o1);
-                            pk.z = *reinterpret_cast<uint32_t*>(&o2);
-                            pk.w = *reinterpret_cast<uint32_t*>(&o3);
-                            *reinterpret_cast<uint4*>(yrow + col) = pk;
-                        }
-                    }
-                }
+                ep.put(r, sa, s_w, tn * BN + c * 32, row0, M, N, lane);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));
         }
+        ep.drain(lane);
     }
 
     tc_fence_before();

@@ -87,6 +87,19 @@ mfp8_status make_map_u8(CUtensorMap* map, const void* base, int64_t rows, int64_
     return r == CUDA_SUCCESS ? MFP8_OK : MFP8_ERR_CUDA;
 }
 
+// Y [rows, cols] bf16 for the TMA-store epilogue: 32 x 32 boxes, 64-byte
+// rows with the 64-byte swizzle (cols % 8 == 0, so rows are 16-byte aligned).
+mfp8_status make_map_y(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MFP8_OK : MFP8_ERR_CUDA;
+}
+
 bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
     return a0 < b0 + nb && b0 < a0 + na;
@@ -214,9 +227,10 @@ mfp8_status launch_tiled_bn(const void* X8, const float* s_a, int64_t M, int64_t
     static bool attr_done[kMaxDevices] = {};
     mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
     if (st != MFP8_OK) return st;
-    CUtensorMap tmX, tmW;
+    CUtensorMap tmX, tmW, tmY;
     if ((st = make_map_u8(&tmX, X8, M, K, tiled::BM)) != MFP8_OK) return st;
     if ((st = make_map_u8(&tmW, W8, N, K, BN)) != MFP8_OK) return st;
+    if ((st = make_map_y(&tmY, Y, M, N)) != MFP8_OK) return st;
     const int64_t tiles = ((M + tiled::BM - 1) / tiled::BM) * ((N + BN - 1) / BN);
     const unsigned grid = static_cast<unsigned>(tiles < info.sm_count ? tiles : info.sm_count);
 
@@ -230,7 +244,7 @@ mfp8_status launch_tiled_bn(const void* X8, const float* s_a, int64_t M, int64_t
     attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, tmY, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
                            int(K)) != cudaSuccess) {
         cudaGetLastError();
         return MFP8_ERR_CUDA;
@@ -300,9 +314,10 @@ mfp8_status launch_pair_bn(const void* X8, const float* s_a, int64_t M, int64_t 
     static bool attr_done[kMaxDevices] = {};
     mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
     if (st != MFP8_OK) return st;
-    CUtensorMap tmX, tmW;
+    CUtensorMap tmX, tmW, tmY;
     if ((st = make_map_u8(&tmX, X8, M, K, pair::HALF)) != MFP8_OK) return st;
     if ((st = make_map_u8(&tmW, W8, N, K, BN / 2)) != MFP8_OK) return st;
+    if ((st = make_map_y(&tmY, Y, M, N)) != MFP8_OK) return st;
     const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + BN - 1) / BN);
     // The grid is persistent: only as many pairs as can be resident at once.
     int64_t max_pairs = max_active_clusters(kern, 2, L::SMEM_BYTES, pair::kThreads, dev);
@@ -323,7 +338,7 @@ mfp8_status launch_pair_bn(const void* X8, const float* s_a, int64_t M, int64_t 
     attr[1].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, tmY, s_a, s_w, static_cast<__nv_bfloat16*>(Y), int(M), int(N),
                            int(K)) != cudaSuccess) {
         cudaGetLastError();
         return MFP8_ERR_CUDA;

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "status.cuh"
 
@@ -106,6 +107,31 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
+// 2-D tile store shared -> global (bulk group completion).  (x, y) =
+// (innermost coordinate in elements, row); rows and columns past the
+// tensor's extent are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N of this thread's committed bulk groups still read
+// their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until at most N of this thread's committed bulk groups are incomplete
+// (their global writes done).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both
 // addresses 16-byte aligned), completion signalled on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -122,6 +148,70 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+
+// --------------------------------------------------- coalesced epilogue --
+// The epilogue of one warp of an accumulator read with tcgen05.ld 32x32b:
+// lane i holds output row row0 + i, 32 fp32 columns per chunk.  Each chunk
+// is scaled by sa (this lane's row scale) and s_w[col], rounded to bf16,
+// written to a 32 x 32 bf16 staging block (64-byte rows with the 64-byte
+// swizzle, so the 16-byte stores of the 32 lanes hit all banks), and stored
+// to global memory with one TMA 2-D store (box 32 x 32, SWIZZLE_64B), which
+// clips rows >= M and columns >= N.  Two staging blocks alternate; `chunk`
+// counts this warp's chunks across calls so the alternation continues.
+struct TmaEpilogue {
+    const CUtensorMap* tmY;
+    uint32_t stage;  // shared address of this warp's 2 x 2 KB, 1024-aligned
+    uint32_t chunk = 0;
+
+    __device__ __forceinline__ void put(const uint32_t (&acc)[32], float sa, const float* __restrict__ s_w,
+                                        int col0, int row0, int M, int N, uint32_t lane) {
+        if (col0 >= N || row0 >= M) return;  // the whole block is outside Y (warp-uniform)
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+            const int col = col0 + j;
+            float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
+            if (col < N) {  // N % 8 == 0: a group of 8 is all in or all out
+                w0 = __ldg(reinterpret_cast<const float4*>(s_w + col));
+                w1 = __ldg(reinterpret_cast<const float4*>(s_w + col + 4));
+            }
+            const float sc[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+            for (int t = 0; t < 8; t += 2) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(acc[j + t]) * sa * sc[t],
+                                                               __uint_as_float(acc[j + t + 1]) * sa * sc[t + 1]);
+                pk[(j + t) / 2] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+        }
+        const uint32_t buf = stage + (chunk & 1u) * 2048u;
+        if (chunk >= 2) {
+            if (lane == 0) bulk_wait_group_read<1>();  // the store that read this block two chunks ago
+            __syncwarp();
+        }
+        const uint32_t row = buf + lane * 64u;
+#pragma unroll
+        for (uint32_t c = 0; c < 4; ++c) {
+            const uint32_t dst = row + ((c ^ ((lane >> 1) & 3u)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                         ::"r"(dst), "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                         : "memory");
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> TMA reads
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmY, buf, col0, row0);
+            bulk_commit_group();
+        }
+        ++chunk;
+    }
+
+    // Every store of this warp written to global memory (before the CTA
+    // leaves or its staging memory is reused for anything else).
+    __device__ __forceinline__ void drain(uint32_t lane) {
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
+};
 
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
