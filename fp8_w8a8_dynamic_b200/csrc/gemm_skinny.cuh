@@ -5,24 +5,17 @@
 //
 // At decode sizes the Linear is a stream of W8 through the SMs, and what
 // bounds a tcgen05 kernel is how many weight bytes one MMA instruction
-// consumes: a tcgen05.mma takes about the same time whether its N is 16 or
-// 256, so the weights are the MMA's B operand (N = 256 output channels per
-// instruction, 8 KB of W8) and the tokens its A operand (M = 128 rows, of
-// which only the first M are real; the rest are zeros).
+// consumes: the weights are the MMA's B operand (N = 256 output channels
+// per instruction, 8 KB of W8) and the tokens its A operand (M = 128 rows,
+// of which only the first M are real; the rest are zeros).
 //
 // Grid: tiles (256 channels each) x splits (K ranges), at most one CTA per
 // SM, no clusters.  Each CTA
 //   1. streams its W8 K-range into a 4-stage TMA ring straight away (the
 //      weights do not depend on the kernel before it when declared static);
-//   2. gets the activation codes of its K-range:
-//        QUANT = false: loads them, per stage, from the codes the quantize
-//                       kernel launched just before wrote (TMA; rows >= M
-//                       are filled with zeros and cost no reads);
-//        QUANT = true (M <= 16): reads the whole rows of X (BF16) itself,
-//                       takes each token's absmax and scale (the same rule
-//                       and device functions as the quantize kernel), and
-//                       its four otherwise idle warps write the codes of each
-//                       k-block into the ring, next to the weights;
+//   2. loads the activation codes of its K-range, per stage, from the codes
+//      the quantize kernel launched just before wrote (TMA; rows >= M are
+//      filled with zeros and cost no reads);
 //   3. issues 4 MMAs per 128-byte k-block into one fp32 TMEM accumulator;
 //   4. writes rows 0..M-1 of the accumulator (fp32) to the workspace
 //      ([tile][split][M][256]), fences, and counts itself on the tile's
@@ -51,7 +44,6 @@ constexpr int BK = 128;
 constexpr int MMA_K = 32;
 constexpr int kThreads = 192;
 constexpr int kMaxM = 128;    // all four epilogue warps read their TMEM lanes
-constexpr int kMaxFusedM = 16;
 constexpr int kMaxSplits = 16;
 
 template <int STAGES>
@@ -65,8 +57,7 @@ struct Layout {
     static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 3;  // full, empty, tfull, drain, reduce
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem holder, abort, last flag
-    static constexpr int SCALE_OFF = (MISC_OFF + 16 + 15) / 16 * 16;               // amax bits, s, 1/s [kMaxFusedM]
-    static constexpr int SW_OFF = (SCALE_OFF + 3 * kMaxFusedM * 4 + 15) / 16 * 16;  // s_w of the tile [BN], read as float4
+    static constexpr int SW_OFF = (MISC_OFF + 16 + 15) / 16 * 16;  // s_w of the tile [BN], read as float4
     static constexpr int SA_OFF = SW_OFF + BN * 4;                                 // s_a [kMaxM]
     static constexpr int SMEM_BYTES = SA_OFF + kMaxM * 4 + 1024;
     static_assert(SW_OFF % 16 == 0 && BAR_OFF % 8 == 0 && RING_BYTES % 1024 == 0, "shared-memory alignment");
@@ -74,19 +65,16 @@ struct Layout {
 };
 
 struct Args {
-    const __nv_bfloat16* X;  // QUANT: activations [M, K]
-    const float* s_a;        // !QUANT: scales from the quantize kernel
+    const float* s_a;        // activation scales from the quantize kernel
     const float* s_w;
     __nv_bfloat16* Y;
     float* partial;
     unsigned int* counters;
-    uint8_t* x8_out;         // QUANT: optional copy of the codes (tile 0 writes them)
-    float* sa_out;           // QUANT: optional copy of the scales
     int M, N, K;
     int weights_static;
 };
 
-template <int STAGES, bool QUANT>
+template <int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const Args args) {
@@ -105,9 +93,6 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
-    uint32_t* amax_sm = reinterpret_cast<uint32_t*>(smem + L::SCALE_OFF);
-    float* s_sm = reinterpret_cast<float*>(amax_sm + kMaxFusedM);
-    float* r_sm = s_sm + kMaxFusedM;
     float* sw_sm = reinterpret_cast<float*>(smem + L::SW_OFF);
     float* sa_sm = reinterpret_cast<float*>(smem + L::SA_OFF);
 
@@ -126,8 +111,7 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            // QUANT: the four code-writing warps arrive too.
-            mbar_init(full_bar(s), QUANT ? 5 : 1);
+            mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(tfull_bar, 1);
@@ -136,22 +120,8 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
-        if (!QUANT) tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
-    }
-    if (QUANT) {
-        // Code rows >= M stay zero in every ring slot; rows < M are rewritten
-        // for each k-block.  The row absmax starts at zero.
-        const int pad_chunks = (BM - M) * (BK / 16);
-        for (int i = int(threadIdx.x); i < STAGES * pad_chunks; i += kThreads) {
-            const int s = i / pad_chunks;
-            const int rem = i % pad_chunks;
-            const int row = M + rem / (BK / 16), chunk = rem % (BK / 16);
-            *reinterpret_cast<uint4*>(smem + L::A_OFF + s * L::A_BYTES + row * BK + chunk * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-        }
-        if (threadIdx.x < kMaxFusedM) amax_sm[threadIdx.x] = 0u;
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zero rows -> tensor-core reads
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), L::TMEM_COLS);
@@ -165,66 +135,26 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     // grid to finish before it touches memory.
     grid_launch_dependents();
 
-    if (QUANT) {
-        // Weights first (static weights do not depend on the previous kernel).
-        if (threadIdx.x == 0) {
-            const uint64_t policy_w = l2_policy_evict_first();
-            if (!args.weights_static) grid_dependency_wait();
-            for (int i = 0; i < prologue; ++i) {
-                mbar_arrive_expect_tx(full_bar(i), L::B_BYTES);
-                tma_load_2d_hint(sB + i * L::B_BYTES, &tmW, full_bar(i), (kb_begin + i) * BK, n0, policy_w);
-            }
-        }
-        // X comes from earlier work on the stream.  Row absmax over all of K.
-        grid_dependency_wait();
-        const int groups = K / 8;
-        uint32_t run_max = 0;
-        int run_row = -1;
-        for (int e = int(threadIdx.x); e < M * groups; e += kThreads) {
-            const int m = e / groups;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(args.X + int64_t(m) * K) + (e % groups));
-            const uint32_t a = absmax_bits_u4(v, 0u);
-            const uint32_t a16 = max(a & 0xffffu, a >> 16);
-            if (m != run_row) {
-                if (run_row >= 0) atomicMax(amax_sm + run_row, run_max);
-                run_row = m;
-                run_max = 0;
-            }
-            run_max = max(run_max, a16);
-        }
-        if (run_row >= 0) atomicMax(amax_sm + run_row, run_max);
-        __syncthreads();
-        if (int(threadIdx.x) < M) {
-            const float s = scale_from_absmax_bits(amax_sm[threadIdx.x]);
-            s_sm[threadIdx.x] = s;
-            r_sm[threadIdx.x] = __frcp_rn(s);
-            if (args.sa_out && tile == 0 && split == 0) args.sa_out[threadIdx.x] = s;
-        }
-        __syncthreads();
-    }
-
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t policy_w = l2_policy_evict_first();
             uint32_t issued_parity = 0;
-            if (!QUANT) {
-                if (!args.weights_static) grid_dependency_wait();
-                for (int i = 0; i < prologue; ++i) {
-                    mbar_arrive_expect_tx(full_bar(i), L::STAGE_BYTES);
-                    tma_load_2d_hint(sB + i * L::B_BYTES, &tmW, full_bar(i), (kb_begin + i) * BK, n0, policy_w);
-                }
-                grid_dependency_wait();  // the codes come from the quantize kernel
-                for (int i = 0; i < prologue; ++i)
-                    tma_load_2d(sA + i * L::A_BYTES, &tmX, full_bar(i), (kb_begin + i) * BK, 0);
+            if (!args.weights_static) grid_dependency_wait();
+            for (int i = 0; i < prologue; ++i) {
+                mbar_arrive_expect_tx(full_bar(i), L::STAGE_BYTES);
+                tma_load_2d_hint(sB + i * L::B_BYTES, &tmW, full_bar(i), (kb_begin + i) * BK, n0, policy_w);
             }
+            grid_dependency_wait();  // the codes come from the quantize kernel
+            for (int i = 0; i < prologue; ++i)
+                tma_load_2d(sA + i * L::A_BYTES, &tmX, full_bar(i), (kb_begin + i) * BK, 0);
             uint32_t issued_mask = (1u << prologue) - 1u;
             int stage = prologue % STAGES;
             uint32_t phase = prologue == STAGES ? 1u : 0u;
             for (int i = prologue; i < nkb; ++i) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) break;
-                mbar_arrive_expect_tx(full_bar(stage), QUANT ? L::B_BYTES : L::STAGE_BYTES);
+                mbar_arrive_expect_tx(full_bar(stage), L::STAGE_BYTES);
                 tma_load_2d_hint(sB + stage * L::B_BYTES, &tmW, full_bar(stage), (kb_begin + i) * BK, n0, policy_w);
-                if (!QUANT) tma_load_2d(sA + stage * L::A_BYTES, &tmX, full_bar(stage), (kb_begin + i) * BK, 0);
+                tma_load_2d(sA + stage * L::A_BYTES, &tmX, full_bar(stage), (kb_begin + i) * BK, 0);
                 issued_mask |= 1u << stage;
                 issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -270,40 +200,10 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         {
             // The scales the last arriver applies, staged while the weights
             // stream (s_a comes from the quantize kernel: wait for it).
-            if (!QUANT) grid_dependency_wait();
+            grid_dependency_wait();
             const int t = int(threadIdx.x) - 64;  // 0..127
             for (int c = t; c < BN; c += 128) sw_sm[c] = (n0 + c < N) ? __ldcg(args.s_w + n0 + c) : 0.f;
-            for (int m = t; m < M; m += 128) sa_sm[m] = QUANT ? s_sm[m] : __ldcg(args.s_a + m);
-        }
-        if (QUANT) {
-            // Warps 2-5 write the codes of each k-block into the ring slot the
-            // weights of that k-block land in: M rows x 16 groups of 8.
-            const int t = int(threadIdx.x) - 64;  // 0..127
-            const bool write_out = args.x8_out != nullptr && tile == 0;
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int i = 0; i < nkb; ++i) {
-                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) break;
-                uint8_t* a_tile = smem + L::A_OFF + stage * L::A_BYTES;
-                const int kb = kb_begin + i;
-                for (int e = t; e < M * (BK / 8); e += 128) {
-                    const int m = e / (BK / 8);
-                    const int kc = (e % (BK / 8)) * 8;  // column within the k-block
-                    const int k = kb * BK + kc;
-                    uint2 code = make_uint2(0u, 0u);
-                    if (k < K) {
-                        code = quantize8(__ldg(reinterpret_cast<const uint4*>(args.X + int64_t(m) * K + k)), s_sm[m],
-                                         r_sm[m]);
-                        if (write_out) *reinterpret_cast<uint2*>(args.x8_out + int64_t(m) * K + k) = code;
-                    }
-                    const int chunk = (kc >> 4) ^ (m & 7);
-                    *reinterpret_cast<uint2*>(a_tile + m * BK + chunk * 16 + (kc & 15)) = code;
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // codes -> tensor-core reads
-                __syncwarp();
-                if (lane == 0) mbar_arrive(full_bar(stage));
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            }
+            for (int m = t; m < M; m += 128) sa_sm[m] = __ldcg(args.s_a + m);
         }
         // Warp w reads TMEM lanes [32 (w % 4), 32 (w % 4) + 32): token rows.
         const int m = int(q * 32 + lane);

@@ -290,6 +290,15 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         if (!args.weights_static) grid_dependency_wait();
         sw_sm[t] = (n0 + t < N) ? __ldg(args.s_w + n0 + t) : 0.f;  // 128 threads, 128 channels
         if (t < kMaxM) amax_loc[t] = 0u;
+        // Ask L2 for this CTA's slice of X (M rows of (k1 - k0) * 2 bytes)
+        // while the previous kernel finishes.  A prefetch returns nothing
+        // to the thread: the values used are read after the wait below, so
+        // X may still be the previous kernel's output.
+        if (t < M) {
+            const __nv_bfloat16* p = args.X + int64_t(t) * K + k0;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                         ::"l"(reinterpret_cast<uint64_t>(p)), "r"(uint32_t(k1 - k0) * 2u) : "memory");
+        }
         // X may be the previous kernel's output.
         grid_dependency_wait();
 

@@ -446,33 +446,26 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool codes, bool split_k, int sm
     return p;
 }
 
-// QUANT: X is BF16 and the kernel quantizes it (M <= 16); otherwise X8/s_a
-// are the codes of the quantize pass.
-template <bool QUANT>
-mfp8_status launch_skinny(const void* X, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+// The split-K GEMM on the codes X8 / scales s_a of the quantize pass.
+mfp8_status launch_skinny(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
                           int64_t N, void* Y, float* partial, unsigned int* counters, const Plan& plan,
-                          bool weights_static, bool dependent, void* x8_out, float* sa_out, int dev,
-                          cudaStream_t stream) {
+                          bool weights_static, bool dependent, int dev, cudaStream_t stream) {
     using L = skinny::Layout<kSkinnyStages>;
-    auto kern = skinny::gemm_skinny_kernel<kSkinnyStages, QUANT>;
+    auto kern = skinny::gemm_skinny_kernel<kSkinnyStages>;
     static bool attr_done[kMaxDevices] = {};
     mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
     if (st != MFP8_OK) return st;
     CUtensorMap tmX, tmW;
     if ((st = make_map_u8(&tmW, W8, N, K, skinny::BN)) != MFP8_OK) return st;
-    if (QUANT) tmX = tmW;  // unused
-    else if ((st = make_map_u8(&tmX, X, M, K, skinny::BM)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmX, X8, M, K, skinny::BM)) != MFP8_OK) return st;
     if (plan.tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
 
     skinny::Args args;
-    args.X = static_cast<const __nv_bfloat16*>(X);
     args.s_a = s_a;
     args.s_w = s_w;
     args.Y = static_cast<__nv_bfloat16*>(Y);
     args.partial = partial;
     args.counters = counters;
-    args.x8_out = static_cast<uint8_t*>(x8_out);
-    args.sa_out = sa_out;
     args.M = int(M);
     args.N = int(N);
     args.K = int(K);
@@ -583,9 +576,9 @@ mfp8_status run_gemm(const void* X8, const float* s_a, int64_t M, int64_t K, con
     if (path == MFP8_PATH_PAIR) return launch_pair(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
     if (path == MFP8_PATH_SPLITK) {
         uint8_t* base = static_cast<uint8_t*>(ws);
-        return launch_skinny<false>(X8, s_a, M, K, W8, s_w, N, Y, reinterpret_cast<float*>(base + plan.part_off),
-                                    reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static,
-                                    dependent, nullptr, nullptr, dev, stream);
+        return launch_skinny(X8, s_a, M, K, W8, s_w, N, Y, reinterpret_cast<float*>(base + plan.part_off),
+                             reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static, dependent,
+                             dev, stream);
     }
     return MFP8_ERR_INVALID_ARG;
 }
