@@ -302,7 +302,8 @@ def stack_sweep(torch, mfp8, W, device, steps, warmup, dist_ctx):
     torch.cuda.synchronize()
     wbytes = sum(lin.N * lin.K + 4 * lin.N for lin, _, _ in weights)
     out = {"workload": "252-Linear stack (36 self-attention layers x 7, ~7 GB of e4m3 weights, per-layer std "
-                       "jitter +-20%), seed 4", "weight_bytes": wbytes, "by_M": {}}
+                       "jitter +-20%), seed 4", "weight_bytes": wbytes,
+           "rates": "per GPU (under torchrun every rank sweeps the same stack)", "by_M": {}}
     for M in W.WORKLOADS[4]["Ms"]:
         xs = {K: W.make_x(M, K, seed=seed, stream=K, device=device) for K in {lin.K for lin, _, _ in weights}}
         ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=device) for N in {lin.N for lin, _, _ in weights}}
@@ -401,18 +402,25 @@ def oracle_decode_sample(budget_s=12.0):
 # ---------------------------------------------------------------- dist --
 
 class DistCtx:
-    def __init__(self, torch):
+    """One process per GPU: rank bookkeeping, the barrier around the timed
+    region and the max over ranks of a timing.  Nothing on the data path
+    goes through it; each rank's batch is its own."""
+
+    def __init__(self, torch, backend=None):
         self.torch = torch
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-        self.pg = None
+        self.backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        self.dev = torch.device("cuda", self.local_rank) if self.backend == "nccl" else torch.device("cpu")
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local_rank)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local_rank))
+            kw = {}
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+                kw["device_id"] = self.dev
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.dist = dist
 
     def barrier(self):
@@ -422,13 +430,24 @@ class DistCtx:
     def max(self, v):
         if self.world == 1:
             return v
-        t = self.torch.tensor([v], dtype=self.torch.float64, device="cuda")
+        t = self.torch.tensor([v], dtype=self.torch.float64, device=self.dev)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.world > 1:
             self.dist.destroy_process_group()
+
+
+def rank_seed(base, rank):
+    """Seed of a rank's independent batch: every rank draws its own inputs."""
+    return base + 1000 * rank
+
+
+def job_throughput(units_per_rank, world, max_ms):
+    """Whole-job rate: the units all ranks processed / the slowest rank's
+    time (ms), per second."""
+    return units_per_rank * world / (max_ms * 1e-3)
 
 
 def run_reference(args):
@@ -491,14 +510,14 @@ def main():
     peaks = load_peaks()
 
     # ---- decode (headline) ----
-    layer = Layer(torch, mfp8, W, seed=1 + 1000 * ctx.rank, weight_sets=3, Ms=DECODE_MS, device=device,
+    layer = Layer(torch, mfp8, W, seed=rank_seed(1, ctx.rank), weight_sets=3, Ms=DECODE_MS, device=device,
                   x_kind="normal")
     wbytes = layer.weight_bytes_per_step()
     with ClockSampler(ctx.local_rank) as clocks:
         ms = time_graph(torch, lambda h: layer.step(mfp8, h), args.steps, args.warmup, ctx)
     assert mfp8.device_status() == mfp8.OK
     step_ms = ms / args.steps
-    value = wbytes * ctx.world * args.steps / (ms * 1e-3) / 1e9
+    value = job_throughput(wbytes * args.steps, ctx.world, ms) / 1e9
 
     kt = kernel_times(torch, mfp8, layer, steps=max(5, min(args.steps, 20)), warmup=args.warmup)
     gemm_gbs = kt["gemm_bytes"] / (kt["gemm_us"] * 1e-6) / 1e9
@@ -513,14 +532,14 @@ def main():
     # same weights, outputs and arithmetic, fewer dependent launches.
     packed = None
     if not args.no_packed:
-        pk_layer = Layer(torch, mfp8, W, seed=1 + 1000 * ctx.rank, weight_sets=3, Ms=DECODE_MS, device=device,
+        pk_layer = Layer(torch, mfp8, W, seed=rank_seed(1, ctx.rank), weight_sets=3, Ms=DECODE_MS, device=device,
                          x_kind="normal", lins=W.PACKED_LAYER_LINEARS)
         assert pk_layer.weight_bytes_per_step() == wbytes
         pms = time_graph(torch, lambda h: pk_layer.step(mfp8, h), args.steps, args.warmup, ctx)
         assert mfp8.device_status() == mfp8.OK
         packed = {"workload": "the same decode step with q/k/v packed into qkv_proj (N=6144) and gate/up into "
                               "gate_up_proj (N=24576): 12 launches per step",
-                  "value": round(wbytes * ctx.world * args.steps / (pms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                  "value": round(job_throughput(wbytes * args.steps, ctx.world, pms) / 1e9, 1), "unit": "GB/s",
                   "ms_per_step": round(pms / args.steps, 5),
                   "frac_of_hbm": round(wbytes * args.steps / (pms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                   "launches_per_step": pk_layer.launches_per_step(mfp8)}
@@ -528,7 +547,7 @@ def main():
         torch.cuda.empty_cache()
 
     e2e_ms, h2d, d2h = e2e_time(torch, mfp8, layer, max(3, args.steps // 5), 3, ctx)
-    e2e_val = wbytes * ctx.world * max(3, args.steps // 5) / (e2e_ms * 1e-3) / 1e9
+    e2e_val = job_throughput(wbytes * max(3, args.steps // 5), ctx.world, e2e_ms) / 1e9
     wq = {"GB/s": round(layer.wq_bytes / (layer.wq_time_ms * 1e-3) / 1e9, 1),
           "bytes": layer.wq_bytes, "ms": round(layer.wq_time_ms, 3),
           "frac_of_hbm": round(layer.wq_bytes / (layer.wq_time_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
@@ -538,17 +557,17 @@ def main():
     # ---- prefill M = 2048 (the TFLOPS half of the metric) ----
     prefill = None
     if not args.no_prefill:
-        pl = Layer(torch, mfp8, W, seed=2 + 1000 * ctx.rank, weight_sets=1, Ms=(PREFILL_M,), device=device,
+        pl = Layer(torch, mfp8, W, seed=rank_seed(2, ctx.rank), weight_sets=1, Ms=(PREFILL_M,), device=device,
                    x_kind="rowscale")
         psteps = max(5, args.steps // 2)
         pms = time_graph(torch, lambda h: pl.step(mfp8, h), psteps, args.warmup, ctx)
-        tflops = pl.flops_per_step() * psteps / (pms * 1e-3) / 1e12
+        tflops = job_throughput(pl.flops_per_step() * psteps, ctx.world, pms) / 1e12
         pk = kernel_times(torch, mfp8, pl, steps=5, warmup=args.warmup)
         g_tf = pk["gemm_flops"] / (pk["gemm_us"] * 1e-6) / 1e12
         fp8_peak = 2.0 * peaks["bf16_tflops"]
         prefill = {"metric": "FP8-dynamic Linear TFLOPS (M=2048, 7 Linears, quantize included)",
                    "value": round(tflops, 1), "unit": "TFLOP/s", "ms_per_step": round(pms / psteps, 4),
-                   "frac_of_fp8_peak": round(tflops / fp8_peak, 4),
+                   "frac_of_fp8_peak": round(tflops / ctx.world / fp8_peak, 4),
                    "roofline": {"bound": "tensor", "achieved": round(g_tf, 1), "peak": round(fp8_peak, 1),
                                 "unit": "TFLOP/s", "frac": round(g_tf / fp8_peak, 4),
                                 # DRAM bytes per launch of the pair kernel, which runs 5 of
@@ -563,16 +582,17 @@ def main():
     # Long video-context prefill: gate/up/down at M = 16384 (seed 3).
     video = None
     if not args.no_prefill:
-        vl = Layer(torch, mfp8, W, seed=3 + 1000 * ctx.rank, weight_sets=1, Ms=(16384,), device=device,
+        vl = Layer(torch, mfp8, W, seed=rank_seed(3, ctx.rank), weight_sets=1, Ms=(16384,), device=device,
                    x_kind="rowscale", lins=W.MLP_LINEARS)
         vsteps = max(3, args.steps // 10)
         vms = time_graph(torch, lambda h: vl.step(mfp8, h), vsteps, args.warmup, ctx)
         assert mfp8.device_status() == mfp8.OK
         video = {"workload": "long video-context prefill: gate/up 4096->12288 and down 12288->4096 at M=16384, "
                              "X as the prefill workload, seed 3",
-                 "value": round(vl.flops_per_step() * vsteps / (vms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
-                 "ms_per_step": round(vms / vsteps, 4),
-                 "frac_of_fp8_peak": round(vl.flops_per_step() * vsteps / (vms * 1e-3) / 1e12 / (2.0 * peaks["bf16_tflops"]), 4)}
+                 "value": round(job_throughput(vl.flops_per_step() * vsteps, ctx.world, vms) / 1e12, 1),
+                 "unit": "TFLOP/s", "ms_per_step": round(vms / vsteps, 4),
+                 "frac_of_fp8_peak": round(vl.flops_per_step() * vsteps / (vms * 1e-3) / 1e12
+                                           / (2.0 * peaks["bf16_tflops"]), 4)}
         del vl
         torch.cuda.empty_cache()
 
