@@ -23,8 +23,11 @@
 // ranges of K blocks.  S is chosen so that the grid is about one CTA per
 // SM.  Per CTA:
 //   1. start the tile's weights of its K range streaming through a TMA ring
-//      (before waiting on the previous kernel when the weights are static),
-//      and ask L2 to prefetch the part that does not fit in the ring;
+//      (before waiting on the previous kernel when the weights are static);
+//      the MMA thread moves the first K blocks from the ring into TMEM
+//      (tcgen05.cp) as they land, so up to 7 more blocks than the ring
+//      holds are on chip before X exists, and L2 is asked to prefetch the
+//      rest;
 //   2. the four quantizer warps load this CTA's K slice of X (BF16) and take
 //      each token's absmax over the slice; the slice maxima go to every CTA
 //      of the cluster with st.async (a remote shared-memory store counted on
@@ -34,14 +37,16 @@
 //      mfp8_quantize_act) into shared memory in the 128-byte-swizzled
 //      K-major layout the MMA reads;
 //   4. one thread issues 4 MMAs per 128-byte K block into an fp32 TMEM
-//      accumulator D[128 channels][16 tokens];
+//      accumulator D[128 channels][16 tokens], with the weight operand read
+//      from TMEM for the parked blocks and from the ring for the others;
 //   5. with S > 1, each channel's partial row is pushed with st.async to
 //      the CTA of the cluster that owns the channel (rank r owns 128/S of
 //      them), which adds the S partials in rank order (deterministic),
 //      scales by s_a[m] * s_w[n] and stores BF16.  With S = 1 the epilogue
 //      stores directly.
-// Shared memory stays near 106 KB and TMEM at 32 columns, so two CTAs fit
-// on an SM: the kernel lets its dependent launch start at once
+// Shared memory stays near 109 KB and TMEM at most 256 columns (the
+// accumulator plus 7 parked K blocks of 32 columns), so two CTAs fit on an
+// SM: the kernel lets its dependent launch start at once
 // (programmatic dependent launch), and the next Linear's CTAs become
 // resident and stream their weights while this one finishes.
 //
@@ -76,6 +81,10 @@ constexpr int kMaxCodeBytes = 64 * 1024;
 constexpr int kMinStages = 2;
 constexpr int kRegItems = 16;             // 16-byte X vectors a quantizer thread keeps in registers
 constexpr int kMaxChunks = 16;            // code barriers: 64 or 128 vectors of every row each
+constexpr int kAccCols = 32;              // TMEM columns set aside for the accumulator (16 used)
+constexpr int kBlockCols = SUB / 4;       // TMEM columns of one weight K block (128 lanes x 128 bytes)
+constexpr int kMaxTmemBlocks = (256 - kAccCols) / kBlockCols;  // weight K blocks parked in TMEM: 7
+static_assert(SUB / MMA_K == 4 && MMA_K / 4 == 8, "a K block is four MMAs of 8 TMEM columns each");
 
 // Launch geometry, computed on the host (stream_geometry in mfp8.cu).
 struct Geometry {
@@ -83,7 +92,15 @@ struct Geometry {
     int mpad;        // code rows per K block in shared memory: 8 (M <= 8) or 16
     int code_bytes;  // (largest K range in blocks) * mpad * 128, rounded up to 1 KB
     int stages;      // weight ring depth
+    int tm_blocks;   // weight K blocks a CTA may park in TMEM (0 .. kMaxTmemBlocks)
 };
+
+// TMEM columns a CTA allocates: the accumulator, then tm_blocks weight
+// blocks, rounded up to a power of two.  Two CTAs per SM fit in the 512.
+__host__ __device__ constexpr uint32_t tmem_cols(int tm_blocks) {
+    const int need = kAccCols + (tm_blocks > 0 ? tm_blocks : 0) * kBlockCols;
+    return need <= 32 ? 32u : need <= 64 ? 64u : need <= 128 ? 128u : 256u;
+}
 
 // Shared memory, from a 1024-byte aligned base:
 //   [code store | weight ring]  kShared bytes (the ring starts at code_bytes)
@@ -98,8 +115,8 @@ struct Smem {
     static constexpr int SA_OFF = AMAX_OFF + kMaxM * 4;
     static constexpr int SW_OFF = SA_OFF + kMaxM * 4;
     static constexpr int BAR_OFF = SW_OFF + TILE * 4;
-    // wfull[8], wempty[8], chunk[16], xbar, tfull, rbar, drain
-    static constexpr int NUM_BARS = 2 * kMaxStages + kMaxChunks + 4;
+    // wfull[8], wempty[8], chunk[16], xbar, tfull, rbar, drain, tcopy, (pad)
+    static constexpr int NUM_BARS = 2 * kMaxStages + kMaxChunks + 6;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int USED = MISC_OFF + 16;
     static constexpr int BYTES = USED + 1024;  // alignment slack
@@ -156,6 +173,7 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
     const uint32_t tfull_bar = xbar + 8u;                              // accumulator complete
     const uint32_t rbar = xbar + 16u;                                  // all partials of my channels received
     const uint32_t drain_bar = xbar + 24u;
+    const uint32_t tcopy_bar = xbar + 32u;                             // weight blocks copied into TMEM
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Smem::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::MISC_OFF + 4);
     uint32_t* amax_all = reinterpret_cast<uint32_t*>(smem + Smem::AMAX_ALL_OFF);
@@ -193,6 +211,7 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         mbar_init(tfull_bar, 1);
         mbar_init(rbar, 1);
         mbar_init(drain_bar, 1);
+        mbar_init(tcopy_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
         // The remote bytes this CTA will receive: S slices of 16 maxima, and
@@ -205,7 +224,7 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         tma_prefetch_desc(&tmW);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), 32);
+        tmem_alloc(smem_u32(tmem_holder), tmem_cols(args.g.tm_blocks));
         tmem_relinquish();
     }
     tc_fence_before();
@@ -252,27 +271,96 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         if (lane == 0) {
             // ----------------------------------------------- MMA issuer --
             constexpr uint32_t idesc = idesc_e4m3_f32(TILE, MMA_N);
+            // K blocks 0 .. T-1 move from the ring into TMEM as soon as they
+            // land (before the dependency wait when the weights are static),
+            // which frees their slots for blocks STAGES .. STAGES+T-1: the
+            // CTA then holds T + STAGES blocks of its slice before X exists.
+            const int spare = nkb - STAGES;
+            const int T = spare <= 0 ? 0 : (spare < args.g.tm_blocks ? spare : args.g.tm_blocks);
+            const uint32_t tmem_w = tmem_base + uint32_t(kAccCols);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true, issued_any = false;
-            int chunks_seen = 0;
-            for (int i = 0; i < nkb && ok; ++i) {
+            for (int i = 0; i < T; ++i) {
                 if (!mbar_wait(wfull_bar(stage), phase, abort_flag)) { ok = false; break; }
-                for (const int need = (i * (SUB / 8)) / CV + 1; chunks_seen < need; ++chunks_seen)
-                    if (!mbar_wait(chunk_bar(chunks_seen), 0, abort_flag)) { ok = false; break; }
-                if (!ok) break;
                 tc_fence_after();
                 const uint32_t a0 = sW + uint32_t(stage * kWStageBytes);
-                const uint32_t b0 = sCode + uint32_t(i * MPAD * SUB);
 #pragma unroll
                 for (int kk = 0; kk < SUB / MMA_K; ++kk)
-                    mma_f8(tmem_base, sw128_kmajor_desc(a0 + kk * MMA_K), sw128_kmajor_desc(b0 + kk * MMA_K), idesc,
-                           (i | kk) != 0);
+                    tmem_cp_128x256b(tmem_w + uint32_t(i * kBlockCols + kk * (MMA_K / 4)),
+                                     sw128_kmajor_desc(a0 + kk * MMA_K));
                 issued_any = true;
-                // A commit holds up this thread for a few hundred cycles:
-                // release a ring slot only if the producer will refill it.
                 if (i + STAGES < nkb) mma_commit(wempty_bar(stage));
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (ok && T > 0) mma_commit(tcopy_bar);
+            // One thread issues every MMA, and at N = 16 its own instruction
+            // latency, not the tensor core, sets the pace: an mbarrier test
+            // that succeeds at once costs about 200 cycles and per-block
+            // bookkeeping as much again, against about 50 cycles per MMA.
+            // So the ring blocks already in flight are waited for here,
+            // while the quantizers work; the loop then waits once per code
+            // chunk (BPC K blocks) and once per block only for blocks still
+            // streaming in, and runs straight 4-MMA groups in between, with
+            // descriptors advanced by addition.
+            const int pre = nkb < T + STAGES ? nkb : T + STAGES;
+            {
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = T; i < pre && ok; ++i) {
+                    if (!mbar_wait(wfull_bar(st), ph, abort_flag)) ok = false;
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+            const uint64_t dA0 = sw128_kmajor_desc(sW);
+            const uint64_t dB0 = sw128_kmajor_desc(sCode);
+            constexpr uint64_t kStep = MMA_K >> 4;        // descriptor units (16 bytes) per 32-byte K step
+            constexpr uint64_t kStageStep = kWStageBytes >> 4;
+            const uint64_t kBlockStepB = uint64_t(MPAD * SUB) >> 4;
+            const int BPC = CV / (SUB / 8);                // K blocks per code chunk: 4 or 8
+            const int refill = nkb - STAGES;
+            // The four 32-byte K steps of one block, weights from the ring.
+            auto mma4 = [&](uint64_t dA, uint64_t dB, uint32_t accf) {
+                mma_f8(tmem_base, dA, dB, idesc, accf);
+                mma_f8(tmem_base, dA + kStep, dB + kStep, idesc, 1u);
+                mma_f8(tmem_base, dA + 2 * kStep, dB + 2 * kStep, idesc, 1u);
+                mma_f8(tmem_base, dA + 3 * kStep, dB + 3 * kStep, idesc, 1u);
+            };
+            int i = 0;
+            for (int c = 0; i < nkb && ok; ++c) {
+                if (!mbar_wait(chunk_bar(c), 0, abort_flag)) { ok = false; break; }
+                if (c == 0 && T > 0 && !mbar_wait(tcopy_bar, 0, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                issued_any = true;
+                const int iend = nkb < i + BPC ? nkb : i + BPC;
+                uint64_t dB = dB0 + uint64_t(i) * kBlockStepB;
+                for (; i < iend && i < T; ++i, dB += kBlockStepB) {  // weights parked in TMEM
+                    const uint32_t aT = tmem_w + uint32_t(i * kBlockCols);
+                    mma_f8_tmem_a(tmem_base, aT, dB, idesc, i != 0);
+                    mma_f8_tmem_a(tmem_base, aT + 8u, dB + kStep, idesc, 1u);
+                    mma_f8_tmem_a(tmem_base, aT + 16u, dB + 2 * kStep, idesc, 1u);
+                    mma_f8_tmem_a(tmem_base, aT + 24u, dB + 3 * kStep, idesc, 1u);
+                }
+                // Weights in the ring.  A block below `refill` releases its
+                // slot for the producer; the blocks from `pre` on are still
+                // streaming in and are waited for one by one.
+                for (; i < iend && i < pre && i < refill; ++i, dB += kBlockStepB) {
+                    const uint64_t dA = dA0 + uint64_t(stage) * kStageStep;
+                    mma4(dA, dB, i != 0);
+                    mma_commit(wempty_bar(stage));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                for (; i < iend && i < pre; ++i, dB += kBlockStepB) {
+                    mma4(dA0 + uint64_t(stage) * kStageStep, dB, i != 0);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                for (; i < iend; ++i, dB += kBlockStepB) {
+                    if (!mbar_wait(wfull_bar(stage), phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    mma4(dA0 + uint64_t(stage) * kStageStep, dB, i != 0);
+                    if (i < refill) mma_commit(wempty_bar(stage));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
             }
             if (ok) {
                 mma_commit(tfull_bar);
@@ -477,7 +565,7 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 32);
+        tmem_dealloc(tmem_base, tmem_cols(args.g.tm_blocks));
     }
 }
 

@@ -513,6 +513,9 @@ bool stream_geometry(int64_t M, int64_t N, int64_t K, int sm_count, stream::Geom
     g->code_bytes = int(code_bytes(S));
     const int st = (stream::kShared - g->code_bytes) / stream::kWStageBytes;
     g->stages = st > stream::kMaxStages ? stream::kMaxStages : st;
+    // K blocks beyond the ring wait in TMEM (up to 7 per CTA).
+    const int64_t spare = (kb + S - 1) / S - g->stages;
+    g->tm_blocks = spare <= 0 ? 0 : int(spare < stream::kMaxTmemBlocks ? spare : stream::kMaxTmemBlocks);
     return g->stages >= stream::kMinStages;
 }
 
