@@ -144,6 +144,11 @@ __device__ __forceinline__ void prefetch_tile_l2(const CUtensorMap* map, int32_t
                  ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
 }
 
+// Position of 16-byte token group g of a partial row in the receive slot
+// of channel cl: g ^ recv_swz(cl).  Eight consecutive channels then cover
+// all 32 banks when one group is read across them.
+__device__ __forceinline__ int recv_swz(int cl) { return (cl >> 1) & 3; }
+
 __device__ __forceinline__ uint4 ldg_nc(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -526,16 +531,21 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
                             __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa_sm[mm] * sw);
             }
         } else {
-            // Partial row of channel c to its owner: slot [rank][c % CPR].
+            // Partial row of channel c to its owner: slot [rank][c % CPR],
+            // 16 token columns in four 16-byte groups, group g stored at
+            // position g ^ swz(c % CPR) so that the owner's reads of one
+            // group across consecutive channels hit distinct banks.
             if (have_acc) {
                 const int owner = c / CPR;
-                const uint32_t local = sbase + uint32_t(Smem::RECV_OFF + ((rank * CPR + c % CPR) * MMA_N) * 4);
+                const int cl = c % CPR;
+                const uint32_t local = sbase + uint32_t(Smem::RECV_OFF + ((rank * CPR + cl) * MMA_N) * 4);
                 const uint32_t dst = mapa_shared(local, uint32_t(owner));
                 const uint32_t bar = mapa_shared(rbar, uint32_t(owner));
 #pragma unroll
-                for (int i = 0; i < MMA_N; i += 4)
-                    if (i < M)  // the token columns that exist, in groups of 4
-                        st_async_v4(dst + 4u * i, make_uint4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]), bar);
+                for (int g = 0; g < MMA_N / 4; ++g)
+                    if (4 * g < M)  // the token columns that exist, in groups of 4
+                        st_async_v4(dst + 16u * uint32_t(g ^ recv_swz(cl)),
+                                    make_uint4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]), bar);
             }
             // Sum the S partials of the channels this rank owns, in rank order.
             const bool have_partials = mbar_wait(rbar, 0, abort_flag);
@@ -544,13 +554,31 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
                 mbar_wait(rbar, 0, &no_abort, 20000000ull);
             }
             if (have_partials) {
-                for (int e = t; e < CPR * M; e += kQuantThreads) {
-                    const int cl = e % CPR, mm = e / CPR;
+                // One thread per (channel, group of 4 tokens): a 16-byte read
+                // per rank, consecutive channels across the warp, so the Y
+                // stores of each token row are contiguous.
+                const int G = (M + 3) / 4;
+                for (int e = t; e < CPR * G; e += kQuantThreads) {
+                    const int cl = e % CPR, g = e / CPR;
                     const int n = n0 + rank * CPR + cl;
-                    float sum = 0.f;
-                    for (int i = 0; i < S; ++i) sum += recv[(i * CPR + cl) * MMA_N + mm];
-                    if (n < N)
-                        args.Y[int64_t(mm) * N + n] = __float2bfloat16_rn(sum * sa_sm[mm] * sw_sm[rank * CPR + cl]);
+                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int i = 0; i < S; ++i) {
+                        const float4 p = *reinterpret_cast<const float4*>(recv + (i * CPR + cl) * MMA_N +
+                                                                          4 * (g ^ recv_swz(cl)));
+                        sum.x += p.x;
+                        sum.y += p.y;
+                        sum.z += p.z;
+                        sum.w += p.w;
+                    }
+                    if (n < N) {
+                        const float sw = sw_sm[rank * CPR + cl];
+                        const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (4 * g + j < M)
+                                args.Y[int64_t(4 * g + j) * N + n] =
+                                    __float2bfloat16_rn(v[j] * sa_sm[4 * g + j] * sw);
+                    }
                 }
             }
         }
