@@ -149,6 +149,10 @@ __device__ __forceinline__ void prefetch_tile_l2(const CUtensorMap* map, int32_t
 // all 32 banks when one group is read across them.
 __device__ __forceinline__ int recv_swz(int cl) { return (cl >> 1) & 3; }
 
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint2 v) {
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y));
+}
+
 __device__ __forceinline__ uint4 ldg_nc(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -455,12 +459,11 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
             // 16-byte chunks swizzled by (m & 7).  Vectors past K (a ragged
             // last block) are zero codes.  Rows whose scale is below
             // kFmaMinScale take the divide, one vector at a time.
-            uint8_t* code_sm = smem;
             const bool write_out = args.x8_out != nullptr && tile == 0;
+            const uint32_t code_row = sCode + uint32_t(m * SUB);
             auto put = [&](int v, uint2 code) {
                 const int blk = v >> 4, c16 = (v & 15) >> 1;
-                *reinterpret_cast<uint2*>(code_sm + (blk * MPAD + m) * SUB + ((c16 ^ (m & 7)) << 4) + ((v & 1) << 3)) =
-                    code;
+                st_shared_v2(code_row + uint32_t(blk * MPAD * SUB + ((c16 ^ (m & 7)) << 4) + ((v & 1) << 3)), code);
                 if (write_out && v < nv)
                     *reinterpret_cast<uint2*>(args.x8_out + int64_t(m) * K + k0 + int64_t(v) * 8) = code;
             };

@@ -80,14 +80,15 @@ __device__ __forceinline__ uint2 quantize8_div(uint4 v, float s) {
     return q;
 }
 
-// fl32(a / s) for a >= 0 without a divide: r = fl32(1 / s) (correctly
-// rounded), q0 = fl32(a * r) is within one unit in the last place of a / s,
-// the residual a - q0 * s is exact in one fused multiply-add, and one more
-// fused multiply-add q0 + (a - q0 s) * r rounds to the correctly rounded
-// quotient (Markstein's theorem on division by reciprocal with a corrected
-// quotient).  Working on |x| keeps the sign of zero out of the arithmetic;
-// the code's sign bit is taken from x.  Checked against the IEEE divide on
-// every pair of bf16 values with |x| <= absmax (mfp8_debug_quantize_check).
+// fl32(a / s) without a divide: r = fl32(1 / s) (correctly rounded),
+// q0 = fl32(a * r) is within one unit in the last place of a / s, the
+// residual a - q0 * s is exact in one fused multiply-add, and one more fused
+// multiply-add q0 + (a - q0 s) * r rounds to the correctly rounded quotient
+// (Markstein's theorem on division by reciprocal with a corrected quotient).
+// Every step rounds to nearest, which is odd-symmetric, so -a gives exactly
+// the negated result; the one exception is a = -0, for which the residual
+// step returns +0.  Checked against the IEEE divide on every pair of bf16
+// values with |x| <= absmax, both signs (mfp8_debug_quantize_check).
 __device__ __forceinline__ float div_rn_by_recip(float a, float s, float r) {
     const float q0 = __fmul_rn(a, r);
     const float e = __fmaf_rn(-q0, s, a);
@@ -96,11 +97,12 @@ __device__ __forceinline__ float div_rn_by_recip(float a, float s, float r) {
 
 // Two bf16 values (one 32-bit word) -> two e4m3 codes (16 bits, low value in
 // the low byte).
+// The quotients carry x's sign except for x = -0 (see div_rn_by_recip), so
+// the sign bits of x are OR-ed into the codes: a no-op for every other x.
 __device__ __forceinline__ uint32_t quantize2_fma(uint32_t w, float s, float r) {
-    const float lo = div_rn_by_recip(__uint_as_float((w & 0x7fffu) << 16), s, r);
-    const float hi = div_rn_by_recip(__uint_as_float(w & 0x7fff0000u), s, r);
-    const uint32_t sign = ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
-    return e4m3x2(lo, hi) | sign;
+    const float lo = div_rn_by_recip(__uint_as_float(w << 16), s, r);
+    const float hi = div_rn_by_recip(__uint_as_float(w & 0xffff0000u), s, r);
+    return e4m3x2(lo, hi) | (__byte_perm(w, 0u, 0x4431u) & 0x8080u);  // bits 15, 31 of w -> 7, 15
 }
 
 // 8 bf16 values -> 8 e4m3 codes, same codes as quantize8_div.  The
