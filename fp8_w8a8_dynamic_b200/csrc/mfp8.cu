@@ -500,8 +500,16 @@ bool stream_geometry(int64_t M, int64_t N, int64_t K, int sm_count, stream::Geom
     const int64_t tiles = (N + stream::TILE - 1) / stream::TILE;
     const int64_t kb = (K + stream::SUB - 1) / stream::SUB;
     const int mpad = M <= 8 ? 8 : 16;
+    // The K split doubles while the grid stays within 1.5 CTAs per SM, and
+    // on up to 2 per SM while every CTA keeps at least 8 K blocks (long-K
+    // Linears such as down_proj, where more CTAs in flight stream faster).
     int S = 1;
-    while (S < stream::kMaxCluster && tiles * S * 2 <= sm_count * 3 / 2 && S * 2 <= kb) S *= 2;
+    auto grow = [&](int s) {
+        if (s >= stream::kMaxCluster || s * 2 > kb) return false;
+        const int64_t ctas = tiles * s * 2;
+        return ctas <= sm_count * 3 / 2 || (ctas <= int64_t(sm_count) * 2 && kb / (s * 2) >= 8);
+    };
+    while (grow(S)) S *= 2;
     auto code_bytes = [&](int s_) {
         const int64_t kbs = (kb + s_ - 1) / s_;
         return (kbs * mpad * stream::SUB + 1023) / 1024 * 1024;
