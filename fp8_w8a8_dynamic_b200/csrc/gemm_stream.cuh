@@ -28,7 +28,7 @@
 //      (tcgen05.cp) as they land, so up to 7 more blocks than the ring
 //      holds are on chip before X exists, and L2 is asked to prefetch the
 //      rest;
-//   2. the four quantizer warps load this CTA's K slice of X (BF16) and take
+//   2. the quantizer warps load this CTA's K slice of X (BF16) and take
 //      each token's absmax over the slice; the slice maxima go to every CTA
 //      of the cluster with st.async (a remote shared-memory store counted on
 //      the receiver's mbarrier), so every CTA ends up with the row absmax
@@ -50,9 +50,9 @@
 // (programmatic dependent launch), and the next Linear's CTAs become
 // resident and stream their weights while this one finishes.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA
-// issuer, warps 2-5 quantizers and epilogue (warp w reads TMEM lanes
-// 32 (w % 4) .. +31).  Every wait is bounded; on a timeout the kernel records
+// Warp roles (64 + 32 QW threads): warp 0 TMA producer, warp 1 TMEM owner
+// and MMA issuer, warps 2 .. QW + 1 quantizers and epilogue (warp w reads
+// TMEM lanes 32 (w % 4) .. +31 and 64 / QW token columns).  Every wait is bounded; on a timeout the kernel records
 // MFP8_ERR_TIMEOUT, drains what it has in flight and frees its TMEM.  A CTA
 // leaves only after every remote store addressed to it has landed.
 #pragma once
@@ -66,8 +66,17 @@
 namespace mfp8 {
 namespace stream {
 
-constexpr int kThreads = 192;
-constexpr int kQuantThreads = 128;        // warps 2-5
+// The kernel is instantiated for 4 or 8 quantizer/epilogue warps (QW): 8
+// hide each other's latency when each CTA has many tokens to quantize
+// (M > 8), 4 cost less in set-up and barriers below that.
+template <int QW>
+struct Warps {
+    static constexpr int kThreads = 64 + 32 * QW;      // + producer and MMA warps
+    static constexpr int kQuantThreads = 32 * QW;
+    static constexpr int kRegItems = 64 / QW;          // X vectors a quantizer thread keeps in registers
+    static constexpr int kCols = 64 / QW;              // token columns per epilogue warp
+    static_assert(QW == 4 || QW == 8, "4 or 8 quantizer warps");
+};
 constexpr int TILE = 128;                 // output channels per cluster (MMA M)
 constexpr int MMA_N = 16;                 // token columns of the MMA (first M real)
 constexpr int MMA_K = 32;
@@ -79,7 +88,6 @@ constexpr int kWStageBytes = TILE * SUB;  // one K block of the tile: 16 KB
 constexpr int kShared = 96 * 1024;        // code store + weight ring
 constexpr int kMaxCodeBytes = 64 * 1024;
 constexpr int kMinStages = 2;
-constexpr int kRegItems = 16;             // 16-byte X vectors a quantizer thread keeps in registers
 constexpr int kMaxChunks = 16;            // code barriers: 64 or 128 vectors of every row each
 constexpr int kAccCols = 32;              // TMEM columns set aside for the accumulator (16 used)
 constexpr int kBlockCols = SUB / 4;       // TMEM columns of one weight K block (128 lanes x 128 bytes)
@@ -165,8 +173,12 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint4 v, uint3
                  ::"r"(remote_addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <int QW>
+__global__ void __launch_bounds__(Warps<QW>::kThreads, 2)
 gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
+    constexpr int kQuantThreads = Warps<QW>::kQuantThreads;
+    constexpr int kRegItems = Warps<QW>::kRegItems;
+    constexpr int kCols = Warps<QW>::kCols;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -216,7 +228,8 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
             mbar_init(wempty_bar(s), 1);
         }
         mbar_init(xbar, 1);
-        for (int c = 0; c < kMaxChunks; ++c) mbar_init(chunk_bar(c), 4);  // one arrival per quantizer warp
+        for (int c = 0; c < kMaxChunks; ++c)
+            mbar_init(chunk_bar(c), kQuantThreads / 32);  // one arrival per quantizer warp
         mbar_init(tfull_bar, 1);
         mbar_init(rbar, 1);
         mbar_init(drain_bar, 1);
@@ -381,11 +394,12 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         }
     } else {
         // ------------------------------------------ quantizers, epilogue --
-        const int t = int(threadIdx.x) - 64;  // 0..127
-        const int q = int(warp & 3u);         // TMEM lane quarter of this warp
+        const int t = int(threadIdx.x) - 64;     // 0 .. kQuantThreads - 1
+        const int q = int(warp & 3u);            // TMEM lane quarter of this warp
+        const int half = (int(warp) - 2) >> 2;   // and its token columns: kCols * half .. + kCols - 1
         // s_w of the tile (static weights: no need to wait).
         if (!args.weights_static) grid_dependency_wait();
-        sw_sm[t] = (n0 + t < N) ? __ldg(args.s_w + n0 + t) : 0.f;  // 128 threads, 128 channels
+        if (t < TILE) sw_sm[t] = (n0 + t < N) ? __ldg(args.s_w + n0 + t) : 0.f;
         if (t < kMaxM) amax_loc[t] = 0u;
         // Ask L2 for this CTA's slice of X (M rows of (k1 - k0) * 2 bytes)
         // while the previous kernel finishes.  A prefetch returns nothing
@@ -399,7 +413,7 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         // X may be the previous kernel's output.
         grid_dependency_wait();
 
-        // Rows are spread over the 128 threads: TPR threads per row (a power
+        // Rows are spread over the kQuantThreads threads: TPR threads per row (a power
         // of two), thread t takes row t / TPR and the vectors j, j + TPR, ...
         // of the slice (j = t % TPR).  Item u of every thread lies in chunk
         // u / IPC (CV = IPC * TPR vectors of the row per chunk).
@@ -515,40 +529,48 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         }
         named_bar_sync(1, kQuantThreads);  // sa_sm complete
 
-        // Epilogue: this warp's 32 channels, 16 token columns each.
+        // Epilogue: this warp's 32 channels, kCols token columns each.
         const int c = q * 32 + int(lane);  // channel within the tile
-        uint32_t acc[MMA_N];
+        const int m0 = kCols * half;       // first token column of this warp
+        uint32_t acc[kCols];
         const bool have_acc = have_scale && mbar_wait(tfull_bar, 0, abort_flag);
-        if (have_acc) {
+        if (have_acc && m0 < M) {
             tc_fence_after();
-            tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16), acc);
+            const uint32_t ta = tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(m0);
+            if constexpr (kCols == 16)
+                tmem_ld_32x32b_x16(ta, acc);
+            else
+                tmem_ld_32x32b_x8(ta, acc);
             tmem_wait_ld();
         }
         if (S == 1) {
-            if (have_acc && n0 + c < N) {
+            if (have_acc && m0 < M && n0 + c < N) {
                 const float sw = sw_sm[c];
 #pragma unroll
-                for (int mm = 0; mm < MMA_N; ++mm)
-                    if (mm < M)
-                        args.Y[int64_t(mm) * N + n0 + c] =
-                            __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa_sm[mm] * sw);
+                for (int mm = 0; mm < kCols; ++mm)
+                    if (m0 + mm < M)
+                        args.Y[int64_t(m0 + mm) * N + n0 + c] =
+                            __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa_sm[m0 + mm] * sw);
             }
         } else {
             // Partial row of channel c to its owner: slot [rank][c % CPR],
             // 16 token columns in four 16-byte groups, group g stored at
             // position g ^ swz(c % CPR) so that the owner's reads of one
-            // group across consecutive channels hit distinct banks.
-            if (have_acc) {
+            // group across consecutive channels hit distinct banks.  This
+            // warp sends the groups of its kCols token columns.
+            if (have_acc && m0 < M) {
                 const int owner = c / CPR;
                 const int cl = c % CPR;
                 const uint32_t local = sbase + uint32_t(Smem::RECV_OFF + ((rank * CPR + cl) * MMA_N) * 4);
                 const uint32_t dst = mapa_shared(local, uint32_t(owner));
                 const uint32_t bar = mapa_shared(rbar, uint32_t(owner));
 #pragma unroll
-                for (int g = 0; g < MMA_N / 4; ++g)
+                for (int h = 0; h < kCols / 4; ++h) {
+                    const int g = m0 / 4 + h;
                     if (4 * g < M)  // the token columns that exist, in groups of 4
                         st_async_v4(dst + 16u * uint32_t(g ^ recv_swz(cl)),
-                                    make_uint4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]), bar);
+                                    make_uint4(acc[4 * h], acc[4 * h + 1], acc[4 * h + 2], acc[4 * h + 3]), bar);
+                }
             }
             // Sum the S partials of the channels this rank owns, in rank order.
             const bool have_partials = mbar_wait(rbar, 0, abort_flag);

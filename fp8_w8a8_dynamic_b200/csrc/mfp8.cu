@@ -534,9 +534,11 @@ mfp8_status launch_stream(const void* X, int64_t M, int64_t K, const void* W8, c
         return MFP8_ERR_UNSUPPORTED_SHAPE;
     stream::Geometry g;
     if (!stream_geometry(M, N, K, info.sm_count, &g)) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    auto kern = stream::gemm_stream_kernel;
-    static bool attr_done[kMaxDevices] = {};
-    mfp8_status st = set_smem(kern, stream::Smem::BYTES, dev, attr_done);
+    // Eight quantizer warps pay off once a CTA has more than 8 token rows.
+    const bool wide = M > 8;
+    auto kern = wide ? stream::gemm_stream_kernel<8> : stream::gemm_stream_kernel<4>;
+    static bool attr_done4[kMaxDevices] = {}, attr_done8[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, stream::Smem::BYTES, dev, wide ? attr_done8 : attr_done4);
     if (st != MFP8_OK) return st;
     const int64_t tiles = (N + stream::TILE - 1) / stream::TILE;
     const int64_t grid = tiles * g.S;
@@ -558,7 +560,7 @@ mfp8_status launch_stream(const void* X, int64_t M, int64_t K, const void* W8, c
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(grid));
-    cfg.blockDim = dim3(stream::kThreads);
+    cfg.blockDim = dim3(unsigned(wide ? stream::Warps<8>::kThreads : stream::Warps<4>::kThreads));
     cfg.dynamicSmemBytes = stream::Smem::BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
