@@ -1,0 +1,356 @@
+// gemm_cluster.cuh — the FP8 GEMM for small and middle M (up to 128 token
+// rows) on activation codes already quantized (the quantize pass of
+// mfp8_linear, or the caller's codes in mfp8_gemm):
+//
+//   Y[m, n] = bf16( (sum_k dec(X8[m,k]) * dec(W8[n,k])) * s_a[m] * s_w[n] )
+//
+// Source of the rule: "MOSS-VL quantization README", FP8-Dynamic recipe
+// (float8_e4m3fn weights with one static scale per output channel, FP8
+// per-token dynamic activations).
+//
+// At these sizes the Linear still streams N*K weight bytes and little else,
+// and a tcgen05.mma costs about the same up to N = 64 however few columns it
+// has.  So the weights are the MMA's 128-row A operand (4 KB per
+// instruction) and the tokens its N = MP columns (M rounded up to 16): the
+// whole batch in one accumulator of MP TMEM columns.  The layout is the one
+// of the decode kernel (gemm_stream.cuh) with the codes loaded by TMA:
+//   - a cluster of S CTAs (S in 1, 2, 4, 8) owns one tile of 128 output
+//     channels and splits K; each CTA streams its weight K blocks and the
+//     matching code blocks (MP rows x 128 bytes) through one TMA ring, the
+//     weights before the dependency wait when they are static;
+//   - one thread issues 4 MMAs per K block;
+//   - with S > 1, once every CTA of the cluster has its accumulator (a
+//     cluster barrier), each channel's partial row goes with st.async to the
+//     CTA that owns the channel, into that CTA's ring (free by then), and the
+//     owner adds the S partials in rank order (deterministic), scales and
+//     stores BF16.  With S = 1 the epilogue stores directly.
+// About 98 KB of shared memory and at most 128 TMEM columns, so two CTAs
+// fit on an SM and the next kernel's CTAs can start alongside.
+//
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA
+// issuer, warps 2-5 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31,
+// one output channel per thread).  Every wait is bounded; on a timeout the
+// kernel records MFP8_ERR_TIMEOUT, drains what it has in flight and frees
+// its TMEM.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace mfp8 {
+namespace cluster {
+
+constexpr int kThreads = 192;
+constexpr int TILE = 128;                   // output channels per cluster (MMA M)
+constexpr int SUB = 128;                    // K bytes per block: swizzle atom, TMA box width
+constexpr int MMA_K = 32;
+constexpr int kMaxM = 128;                  // token rows (MMA N up to 128)
+constexpr int kMaxCluster = 8;
+constexpr int kMaxStages = 8;
+constexpr int kWBlockBytes = TILE * SUB;    // one weight K block of the tile: 16 KB
+constexpr int kRingBytes = 96 * 1024;       // weight + code ring; later the partial-row receive area
+constexpr int kMinStages = 2;
+static_assert(SUB / MMA_K == 4, "a K block is four MMAs");
+
+// Launch geometry, computed on the host (cluster_geometry in mfp8.cu).
+struct Geometry {
+    int S;       // CTAs per cluster (K split)
+    int mp;      // token columns of the MMA: M rounded up to 16
+    int stages;  // ring depth; a stage is a weight block and a code block
+};
+
+__host__ __device__ constexpr int stage_bytes(int mp) { return kWBlockBytes + mp * SUB; }
+
+__host__ __device__ constexpr uint32_t tmem_cols(int mp) { return mp <= 32 ? 32u : mp <= 64 ? 64u : 128u; }
+
+// Shared memory, from a 1024-byte aligned base:
+//   [ring] kRingBytes: stage s at s * stage_bytes(mp) (weights, then codes);
+//          with S > 1 it later receives the partial rows this CTA owns,
+//          [S][128/S][mp] fp32 (at most 64 KB)
+//   [sa] [128] f32, [sw] [128] f32, barriers, TMEM base and abort flag
+struct Smem {
+    static constexpr int SA_OFF = kRingBytes;
+    static constexpr int SW_OFF = SA_OFF + kMaxM * 4;
+    static constexpr int BAR_OFF = SW_OFF + TILE * 4;
+    // full[8], empty[8], tfull, rbar, drain, (pad)
+    static constexpr int NUM_BARS = 2 * kMaxStages + 4;
+    static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+    static constexpr int USED = MISC_OFF + 16;
+    static constexpr int BYTES = USED + 1024;  // alignment slack
+    static_assert(TILE * kMaxM * 4 <= kRingBytes, "partial rows fit in the ring");
+    static_assert(kMinStages * stage_bytes(kMaxM) <= kRingBytes, "ring room");
+};
+
+struct Args {
+    const float* s_a;  // [M]
+    const float* s_w;  // [N]
+    __nv_bfloat16* Y;  // [M, N]
+    int M, N, K;
+    int weights_static;
+    Geometry g;
+};
+
+// Position of 16-byte token group g of a partial row in the receive slot of
+// channel cl: g ^ swz(cl), so that the owner's 16-byte reads of one group
+// across consecutive channels hit distinct banks.  A slot has mp / 4 groups
+// (a multiple of 4); the XOR stays inside an aligned run of 8 groups when
+// mp is a multiple of 32, of 4 otherwise.
+__device__ __forceinline__ int recv_swz(int cl, int mp) { return (mp & 31) == 0 ? (cl & 7) : ((cl >> 1) & 3); }
+
+__global__ void __launch_bounds__(kThreads, 2)
+gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    const Args args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int M = args.M, N = args.N, K = args.K;
+    const int S = args.g.S, MP = args.g.mp, STAGES = args.g.stages;
+    const int SB = stage_bytes(MP);
+    const uint32_t bar0 = sbase + Smem::BAR_OFF;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (kMaxStages + s); };
+    const uint32_t tfull_bar = bar0 + 8u * (2 * kMaxStages);  // accumulator complete
+    const uint32_t rbar = tfull_bar + 8u;                     // all partials of my channels received
+    const uint32_t drain_bar = tfull_bar + 16u;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Smem::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::MISC_OFF + 4);
+    float* sa_sm = reinterpret_cast<float*>(smem + Smem::SA_OFF);
+    float* sw_sm = reinterpret_cast<float*>(smem + Smem::SW_OFF);
+    const float* recv = reinterpret_cast<const float*>(smem);
+
+    const uint32_t warp = warp_id_sync();
+    const uint32_t lane = lane_id();
+    const int rank = S > 1 ? int(cluster_ctarank()) : 0;
+    const int tile = int(blockIdx.x) / S;
+    const int n0 = tile * TILE;
+    const int KB = (K + SUB - 1) / SUB;
+    const int kb0 = int((int64_t(KB) * rank) / S);
+    const int kb1 = int((int64_t(KB) * (rank + 1)) / S);
+    const int nkb = kb1 - kb0;  // >= 1 (the host keeps S <= KB)
+    const int CPR = TILE / S;   // channels each rank owns in the reduction
+    const uint32_t tcols = tmem_cols(MP);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kMaxStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(tfull_bar, 1);
+        mbar_init(rbar, 1);
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        // (S > 1) the S partial rows of each of the 128/S channels it owns
+        if (S > 1) mbar_arrive_expect_tx(rbar, uint32_t(TILE * MP * 4));
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    if (S > 1) {
+        // Every CTA's barriers are initialised before any remote store.
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    } else {
+        __syncthreads();
+    }
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    // The next kernel on the stream may start launching now: before its own
+    // dependency wait it only sets itself up and fetches static weights.
+    grid_launch_dependents();
+
+    bool have_acc = false;
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------- TMA producer --
+            // Weight blocks may go before the dependency wait (static
+            // weights); code blocks only after it: the codes come from the
+            // quantize pass just before this kernel.
+            const uint64_t policy = l2_policy_evict_first();
+            const int first = nkb < STAGES ? nkb : STAGES;
+            bool waited = false;
+            if (!args.weights_static) {
+                grid_dependency_wait();
+                waited = true;
+            }
+            for (int e = 0; e < first; ++e) {
+                const uint32_t st = sbase + uint32_t(e * SB);
+                mbar_arrive_expect_tx(full_bar(e), uint32_t(SB));
+                tma_load_2d_hint(st, &tmW, full_bar(e), (kb0 + e) * SUB, n0, policy);
+            }
+            for (int e = first; e < nkb; ++e) prefetch_tile_l2(&tmW, (kb0 + e) * SUB, n0);
+            if (!waited) grid_dependency_wait();
+            for (int e = 0; e < first; ++e)
+                tma_load_2d(sbase + uint32_t(e * SB + kWBlockBytes), &tmX, full_bar(e), (kb0 + e) * SUB, 0);
+            int stage = first == STAGES ? 0 : first;
+            uint32_t phase = first == STAGES ? 1u : 0u;
+            uint32_t issued_mask = (1u << first) - 1u, issued_parity = 0;
+            for (int e = first; e < nkb; ++e) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) break;
+                const uint32_t st = sbase + uint32_t(stage * SB);
+                mbar_arrive_expect_tx(full_bar(stage), uint32_t(SB));
+                tma_load_2d_hint(st, &tmW, full_bar(stage), (kb0 + e) * SUB, n0, policy);
+                tma_load_2d(st + uint32_t(kWBlockBytes), &tmX, full_bar(stage), (kb0 + e) * SUB, 0);
+                issued_mask |= 1u << stage;
+                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (*abort_flag) {
+                volatile int no_abort = 0;
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued_mask & (1u << s))
+                        mbar_wait(full_bar(s), (issued_parity >> s) & 1u, &no_abort, 10000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ----------------------------------------------- MMA issuer --
+            // One wait per K block and four straight MMAs: at these N the
+            // issuing thread's own latency sets the pace.
+            const uint32_t idesc = idesc_e4m3_f32(TILE, uint32_t(MP));
+            constexpr uint64_t kStep = MMA_K >> 4;  // descriptor units (16 bytes) per 32-byte K step
+            const uint64_t d0 = sw128_kmajor_desc(sbase);
+            const uint64_t dX = uint64_t(kWBlockBytes) >> 4;
+            const uint64_t dS = uint64_t(SB) >> 4;
+            const int refill = nkb - STAGES;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, issued_any = false;
+            for (int e = 0; e < nkb; ++e) {
+                if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+                if (e == 0) tc_fence_after();
+                issued_any = true;
+                const uint64_t dA = d0 + uint64_t(stage) * dS;
+                const uint64_t dB = dA + dX;
+                mma_f8(tmem_base, dA, dB, idesc, e != 0);
+                mma_f8(tmem_base, dA + kStep, dB + kStep, idesc, 1u);
+                mma_f8(tmem_base, dA + 2 * kStep, dB + 2 * kStep, idesc, 1u);
+                mma_f8(tmem_base, dA + 3 * kStep, dB + 3 * kStep, idesc, 1u);
+                if (e < refill) mma_commit(empty_bar(stage));  // the producer refills this slot
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (ok) {
+                mma_commit(tfull_bar);
+            } else if (issued_any) {
+                volatile int no_abort = 0;
+                mma_commit(drain_bar);
+                mbar_wait(drain_bar, 0, &no_abort, 10000000ull);
+            }
+        }
+    } else {
+        // -------------------------------------------- epilogue, part 1 --
+        const int t = int(threadIdx.x) - 64;  // 0..127
+        sw_sm[t] = (n0 + t < N) ? __ldg(args.s_w + n0 + t) : 0.f;
+        grid_dependency_wait();  // s_a comes from the quantize pass
+        sa_sm[t] = t < M ? __ldg(args.s_a + t) : 0.f;
+        have_acc = mbar_wait(tfull_bar, 0, abort_flag);
+        named_bar_sync(1, 128);  // sa_sm, sw_sm complete
+    }
+
+    // With S > 1 every CTA of the cluster has its accumulator before any
+    // partial row lands in a ring: the rings are free from here on.
+    __syncwarp();
+    if (S > 1) {
+        tc_fence_before();
+        cluster_arrive_release();
+        cluster_wait_acquire();
+        tc_fence_after();
+    }
+
+    if (warp >= 2) {
+        // -------------------------------------------- epilogue, part 2 --
+        const int t = int(threadIdx.x) - 64;
+        const int q = int(warp & 3u);       // TMEM lane quarter of this warp
+        const int c = q * 32 + int(lane);  // channel within the tile
+        if (have_acc) tc_fence_after();
+        if (S == 1) {
+            for (int c0 = 0; c0 < MP && have_acc; c0 += 16) {
+                uint32_t acc[16];
+                tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(c0), acc);
+                tmem_wait_ld();
+                if (n0 + c < N) {
+                    const float sw = sw_sm[c];
+#pragma unroll
+                    for (int mm = 0; mm < 16; ++mm)
+                        if (c0 + mm < M)
+                            args.Y[int64_t(c0 + mm) * N + n0 + c] =
+                                __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa_sm[c0 + mm] * sw);
+                }
+            }
+        } else {
+            // Partial row of channel c to its owner: slot [rank][c % CPR],
+            // MP token columns in 16-byte groups, group g at position
+            // g ^ recv_swz(c % CPR).
+            const int owner = c / CPR;
+            const int cl = c % CPR;
+            const int swz = recv_swz(cl, MP);
+            const uint32_t local = sbase + uint32_t(((rank * CPR + cl) * MP) * 4);
+            const uint32_t dst = mapa_shared(local, uint32_t(owner));
+            const uint32_t bar = mapa_shared(rbar, uint32_t(owner));
+            for (int c0 = 0; c0 < MP && have_acc; c0 += 16) {
+                uint32_t acc[16];
+                tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(c0), acc);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int g = c0 / 4 + h;
+                    st_async_v4(dst + 16u * uint32_t(g ^ swz),
+                                make_uint4(acc[4 * h], acc[4 * h + 1], acc[4 * h + 2], acc[4 * h + 3]), bar);
+                }
+            }
+            // Sum the S partials of the channels this rank owns, in rank order.
+            const bool have_partials = mbar_wait(rbar, 0, abort_flag);
+            if (!have_partials && t == 0) {
+                volatile int no_abort = 0;
+                mbar_wait(rbar, 0, &no_abort, 20000000ull);
+            }
+            if (have_partials) {
+                // One thread per (channel, group of 4 tokens): a 16-byte read
+                // per rank, consecutive channels across the warp, so the Y
+                // stores of each token row are contiguous.
+                const int G = (M + 3) / 4;
+                for (int e = t; e < CPR * G; e += 128) {
+                    const int cl2 = e % CPR, g = e / CPR;
+                    const int n = n0 + rank * CPR + cl2;
+                    const int pos = g ^ recv_swz(cl2, MP);
+                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int i = 0; i < S; ++i) {
+                        const float4 p = *reinterpret_cast<const float4*>(recv + (i * CPR + cl2) * MP + 4 * pos);
+                        sum.x += p.x;
+                        sum.y += p.y;
+                        sum.z += p.z;
+                        sum.w += p.w;
+                    }
+                    if (n < N) {
+                        const float sw = sw_sm[rank * CPR + cl2];
+                        const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (4 * g + j < M)
+                                args.Y[int64_t(4 * g + j) * N + n] = __float2bfloat16_rn(v[j] * sa_sm[4 * g + j] * sw);
+                    }
+                }
+            }
+        }
+    }
+
+    // A CTA receives remote stores only into its own ring after the cluster
+    // barrier above, and has waited for all of them (rbar) before it gets
+    // here.  After a timeout the waiting thread gave the late bytes a second
+    // bounded wait.
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, tcols);
+    }
+}
+
+}  // namespace cluster
+}  // namespace mfp8

@@ -16,9 +16,9 @@
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "gemm_tiled.cuh"
-#include "gemm_skinny.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_stream.cuh"
+#include "gemm_cluster.cuh"
 
 namespace mfp8 {
 namespace {
@@ -113,7 +113,7 @@ mfp8_status launch_status() {
 
 template <class Kern>
 mfp8_status launch_quant(Kern kern, bool dependent, int64_t R, const uint4* x, int64_t K, uint2* q, float* S,
-                         unsigned int* zero, int nzero, cudaStream_t stream) {
+                         cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(R));  // one block per row
     cfg.blockDim = dim3(kQuantThreads);
@@ -123,7 +123,7 @@ mfp8_status launch_quant(Kern kern, bool dependent, int64_t R, const uint4* x, i
     attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, x, K, q, S, zero, nzero) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, x, K, q, S) != cudaSuccess) {
         cudaGetLastError();
         return MFP8_ERR_CUDA;
     }
@@ -133,7 +133,7 @@ mfp8_status launch_quant(Kern kern, bool dependent, int64_t R, const uint4* x, i
 // The warp-per-row kernel: `blocks` blocks of 8 rows, R rows in all.
 template <class Kern>
 mfp8_status launch_quant(Kern kern, bool dependent, int64_t blocks, int64_t R, const uint4* x, int64_t K, uint2* q,
-                         float* S, unsigned int* zero, int nzero, cudaStream_t stream) {
+                         float* S, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
     cfg.blockDim = dim3(kQuantThreads);
@@ -143,7 +143,7 @@ mfp8_status launch_quant(Kern kern, bool dependent, int64_t blocks, int64_t R, c
     attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, x, R, K, q, S, zero, nzero) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, x, R, K, q, S) != cudaSuccess) {
         cudaGetLastError();
         return MFP8_ERR_CUDA;
     }
@@ -151,8 +151,7 @@ mfp8_status launch_quant(Kern kern, bool dependent, int64_t blocks, int64_t R, c
 }
 
 template <bool EARLY_TRIGGER>
-mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float* S, unsigned int* zero, int nzero,
-                            cudaStream_t stream) {
+mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
     if (R == 0) return MFP8_OK;
     const int64_t nvec = K / 8;
     const uint4* x = static_cast<const uint4*>(X);
@@ -163,32 +162,27 @@ mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float*
     const int64_t wblocks = (R + rows_per_block - 1) / rows_per_block;
     if (R >= 256 && nvec <= 32 * 16 && wblocks <= INT32_MAX) {
         if (nvec <= 32 * 4)
-            return launch_quant(quant_rows_warp_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, zero,
-                                nzero, stream);
+            return launch_quant(quant_rows_warp_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, stream);
         if (nvec <= 32 * 8)
-            return launch_quant(quant_rows_warp_kernel<8, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, zero,
-                                nzero, stream);
-        return launch_quant(quant_rows_warp_kernel<16, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, zero,
-                            nzero, stream);
+            return launch_quant(quant_rows_warp_kernel<8, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, stream);
+        return launch_quant(quant_rows_warp_kernel<16, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, stream);
     }
-    if (nvec <= 256) return launch_quant(quant_rows_reg_kernel<1, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
-    if (nvec <= 512) return launch_quant(quant_rows_reg_kernel<2, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
-    if (nvec <= 1024) return launch_quant(quant_rows_reg_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
-    if (nvec <= 1536) return launch_quant(quant_rows_reg_kernel<6, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
-    if (nvec <= 2048) return launch_quant(quant_rows_reg_kernel<8, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
-    return launch_quant(quant_rows_loop_kernel<EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, zero, nzero, stream);
+    if (nvec <= 256) return launch_quant(quant_rows_reg_kernel<1, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);
+    if (nvec <= 512) return launch_quant(quant_rows_reg_kernel<2, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);
+    if (nvec <= 1024) return launch_quant(quant_rows_reg_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);
+    if (nvec <= 1536) return launch_quant(quant_rows_reg_kernel<6, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);
+    if (nvec <= 2048) return launch_quant(quant_rows_reg_kernel<8, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);
+    return launch_quant(quant_rows_loop_kernel<EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);
 }
 
-// Activations: the GEMM launched next may start its prologue early.  Block 0
-// also clears the GEMM's split-K counters, if any.
-mfp8_status quantize_act_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream,
-                              unsigned int* zero = nullptr, int nzero = 0) {
-    return quantize_rows_t<true>(X, R, K, Q, S, zero, nzero, stream);
+// Activations: the GEMM launched next may start its prologue early.
+mfp8_status quantize_act_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
+    return quantize_rows_t<true>(X, R, K, Q, S, stream);
 }
 
 // Weights: no early start for whatever follows.
 mfp8_status quantize_weight_rows(const void* X, int64_t R, int64_t K, void* Q, float* S, cudaStream_t stream) {
-    return quantize_rows_t<false>(X, R, K, Q, S, nullptr, 0, stream);
+    return quantize_rows_t<false>(X, R, K, Q, S, stream);
 }
 
 mfp8_status check_quant_args(const void* X, int64_t R, int64_t K, const void* Q, const float* S) {
@@ -366,16 +360,18 @@ mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, 
     return launch_pair_bn<256, 6>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
 }
 
-constexpr int64_t kSkinnyMaxM = skinny::kMaxM;
 constexpr int64_t kStreamMaxM = stream::kMaxM;
-constexpr int kSkinnyStages = 4;
+constexpr int64_t kClusterMaxM = cluster::kMaxM;
 
 int sm_count_for_sizing();
 
 int choose_path(int64_t M, int64_t N, int64_t K) {
     (void)K;
     if (M <= kStreamMaxM) return MFP8_PATH_FUSED;
-    if (M <= 64 && (N + 255) / 256 <= 4096) return MFP8_PATH_SPLITK;
+    // The cluster split-K kernel up to 112 rows: at 128 its 32 KB stages
+    // (a weight block and 128 code rows) leave a 3-deep ring and the 128-row
+    // tiles were measured faster on the layer's shapes.
+    if (M <= 112) return MFP8_PATH_SPLITK;
     if (M < 256) return MFP8_PATH_TILED;
     // Too few 256 x 256 pair tiles to occupy half the CTA pairs (the k/v
     // projections at M = 2048 make 32): narrower single-CTA tiles fill the
@@ -400,92 +396,20 @@ mfp8_status check_gemm_args(int64_t M, int64_t N, int64_t K, const void* W8, con
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// K-splits of the skinny kernel: as many CTAs as SMs, no CTA without
-// k-blocks, and at most 16 partials for the last CTA of a tile to add up.
-int64_t skinny_splits(int64_t N, int64_t K, int sm_count) {
-    const int64_t tiles = (N + skinny::BN - 1) / skinny::BN;
-    const int64_t kb_total = (K + skinny::BK - 1) / skinny::BK;
-    int64_t splits = sm_count / tiles;
-    if (splits > 16) splits = 16;
-    if (splits < 1) splits = 1;
-    if (splits > kb_total) splits = kb_total;
-    return splits;
-}
-
-// How one call uses the caller's workspace.  The split-K tile counters sit
-// at a fixed place, the first kCounterBytes, in every layout: they must stay
-// zero between calls whatever shapes and paths share the workspace.  Then
-// the activation codes and scales of the quantize pass, then the split-K
-// fp32 partials [tile][split][M][256]; each region 256-byte aligned.
-constexpr int64_t kMaxSplitKTiles = 4096;  // N <= 1M for the split-K path
-constexpr size_t kCounterBytes = size_t(kMaxSplitKTiles) * 4;
-
+// How one call uses the caller's workspace: the activation codes X8 [M, K]
+// and scales s_a [M] of the quantize pass, each 256-byte aligned.  Nothing
+// in it outlives the call.
 struct Plan {
-    size_t x8_off = 0, sa_off = 0, part_off = 0, cnt_off = 0, total = 0;
-    int64_t tiles = 0, splits = 0;
+    size_t x8_off = 0, sa_off = 0, total = 0;
 };
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, bool codes, bool split_k, int sm_count) {
+Plan make_plan(int64_t M, int64_t K, bool codes) {
     Plan p;
-    if (!codes && !split_k) return p;  // nothing to keep: no workspace needed
-    size_t off = kCounterBytes;
-    p.cnt_off = 0;
-    if (codes) {
-        p.x8_off = off;
-        off += round_up(size_t(M) * size_t(K), 256);
-        p.sa_off = off;
-        off += round_up(size_t(M) * 4, 256);
-    }
-    if (split_k) {
-        p.tiles = (N + skinny::BN - 1) / skinny::BN;
-        p.splits = skinny_splits(N, K, sm_count);
-        p.part_off = off;
-        off += round_up(size_t(p.tiles * p.splits) * size_t(M) * skinny::BN * 4, 256);
-    }
-    p.total = off;
+    if (!codes) return p;  // nothing to keep: no workspace needed
+    p.x8_off = 0;
+    p.sa_off = round_up(size_t(M) * size_t(K), 256);
+    p.total = p.sa_off + round_up(size_t(M) * 4, 256);
     return p;
-}
-
-// The split-K GEMM on the codes X8 / scales s_a of the quantize pass.
-mfp8_status launch_skinny(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                          int64_t N, void* Y, float* partial, unsigned int* counters, const Plan& plan,
-                          bool weights_static, bool dependent, int dev, cudaStream_t stream) {
-    using L = skinny::Layout<kSkinnyStages>;
-    auto kern = skinny::gemm_skinny_kernel<kSkinnyStages>;
-    static bool attr_done[kMaxDevices] = {};
-    mfp8_status st = set_smem(kern, L::SMEM_BYTES, dev, attr_done);
-    if (st != MFP8_OK) return st;
-    CUtensorMap tmX, tmW;
-    if ((st = make_map_u8(&tmW, W8, N, K, skinny::BN)) != MFP8_OK) return st;
-    if ((st = make_map_u8(&tmX, X8, M, K, skinny::BM)) != MFP8_OK) return st;
-    if (plan.tiles > 65535) return MFP8_ERR_UNSUPPORTED_SHAPE;
-
-    skinny::Args args;
-    args.s_a = s_a;
-    args.s_w = s_w;
-    args.Y = static_cast<__nv_bfloat16*>(Y);
-    args.partial = partial;
-    args.counters = counters;
-    args.M = int(M);
-    args.N = int(N);
-    args.K = int(K);
-    args.weights_static = weights_static ? 1 : 0;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(plan.splits), unsigned(plan.tiles));
-    cfg.blockDim = dim3(skinny::kThreads);
-    cfg.dynamicSmemBytes = L::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, args) != cudaSuccess) {
-        cudaGetLastError();
-        return MFP8_ERR_CUDA;
-    }
-    return MFP8_OK;
 }
 
 // ------------------------------------------- decode: one-kernel Linear --
@@ -579,20 +503,86 @@ mfp8_status launch_stream(const void* X, int64_t M, int64_t K, const void* W8, c
     return MFP8_OK;
 }
 
+// ------------------------------ small / middle M: cluster split-K on codes --
+
+// Cluster size S (K split) of the split-K path: the decode kernel's rule (up
+// to 1.5 CTAs per SM, or 2 while each CTA keeps 8+ K blocks).  Ring: as many
+// weight + code stages as fit.
+bool cluster_geometry(int64_t M, int64_t N, int64_t K, int sm_count, cluster::Geometry* g) {
+    if (M < 1 || M > cluster::kMaxM) return false;
+    const int64_t tiles = (N + cluster::TILE - 1) / cluster::TILE;
+    const int64_t kb = (K + cluster::SUB - 1) / cluster::SUB;
+    int S = 1;
+    auto grow = [&](int s) {
+        if (s >= cluster::kMaxCluster || s * 2 > kb) return false;
+        const int64_t ctas = tiles * s * 2;
+        return ctas <= sm_count * 3 / 2 || (ctas <= int64_t(sm_count) * 2 && kb / (s * 2) >= 8);
+    };
+    while (grow(S)) S *= 2;
+    g->S = S;
+    g->mp = int((M + 15) / 16 * 16);
+    const int st = cluster::kRingBytes / cluster::stage_bytes(g->mp);
+    g->stages = st > cluster::kMaxStages ? cluster::kMaxStages : st;
+    return g->stages >= cluster::kMinStages;
+}
+
+mfp8_status launch_cluster(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
+                           int64_t N, void* Y, bool weights_static, bool dependent, int dev, const DeviceInfo& info,
+                           cudaStream_t stream) {
+    cluster::Geometry g;
+    if (!cluster_geometry(M, N, K, info.sm_count, &g)) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    auto kern = cluster::gemm_cluster_kernel;
+    static bool attr_done[kMaxDevices] = {};
+    mfp8_status st = set_smem(kern, cluster::Smem::BYTES, dev, attr_done);
+    if (st != MFP8_OK) return st;
+    const int64_t tiles = (N + cluster::TILE - 1) / cluster::TILE;
+    const int64_t grid = tiles * g.S;
+    if (grid > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    CUtensorMap tmX, tmW;
+    if ((st = make_map_u8(&tmW, W8, N, K, cluster::TILE)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmX, X8, M, K, g.mp)) != MFP8_OK) return st;
+
+    cluster::Args args;
+    args.s_a = s_a;
+    args.s_w = s_w;
+    args.Y = static_cast<__nv_bfloat16*>(Y);
+    args.M = int(M);
+    args.N = int(N);
+    args.K = int(K);
+    args.weights_static = weights_static ? 1 : 0;
+    args.g = g;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(cluster::kThreads);
+    cfg.dynamicSmemBytes = cluster::Smem::BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = dependent ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = unsigned(g.S);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmW, args) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
 // The GEMM on codes already in memory (tiled, pair, or split-K).
 mfp8_status run_gemm(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                     int64_t N, void* Y, int path, void* ws, const Plan& plan, bool weights_static, bool dependent,
-                     int dev, const DeviceInfo& info, cudaStream_t stream) {
+                     int64_t N, void* Y, int path, bool weights_static, bool dependent, int dev,
+                     const DeviceInfo& info, cudaStream_t stream) {
     // The kernels take M, N, K as 32-bit.
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (path == MFP8_PATH_TILED) return launch_tiled(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
     if (path == MFP8_PATH_PAIR) return launch_pair(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-    if (path == MFP8_PATH_SPLITK) {
-        uint8_t* base = static_cast<uint8_t*>(ws);
-        return launch_skinny(X8, s_a, M, K, W8, s_w, N, Y, reinterpret_cast<float*>(base + plan.part_off),
-                             reinterpret_cast<unsigned int*>(base + plan.cnt_off), plan, weights_static, dependent,
-                             dev, stream);
-    }
+    if (path == MFP8_PATH_SPLITK)
+        return launch_cluster(X8, s_a, M, K, W8, s_w, N, Y, weights_static, dependent, dev, info, stream);
     return MFP8_ERR_INVALID_ARG;
 }
 
@@ -612,24 +602,16 @@ int sm_count_for_sizing() {
 // in full up front (a fixed budget per GPU).  Every call on a device uses
 // the same bytes, so two calls that can be in flight at once race.
 constexpr size_t kStaticWsBytes = MFP8_STATIC_WORKSPACE_BYTES;
-static_assert(kStaticWsBytes >= kCounterBytes + 256, "static scratch must hold the split-K counters");
 static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
 
 void* g_static_ws_ptr[kMaxDevices] = {};
 
-// Once per device: the array's device address, and its split-K counters set
-// to zero (later calls leave them at zero).  The memset runs on the legacy
-// stream and is waited for here, so it is ordered before every later call on
-// any stream.  This is the only place the entry point synchronises.
+// Once per device: the array's device address.
 mfp8_status static_workspace(int dev, void** out) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_static_ws_ptr[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) {
-            cudaGetLastError();
-            return MFP8_ERR_CUDA;
-        }
-        if (cudaMemset(p, 0, kCounterBytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
             cudaGetLastError();
             return MFP8_ERR_CUDA;
         }
@@ -683,7 +665,7 @@ mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K, void* X_
 
 size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return 0;
-    return make_plan(M, N, K, true, M <= kSkinnyMaxM, sm_count_for_sizing()).total;
+    return make_plan(M, K, true).total;
 }
 
 mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
@@ -693,8 +675,7 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     if (st != MFP8_OK) return st;
     if (path < MFP8_PATH_AUTO || path > MFP8_PATH_FUSED) return MFP8_ERR_INVALID_ARG;
     if ((flags & ~MFP8_FLAG_STATIC_WEIGHTS) != 0) return MFP8_ERR_INVALID_ARG;
-    if (path == MFP8_PATH_SPLITK && (N + 255) / 256 > 4096) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    if (path == MFP8_PATH_SPLITK && M > kSkinnyMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_SPLITK && M > kClusterMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (path == MFP8_PATH_FUSED && M > kStreamMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_bf16) return MFP8_ERR_INVALID_ARG;
@@ -713,8 +694,7 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     // FUSED (M <= 16): one kernel quantizes X on chip and streams the
     // weights; it keeps nothing in the workspace.
     const bool fused = path == MFP8_PATH_FUSED;
-    const bool split_k = path == MFP8_PATH_SPLITK;
-    const Plan plan = fused ? Plan() : make_plan(M, N, K, X_fp8_out == nullptr, split_k, sm_count_for_sizing());
+    const Plan plan = fused ? Plan() : make_plan(M, K, X_fp8_out == nullptr);
     if (plan.total > 0) {
         if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
         if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
@@ -733,10 +713,8 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
                              X_fp8_out, x_scale_out, dev, info, s);
     void* X8 = X_fp8_out ? X_fp8_out : base + plan.x8_off;
     float* s_a = x_scale_out ? x_scale_out : reinterpret_cast<float*>(base + plan.sa_off);
-    unsigned int* counters = split_k ? reinterpret_cast<unsigned int*>(base + plan.cnt_off) : nullptr;
-    if ((st = quantize_act_rows(X_bf16, M, K, X8, s_a, s, counters, split_k ? int(plan.tiles) : 0)) != MFP8_OK)
-        return st;
-    return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, path, workspace, plan, weights_static,
+    if ((st = quantize_act_rows(X_bf16, M, K, X8, s_a, s)) != MFP8_OK) return st;
+    return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, path, weights_static,
                     /*dependent=*/true, dev, info, s);
 }
 
@@ -766,8 +744,8 @@ int mfp8_choose_path(int64_t M, int64_t N, int64_t K) {
 }
 
 size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return 0;
-    return make_plan(M, N, K, false, M <= kSkinnyMaxM, sm_count_for_sizing()).total;
+    (void)M, (void)N, (void)K;
+    return 0;  // the GEMM kernels keep nothing in a workspace
 }
 
 mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K, const void* W_fp8,
@@ -776,7 +754,7 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
     mfp8_status st = check_gemm_args(M, N, K, W_fp8, w_scale, Y_bf16);
     if (st != MFP8_OK) return st;
     if (path < MFP8_PATH_AUTO || path > MFP8_PATH_PAIR) return MFP8_ERR_INVALID_ARG;
-    if (path == MFP8_PATH_SPLITK && (M > kSkinnyMaxM || (N + 255) / 256 > 4096)) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (path == MFP8_PATH_SPLITK && M > kClusterMaxM) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return MFP8_OK;
     if (!X_fp8 || !x_scale) return MFP8_ERR_INVALID_ARG;
     if (!aligned16(X_fp8) || !aligned16(x_scale)) return MFP8_ERR_MISALIGNED;
@@ -785,19 +763,13 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
         return MFP8_ERR_INVALID_ARG;
     if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
     if (path == MFP8_PATH_FUSED) path = MFP8_PATH_SPLITK;  // codes given: the split-K kernel streams them
-    const bool split_k = path == MFP8_PATH_SPLITK;
-    const Plan plan = make_plan(M, N, K, false, split_k, sm_count_for_sizing());
-    if (plan.total > 0) {
-        if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
-        if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
-        if (ranges_overlap(workspace, plan.total, Y_bf16, size_t(M * N * 2))) return MFP8_ERR_INVALID_ARG;
-    }
+    (void)workspace, (void)workspace_bytes_given;  // kept in the signature; nothing needs it
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, workspace, plan,
-                    /*weights_static=*/false, /*dependent=*/false, dev, info, s);
+    return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, /*weights_static=*/false,
+                    /*dependent=*/false, dev, info, s);
 }
 
 mfp8_status mfp8_e4m3_encode_f32(const float* in, int64_t n, uint8_t* out, void* stream) {

@@ -148,12 +148,10 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red /* [
 // (that GEMM waits for the codes before reading them), then waits for the
 // grid before it.  The weight quantizer leaves it off, so nothing that
 // follows starts before the weight codes are complete.
-// Block 0 also clears `nzero` words at `zero` (the split-K counters of the
-// GEMM that follows in the same call).
 template <int VPT, bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
-                      float* __restrict__ S, unsigned int* __restrict__ zero, int nzero) {
+                      float* __restrict__ S) {
     // Launched as a programmatic dependent of the previous kernel.  The GEMM
     // that follows may start launching at once: before its own wait it only
     // sets itself up and (static weights) reads W, and one of its CTAs and
@@ -164,8 +162,6 @@ quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict_
         grid_launch_dependents();
         grid_dependency_wait();
     }
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < nzero; i += kQuantThreads) zero[i] = 0u;
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = K >> 3;
@@ -197,18 +193,16 @@ quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict_
 // One warp per row, 8 rows per block, for rows of at most 32 * VPL 16-byte
 // vectors (K <= 256 * VPL): the row stays in registers, the absmax is a warp
 // reduction, and no block barrier holds up the other rows.  Loads and stores
-// are lane-contiguous (512 and 256 bytes per instruction).  EARLY_TRIGGER,
-// `zero` and `nzero` as in quant_rows_reg_kernel.
+// are lane-contiguous (512 and 256 bytes per instruction).  EARLY_TRIGGER as
+// in quant_rows_reg_kernel.
 template <int VPL, bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_warp_kernel(const uint4* __restrict__ X, int64_t R, int64_t K, uint2* __restrict__ Q,
-                       float* __restrict__ S, unsigned int* __restrict__ zero, int nzero) {
+                       float* __restrict__ S) {
     if (EARLY_TRIGGER) {
         grid_launch_dependents();
         grid_dependency_wait();
     }
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < nzero; i += kQuantThreads) zero[i] = 0u;
     const int64_t row = int64_t(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5);
     if (row >= R) return;
     const int lane = threadIdx.x & 31;
@@ -245,13 +239,11 @@ quant_rows_warp_kernel(const uint4* __restrict__ X, int64_t R, int64_t K, uint2*
 template <bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_loop_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict__ Q,
-                       float* __restrict__ S, unsigned int* __restrict__ zero, int nzero) {
+                       float* __restrict__ S) {
     if (EARLY_TRIGGER) {  // as in quant_rows_reg_kernel
         grid_launch_dependents();
         grid_dependency_wait();
     }
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < nzero; i += kQuantThreads) zero[i] = 0u;
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = K >> 3;

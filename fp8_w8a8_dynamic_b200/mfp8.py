@@ -107,7 +107,7 @@ def mfp8_choose_path(M, N, K):
     return lib().mfp8_choose_path(M, N, K)
 
 
-KERNEL_OF_PATH = {PATH_TILED: "gemm_tiled_kernel", PATH_SPLITK: "gemm_skinny_kernel",
+KERNEL_OF_PATH = {PATH_TILED: "gemm_tiled_kernel", PATH_SPLITK: "gemm_cluster_kernel",
                   PATH_PAIR: "gemm_pair_kernel", PATH_FUSED: "gemm_stream_kernel"}
 
 

@@ -86,10 +86,10 @@ MFP8_API mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K,
                               void* X_fp8, float* x_scale, void* stream);
 
 /* Bytes of device workspace that are enough for mfp8_linear and for every
- * kernel choice of mfp8_linear_ex at these sizes on the current device: the
- * activation codes and scales of the quantize pass and, for M <= 128, the
- * fp32 split-K partials and per-tile counters.  Never fails; returns 0 for
- * invalid sizes (mfp8_linear then reports the error). */
+ * kernel choice of mfp8_linear_ex at these sizes: the activation codes
+ * [M, K] and scales [M] of the quantize pass, each rounded up to 256 bytes.
+ * Never fails; returns 0 for invalid sizes (mfp8_linear then reports the
+ * error). */
 MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* The FP8_DYNAMIC Linear: Y = bf16(  (Xq . Wq^T) * x_scale (x) w_scale  ).
@@ -101,12 +101,11 @@ MFP8_API size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   Y_bf16   [M, N] bf16, written.  Must not overlap any input.
  *   workspace / workspace_bytes: device scratch of at least
  *            mfp8_linear_workspace_bytes(M, N, K) bytes, 16-byte aligned,
- *            ZERO-FILLED before its first use (e.g. one cudaMemset).  It
- *            holds the activation codes and, for decode sizes, the split-K
- *            partials and one counter per output tile; every call leaves the
- *            counters at zero, so the zero-fill is needed once, and again
- *            only after a call reported MFP8_ERR_TIMEOUT.  Calls that may run
- *            at the same time need separate workspaces.
+ *            any contents.  It holds the activation codes and scales between
+ *            the quantize pass and the GEMM of this call; nothing in it
+ *            outlives the call.  Calls that may run at the same time need
+ *            separate workspaces.  The one-kernel decode path (M <= 16) does
+ *            not touch it.
  * The activation quantization (per-token scale + e4m3 codes) happens inside
  * this call: its codes and scales are bit-identical to mfp8_quantize_act.
  * Outputs are within |y - y_ref| <= 2^-7 |y_ref| + 1e-5 * sum_k |a_k w_k| s_a s_w
@@ -120,14 +119,14 @@ MFP8_API mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K,
 typedef enum {
     MFP8_PATH_AUTO = 0,   /* what mfp8_linear does: chosen from M, N, K */
     MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
-    MFP8_PATH_SPLITK = 2, /* quantize pass, then the weight-streaming split-K GEMM over all SMs (M <= 128) */
+    MFP8_PATH_SPLITK = 2, /* quantize pass, then the split-K GEMM on CTA clusters, partials summed on chip (M <= 128) */
     MFP8_PATH_PAIR = 3,   /* quantize pass, then the 256-row-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
     MFP8_PATH_FUSED = 4   /* one kernel: quantizes X on chip and streams the weights, whole K per CTA (M <= 16) */
 } mfp8_path;
 
 /* The kernel MFP8_PATH_AUTO takes at these sizes (FUSED for M <= 16, SPLITK
- * up to 64, TILED below 256, PAIR above); MFP8_PATH_AUTO itself for sizes no
- * kernel takes. */
+ * up to 112, TILED below 256, PAIR above); MFP8_PATH_AUTO itself for sizes
+ * no kernel takes. */
 MFP8_API int mfp8_choose_path(int64_t M, int64_t N, int64_t K);
 
 /* Flags for mfp8_linear_ex. */
@@ -168,31 +167,25 @@ MFP8_API mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K,
  *   Arguments, results and tolerance: as mfp8_linear (kernel choice AUTO).
  *   Sizes whose mfp8_linear_workspace_bytes(M, N, K) exceeds
  *   MFP8_STATIC_WORKSPACE_BYTES are rejected with MFP8_ERR_WORKSPACE before
- *   any device work (e.g. M <= 64 fits every projection up to N, K = 12288;
- *   the quantized activations of larger M need M * K bytes).
- *   Set-up: the first call on each device looks up the array's address and
- *   zeroes its counters, then waits for the device (cudaDeviceSynchronize).
- *   Make that first call before any stream capture begins.
+ *   any device work (the quantized activations need about M * K bytes:
+ *   every projection up to K = 12288 fits for M <= 1300).
+ *   Set-up: the first call on each device looks up the array's address.
  *   Concurrency: every call on a device shares the one scratch array.  Calls
  *   that may be in flight at the same time (different streams, or host
- *   threads) race and give wrong results; serialise them, e.g. on one stream.
- *   After a call reported MFP8_ERR_TIMEOUT the next call still starts from
- *   zeroed counters (the quantize pass clears them). */
+ *   threads) race and give wrong results; serialise them, e.g. on one stream. */
 MFP8_API mfp8_status mfp8_linear_noalloc(const void* X_bf16, int64_t M, int64_t K,
                                 const void* W_fp8, const float* w_scale, int64_t N,
                                 void* Y_bf16, void* stream);
 
-/* Workspace bytes mfp8_gemm needs at these sizes on the current device
- * (the split-K partials and counters; 0 when no kernel choice needs any). */
+/* Workspace bytes mfp8_gemm needs: 0, since no GEMM kernel keeps anything
+ * in one (kept for callers that size a workspace before they call). */
 MFP8_API size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* The contraction and epilogue alone, on activations already quantized by
  * mfp8_quantize_act: Y = bf16((X_fp8 . W_fp8^T) * x_scale (x) w_scale).
  * Lets the GEMM be timed and checked without the quantize pass.  path is
- * AUTO, TILED, SPLITK or PAIR; the split-K kernel takes its partials and
- * tile counters from `workspace` (at least mfp8_gemm_workspace_bytes), under
- * the same contract as mfp8_linear: zero-filled before its first use, the
- * counters left at zero by every call. */
+ * AUTO, TILED, SPLITK or PAIR (FUSED is taken as SPLITK: the codes are
+ * given).  `workspace` and `workspace_bytes` are not used. */
 MFP8_API mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K,
                       const void* W_fp8, const float* w_scale, int64_t N,
                       void* Y_bf16, void* workspace, size_t workspace_bytes,

@@ -56,26 +56,22 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_bytes(lib):
-    # 16 KB of split-K counters first (a fixed place in every layout), then X8
-    # [M, K] and s_a [M], each rounded up to 256 bytes, then for M <= 128 the
-    # split-K partials [tiles][splits][M][256] fp32 (sized for 148 SMs when no
-    # device is present)
-    C = 16384
-    assert mfp8.mfp8_linear_workspace_bytes(300, 4096, 4096) == C + 300 * 4096 + 1280
-    tiles, splits = 16, 9  # N = 4096 in 256-wide tiles; 148 // 16 K-splits
-    assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == C + 65536 + 256 + tiles * splits * 16 * 1024
-    assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == C + tiles * splits * 16 * 1024
+    # X8 [M, K] and s_a [M] of the quantize pass, each rounded up to 256 bytes
+    assert mfp8.mfp8_linear_workspace_bytes(300, 4096, 4096) == 300 * 4096 + 1280
+    assert mfp8.mfp8_linear_workspace_bytes(16, 4096, 4096) == 65536 + 256
+    assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == 256 + 256
+    assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == 0
     assert mfp8.mfp8_gemm_workspace_bytes(300, 4096, 4096) == 0
-    # the AUTO choice: the one-kernel path up to 16 tokens, split-K to 64,
-    # 128-row tiles for mid M, pairs above
+    # the AUTO choice: the one-kernel path up to 16 tokens, the cluster
+    # split-K kernel to 112, 128-row tiles for mid M, pairs above
     assert mfp8.mfp8_choose_path(8, 12288, 4096) == mfp8.PATH_FUSED
     assert mfp8.mfp8_choose_path(16, 4096, 12288) == mfp8.PATH_FUSED
     assert mfp8.mfp8_choose_path(17, 4096, 4096) == mfp8.PATH_SPLITK
+    assert mfp8.mfp8_choose_path(112, 4096, 4096) == mfp8.PATH_SPLITK
+    assert mfp8.mfp8_choose_path(128, 4096, 4096) == mfp8.PATH_TILED
     assert mfp8.mfp8_choose_path(200, 4096, 4096) == mfp8.PATH_TILED
     assert mfp8.mfp8_choose_path(2048, 4096, 4096) == mfp8.PATH_PAIR
     assert mfp8.mfp8_choose_path(0, 4096, 4096) == mfp8.PATH_AUTO
-    # one K-block only: one split
-    assert mfp8.mfp8_linear_workspace_bytes(3, 8, 48) == C + 256 + 256 + 3 * 1024
     assert mfp8.mfp8_linear_workspace_bytes(0, 8, 48) == 0
     assert mfp8.mfp8_linear_workspace_bytes(4, 8, -1) == 0
 
@@ -115,7 +111,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert call(path=7) == mfp8.ERR_INVALID_ARG
     assert call(path=5) == mfp8.ERR_INVALID_ARG
     assert call(path=mfp8.PATH_FUSED, M=17) == mfp8.ERR_UNSUPPORTED_SHAPE
-    assert call(ws=None, path=mfp8.PATH_SPLITK) == mfp8.ERR_WORKSPACE  # split-K partials
+    assert call(ws=None, path=mfp8.PATH_SPLITK) == mfp8.ERR_WORKSPACE  # the quantize pass's codes
     assert call(path=mfp8.PATH_SPLITK, M=129) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
     assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X
@@ -127,7 +123,9 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert NA(FAKE, 4096, 8192, FAKE * 2, FAKE * 3, 64, FAKE * 4, None) == mfp8.ERR_WORKSPACE
     G = mfp8.mfp8_gemm
     assert G(None, FAKE, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_INVALID_ARG
-    assert G(FAKE, FAKE * 9, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_WORKSPACE
+    assert G(FAKE, FAKE * 9 + 4, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_MISALIGNED
+    assert G(FAKE, FAKE * 9, 129, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, mfp8.PATH_SPLITK,
+             None) == mfp8.ERR_UNSUPPORTED_SHAPE  # split-K kernel: M <= 128
     assert G(FAKE, FAKE * 9, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, mfp8.PATH_FUSED, None) == mfp8.ERR_INVALID_ARG
     assert mfp8.mfp8_e4m3_encode_f32(FAKE, -1, FAKE * 2, None) == mfp8.ERR_INVALID_ARG
     assert mfp8.mfp8_debug_bounded_wait(0, None) == mfp8.ERR_INVALID_ARG

@@ -239,14 +239,13 @@ def test_long_video_full_size_sampled(lin):
 
 
 def test_workspace_reused_across_calls_and_shapes():
-    """The split-K counters live in the caller's workspace and every call
-    leaves them at zero: one zero-filled workspace serves a sequence of
-    calls of different sizes and paths, each within tolerance."""
+    """One workspace serves a sequence of calls of different sizes and
+    paths, whatever earlier calls left in it: each is within tolerance."""
     cases = [(16, 12288, 4096, mfp8.PATH_AUTO), (1, 4096, 4096, mfp8.PATH_SPLITK), (8, 1024, 4096, mfp8.PATH_AUTO),
              (40, 2048, 1024, mfp8.PATH_SPLITK), (300, 512, 1024, mfp8.PATH_TILED), (3, 4096, 4096, mfp8.PATH_AUTO),
              (16, 12288, 4096, mfp8.PATH_SPLITK)]
     nbytes = max(mfp8.mfp8_linear_workspace_bytes(M, N, K) for M, N, K, _ in cases)
-    big = torch.zeros((nbytes,), dtype=torch.uint8, device=DEV)
+    big = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device=DEV)  # not zero-filled: nothing needs it
     for i, (M, N, K, path) in enumerate(cases):
         x = W.make_x(M, K, seed=30 + i, device=DEV)
         W8, sw = mfp8.quantize_weight(W.make_w(N, K, seed=30 + i, device=DEV))

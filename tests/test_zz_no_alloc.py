@@ -13,9 +13,9 @@ from fp8_w8a8_dynamic_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
-# decode sizes (split-K partials and counters in the scratch), a ragged
-# mid-size M (activation codes in the scratch, 128-row tiles), and a
-# prefill-sized M (the CTA-pair kernel)
+# decode sizes (the one-kernel path, no scratch), M = 64 (activation codes
+# in the scratch, the cluster split-K kernel), a ragged mid-size M
+# (128-row tiles), and a prefill-sized M (the CTA-pair kernel)
 CASES = [(4, 1024, 4096), (16, 12288, 4096), (1, 4096, 12288), (64, 4096, 12288),
          (200, 4096, 4096), (1000, 4096, 4096)]
 
