@@ -91,6 +91,23 @@ def test_fused_stream_geometry(M, N, K):
     run_case(M, N, K, mfp8.PATH_FUSED, seed=M * 5 + K, flags=mfp8.FLAG_STATIC_WEIGHTS if M % 2 else 0)
 
 
+# The cluster split-K kernel on codes: token columns 16..128 (M rounded up
+# to 16, with ragged M), cluster sizes 1..8, a ragged last K block, a K
+# shorter than one block, a partial last channel tile (N % 128 != 0), grids
+# of many tiles, and long K.
+CLUSTER = [
+    (17, 8, 16), (24, 136, 272), (48, 1032, 4112), (64, 6144, 4096), (80, 264, 4992), (96, 4096, 12288),
+    (112, 520, 1040), (128, 12296, 2064), (33, 40960, 256), (127, 1024, 8320), (65, 24576, 4096),
+]
+
+
+@pytest.mark.parametrize("M,N,K", CLUSTER)
+def test_cluster_splitk_geometry(M, N, K):
+    big = M * N * K > 1 << 30  # the oracle's exact contraction on sampled rows only
+    run_case(M, N, K, mfp8.PATH_SPLITK, seed=M * 3 + K, kind="rowscale",
+             rows=sampled_rows(M, 8, K) if big else None, flags=mfp8.FLAG_STATIC_WEIGHTS if M % 2 else 0)
+
+
 @pytest.mark.parametrize("M", list(range(1, 17)))
 def test_fused_every_m(M):
     run_case(M, 4096, 4096, mfp8.PATH_FUSED, seed=100 + M, kind="rowscale" if M > 2 else "normal")
