@@ -156,16 +156,27 @@ mfp8_status quantize_rows_t(const void* X, int64_t R, int64_t K, void* Q, float*
     const int64_t nvec = K / 8;
     const uint4* x = static_cast<const uint4*>(X);
     uint2* q = static_cast<uint2*>(Q);
-    // Many rows: one warp per row (8 rows per block) while a row fits in a
-    // warp's registers.
-    const int64_t rows_per_block = kQuantThreads / 32;
-    const int64_t wblocks = (R + rows_per_block - 1) / rows_per_block;
-    if (R >= 256 && nvec <= 32 * 16 && wblocks <= INT32_MAX) {
+    // Many rows: 1, 2 or 4 warps per row (8 warps per block) while a row
+    // fits in their registers; longer rows get more warps.
+    auto blocks = [&](int wpr) { return (R * wpr + kQuantThreads / 32 - 1) / (kQuantThreads / 32); };
+    if (R >= 256 && nvec <= 32 * 16 * 4 && blocks(4) <= INT32_MAX) {
         if (nvec <= 32 * 4)
-            return launch_quant(quant_rows_warp_kernel<4, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, stream);
+            return launch_quant(quant_rows_warp_kernel<4, 1, EARLY_TRIGGER>, EARLY_TRIGGER, blocks(1), R, x, K, q, S,
+                                stream);
         if (nvec <= 32 * 8)
-            return launch_quant(quant_rows_warp_kernel<8, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, stream);
-        return launch_quant(quant_rows_warp_kernel<16, EARLY_TRIGGER>, EARLY_TRIGGER, wblocks, R, x, K, q, S, stream);
+            return launch_quant(quant_rows_warp_kernel<8, 1, EARLY_TRIGGER>, EARLY_TRIGGER, blocks(1), R, x, K, q, S,
+                                stream);
+        if (nvec <= 32 * 8 * 2)
+            return launch_quant(quant_rows_warp_kernel<8, 2, EARLY_TRIGGER>, EARLY_TRIGGER, blocks(2), R, x, K, q, S,
+                                stream);
+        if (nvec <= 32 * 8 * 4)
+            return launch_quant(quant_rows_warp_kernel<8, 4, EARLY_TRIGGER>, EARLY_TRIGGER, blocks(4), R, x, K, q, S,
+                                stream);
+        if (nvec <= 32 * 12 * 4)
+            return launch_quant(quant_rows_warp_kernel<12, 4, EARLY_TRIGGER>, EARLY_TRIGGER, blocks(4), R, x, K, q, S,
+                                stream);
+        return launch_quant(quant_rows_warp_kernel<16, 4, EARLY_TRIGGER>, EARLY_TRIGGER, blocks(4), R, x, K, q, S,
+                            stream);
     }
     if (nvec <= 256) return launch_quant(quant_rows_reg_kernel<1, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);
     if (nvec <= 512) return launch_quant(quant_rows_reg_kernel<2, EARLY_TRIGGER>, EARLY_TRIGGER, R, x, K, q, S, stream);

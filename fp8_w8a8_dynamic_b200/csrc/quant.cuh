@@ -190,47 +190,62 @@ quant_rows_reg_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict_
     }
 }
 
-// One warp per row, 8 rows per block, for rows of at most 32 * VPL 16-byte
-// vectors (K <= 256 * VPL): the row stays in registers, the absmax is a warp
-// reduction, and no block barrier holds up the other rows.  Loads and stores
-// are lane-contiguous (512 and 256 bytes per instruction).  EARLY_TRIGGER as
-// in quant_rows_reg_kernel.
-template <int VPL, bool EARLY_TRIGGER>
+// WPR warps per row (1, 2 or 4), 8 / WPR rows per block, for rows of at
+// most 32 * VPL * WPR 16-byte vectors: the row stays in registers, each warp
+// holds a contiguous share of it, the absmax is a warp reduction (and, with
+// WPR > 1, a max over the row's warps through shared memory), and each warp
+// then quantizes and stores its own share.  Loads and stores are
+// lane-contiguous (512 and 256 bytes per instruction).  More warps per row
+// give the SM more loads in flight and shorten each warp's serial chain.
+// EARLY_TRIGGER as in quant_rows_reg_kernel.
+template <int VPL, int WPR, bool EARLY_TRIGGER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_warp_kernel(const uint4* __restrict__ X, int64_t R, int64_t K, uint2* __restrict__ Q,
                        float* __restrict__ S) {
+    static_assert(WPR == 1 || WPR == 2 || WPR == 4, "1, 2 or 4 warps per row");
+    constexpr int kRowsPerBlock = kQuantThreads / 32 / WPR;
     if (EARLY_TRIGGER) {
         grid_launch_dependents();
         grid_dependency_wait();
     }
-    const int64_t row = int64_t(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5);
-    if (row >= R) return;
+    const int w = threadIdx.x >> 5;
+    const int part = w % WPR;
+    const int64_t row = int64_t(blockIdx.x) * kRowsPerBlock + w / WPR;
+    const bool live = row < R;
     const int lane = threadIdx.x & 31;
     const int64_t nvec = K >> 3;
-    const uint4* xr = X + row * nvec;
+    const uint4* xr = X + (live ? row : 0) * nvec;
     uint4 v[VPL];
     uint32_t acc = 0;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-        const int64_t j = lane + 32 * i;
-        v[i] = j < nvec ? __ldg(xr + j) : make_uint4(0, 0, 0, 0);
+        const int64_t j = int64_t(part * VPL + i) * 32 + lane;
+        v[i] = (live && j < nvec) ? __ldg(xr + j) : make_uint4(0, 0, 0, 0);
         acc = absmax_bits_u4(v[i], acc);
     }
-    const uint32_t amax = __reduce_max_sync(0xffffffffu, max(acc & 0xffffu, acc >> 16));
+    uint32_t amax = __reduce_max_sync(0xffffffffu, max(acc & 0xffffu, acc >> 16));
+    if (WPR > 1) {
+        __shared__ uint32_t red[kQuantThreads / 32];
+        if (lane == 0) red[w] = amax;
+        __syncthreads();
+#pragma unroll
+        for (int p = 0; p < WPR; ++p) amax = max(amax, red[(w / WPR) * WPR + p]);
+    }
+    if (!live) return;
     const float s = scale_from_absmax_bits(amax);
     const float r = __frcp_rn(s);
-    if (lane == 0) S[row] = s;
+    if (part == 0 && lane == 0) S[row] = s;
     uint2* qr = Q + row * nvec;
     if (s < kFmaMinScale) {
         for (int i = 0; i < VPL; ++i) {
-            const int64_t j = lane + 32 * i;
+            const int64_t j = int64_t(part * VPL + i) * 32 + lane;
             if (j < nvec) qr[j] = quantize8_div_call(v[i], s);
         }
         return;
     }
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-        const int64_t j = lane + 32 * i;
+        const int64_t j = int64_t(part * VPL + i) * 32 + lane;
         if (j < nvec) qr[j] = quantize8_fast(v[i], s, r);
     }
 }
