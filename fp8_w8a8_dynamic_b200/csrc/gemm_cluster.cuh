@@ -20,8 +20,9 @@
 //     weights before the dependency wait when they are static;
 //   - one thread issues 4 MMAs per K block;
 //   - with S > 1, once every CTA of the cluster has its accumulator (a
-//     cluster barrier), each channel's partial row goes with st.async to the
-//     CTA that owns the channel, into that CTA's ring (free by then), and the
+//     cluster barrier), each channel's partial row goes with plain remote
+//     stores to the CTA that owns the channel, into that CTA's ring (free by
+//     then), followed by one releasing arrival on the owner's barrier; the
 //     owner adds the S partials in rank order (deterministic), scales and
 //     stores BF16.  With S = 1 the epilogue stores directly.
 // About 98 KB of shared memory and at most 128 TMEM columns, so two CTAs
@@ -138,12 +139,12 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(tfull_bar, 1);
-        mbar_init(rbar, 1);
+        // (S > 1) one arrival from each thread, in every CTA, whose channel
+        // this CTA owns: S ranks x 128/S channels
+        mbar_init(rbar, S > 1 ? TILE : 1);
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        // (S > 1) the S partial rows of each of the 128/S channels it owns
-        if (S > 1) mbar_arrive_expect_tx(rbar, uint32_t(TILE * MP * 4));
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
     }
@@ -286,7 +287,9 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         } else {
             // Partial row of channel c to its owner: slot [rank][c % CPR],
             // MP token columns in 16-byte groups, group g at position
-            // g ^ recv_swz(c % CPR).
+            // g ^ recv_swz(c % CPR).  Plain remote stores, then one arrival
+            // on the owner's barrier that releases them (per-store
+            // transaction counting made each store a round trip).
             const int owner = c / CPR;
             const int cl = c % CPR;
             const int swz = recv_swz(cl, MP);
@@ -300,49 +303,57 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int g = c0 / 4 + h;
-                    st_async_v4(dst + 16u * uint32_t(g ^ swz),
-                                make_uint4(acc[4 * h], acc[4 * h + 1], acc[4 * h + 2], acc[4 * h + 3]), bar);
+                    st_cluster_v4(dst + 16u * uint32_t(g ^ swz),
+                                  make_uint4(acc[4 * h], acc[4 * h + 1], acc[4 * h + 2], acc[4 * h + 3]));
                 }
             }
+            if (have_acc) mbar_arrive_remote_release(bar);
             // Sum the S partials of the channels this rank owns, in rank order.
-            const bool have_partials = mbar_wait(rbar, 0, abort_flag);
+            const bool have_partials = mbar_wait_cluster(rbar, 0, abort_flag);
             if (!have_partials && t == 0) {
                 volatile int no_abort = 0;
-                mbar_wait(rbar, 0, &no_abort, 20000000ull);
+                mbar_wait_cluster(rbar, 0, &no_abort, 20000000ull);
             }
             if (have_partials) {
                 // One thread per (channel, group of 4 tokens): a 16-byte read
-                // per rank, consecutive channels across the warp, so the Y
-                // stores of each token row are contiguous.
+                // per rank (all S issued together), consecutive channels
+                // across the warp, so the Y stores of each token row are
+                // contiguous.  Thread t keeps channel t % CPR and walks the
+                // groups t / CPR, t / CPR + 128 / CPR, ...
                 const int G = (M + 3) / 4;
-                for (int e = t; e < CPR * G; e += 128) {
-                    const int cl2 = e % CPR, g = e / CPR;
-                    const int n = n0 + rank * CPR + cl2;
-                    const int pos = g ^ recv_swz(cl2, MP);
-                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int i = 0; i < S; ++i) {
-                        const float4 p = *reinterpret_cast<const float4*>(recv + (i * CPR + cl2) * MP + 4 * pos);
-                        sum.x += p.x;
-                        sum.y += p.y;
-                        sum.z += p.z;
-                        sum.w += p.w;
-                    }
-                    if (n < N) {
-                        const float sw = sw_sm[rank * CPR + cl2];
-                        const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+                const int cl2 = t % CPR;
+                const int n = n0 + rank * CPR + cl2;
+                const float sw = sw_sm[rank * CPR + cl2];
+                const int swz2 = recv_swz(cl2, MP);
+                const float* base = recv + cl2 * MP;
+                for (int g = t / CPR; g < G && n < N; g += 128 / CPR) {
+                    const int pos = g ^ swz2;
+                    float4 p[kMaxCluster];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            if (4 * g + j < M)
-                                args.Y[int64_t(4 * g + j) * N + n] = __float2bfloat16_rn(v[j] * sa_sm[4 * g + j] * sw);
-                    }
+                    for (int i = 0; i < kMaxCluster; ++i)
+                        if (i < S) p[i] = *reinterpret_cast<const float4*>(base + i * CPR * MP + 4 * pos);
+                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int i = 0; i < kMaxCluster; ++i)
+                        if (i < S) {
+                            sum.x += p[i].x;
+                            sum.y += p[i].y;
+                            sum.z += p[i].z;
+                            sum.w += p[i].w;
+                        }
+                    const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (4 * g + j < M)
+                            args.Y[int64_t(4 * g + j) * N + n] = __float2bfloat16_rn(v[j] * sa_sm[4 * g + j] * sw);
                 }
             }
         }
     }
 
     // A CTA receives remote stores only into its own ring after the cluster
-    // barrier above, and has waited for all of them (rbar) before it gets
-    // here.  After a timeout the waiting thread gave the late bytes a second
+    // barrier above, and has waited for all of them (the senders' releasing
+    // arrivals on rbar) before it gets here.  After a timeout the waiting thread gave the late bytes a second
     // bounded wait.
     tc_fence_before();
     __syncthreads();
