@@ -140,6 +140,35 @@ def test_fused_back_to_back_on_one_stream():
     assert torch.isfinite(a.float()).all()
 
 
+@pytest.mark.parametrize("M,path", [(32, mfp8.PATH_SPLITK), (112, mfp8.PATH_SPLITK), (200, mfp8.PATH_TILED),
+                                    (512, mfp8.PATH_PAIR)])
+def test_dependent_chain_every_path(M, path):
+    """Each call is a quantize pass that lets its GEMM start early and a GEMM
+    that waits for the codes; consecutive calls overlap the same way.  A
+    chain where each Linear's input is the previous Linear's output must
+    equal the same chain run one call at a time with a synchronisation in
+    between, bit for bit."""
+    H = 2048
+    Ws = [mfp8.quantize_weight(W.make_w(H, H, seed=70 + i, device=DEV)) for i in range(5)]
+    x0 = W.make_x(M, H, seed=71, kind="rowscale", device=DEV)
+    ws = torch.zeros((mfp8.mfp8_linear_workspace_bytes(M, H, H),), dtype=torch.uint8, device=DEV)
+    torch.cuda.synchronize()
+
+    def chain(sync):
+        x = x0
+        for W8, sw in Ws:
+            x = mfp8.linear(x, W8, sw, workspace=ws, path=path, flags=mfp8.FLAG_STATIC_WEIGHTS)
+            if sync:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return x
+
+    a, b = chain(False), chain(True)
+    assert mfp8.device_status() == mfp8.OK
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.isfinite(a.float()).all()
+
+
 @pytest.mark.parametrize("M,N,K", TILED_ONLY + [(513, 776, 1024), (2048, 1024, 4096)])
 @pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_PAIR])
 def test_linear_tiled_ragged(M, N, K, path):
