@@ -119,7 +119,6 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::MISC_OFF + 4);
     float* sa_sm = reinterpret_cast<float*>(smem + Smem::SA_OFF);
     float* sw_sm = reinterpret_cast<float*>(smem + Smem::SW_OFF);
-    const float* recv = reinterpret_cast<const float*>(smem);
 
     const uint32_t warp = warp_id_sync();
     const uint32_t lane = lane_id();
@@ -276,12 +275,22 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(c0), acc);
                 tmem_wait_ld();
                 if (n0 + c < N) {
-                    const float sw = sw_sm[c];
+                    // scales read before the stores (see ld_shared_f4)
+                    const float sw = ld_shared_f32(smem_u32(sw_sm + c));
+                    float sa[16];
+#pragma unroll
+                    for (int mm = 0; mm < 16; mm += 4) {
+                        const float4 v = ld_shared_f4(smem_u32(sa_sm + c0 + mm));
+                        sa[mm] = v.x;
+                        sa[mm + 1] = v.y;
+                        sa[mm + 2] = v.z;
+                        sa[mm + 3] = v.w;
+                    }
 #pragma unroll
                     for (int mm = 0; mm < 16; ++mm)
                         if (c0 + mm < M)
                             args.Y[int64_t(c0 + mm) * N + n0 + c] =
-                                __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa_sm[c0 + mm] * sw);
+                                __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa[mm] * sw);
                 }
             }
         } else {
@@ -320,18 +329,21 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 // across the warp, so the Y stores of each token row are
                 // contiguous.  Thread t keeps channel t % CPR and walks the
                 // groups t / CPR, t / CPR + 128 / CPR, ...
+                // Shared memory is read by shared-space address (ld_shared_*)
+                // so that the reads are not ordered behind the Y stores.
                 const int G = (M + 3) / 4;
                 const int cl2 = t % CPR;
                 const int n = n0 + rank * CPR + cl2;
-                const float sw = sw_sm[rank * CPR + cl2];
+                const float sw = ld_shared_f32(smem_u32(sw_sm + rank * CPR + cl2));
                 const int swz2 = recv_swz(cl2, MP);
-                const float* base = recv + cl2 * MP;
+                const uint32_t base = sbase + uint32_t(cl2 * MP * 4);
+                const uint32_t sa_base = smem_u32(sa_sm);
                 for (int g = t / CPR; g < G && n < N; g += 128 / CPR) {
                     const int pos = g ^ swz2;
                     float4 p[kMaxCluster];
 #pragma unroll
                     for (int i = 0; i < kMaxCluster; ++i)
-                        if (i < S) p[i] = *reinterpret_cast<const float4*>(base + i * CPR * MP + 4 * pos);
+                        if (i < S) p[i] = ld_shared_f4(base + uint32_t((i * CPR * MP + 4 * pos) * 4));
                     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                     for (int i = 0; i < kMaxCluster; ++i)
@@ -342,10 +354,12 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                             sum.w += p[i].w;
                         }
                     const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+                    const float4 sa4 = ld_shared_f4(sa_base + uint32_t(16 * g));
+                    const float sa[4] = {sa4.x, sa4.y, sa4.z, sa4.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         if (4 * g + j < M)
-                            args.Y[int64_t(4 * g + j) * N + n] = __float2bfloat16_rn(v[j] * sa_sm[4 * g + j] * sw);
+                            args.Y[int64_t(4 * g + j) * N + n] = __float2bfloat16_rn(v[j] * sa[j] * sw);
                 }
             }
         }

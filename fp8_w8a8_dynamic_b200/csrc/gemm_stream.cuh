@@ -187,7 +187,6 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
     uint32_t* amax_loc = reinterpret_cast<uint32_t*>(smem + Smem::AMAX_OFF);
     float* sa_sm = reinterpret_cast<float*>(smem + Smem::SA_OFF);
     float* sw_sm = reinterpret_cast<float*>(smem + Smem::SW_OFF);
-    const float* recv = reinterpret_cast<const float*>(smem + Smem::RECV_OFF);
 
     const uint32_t warp = warp_id_sync();
     const uint32_t lane = lane_id();
@@ -531,12 +530,23 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
         }
         if (S == 1) {
             if (have_acc && m0 < M && n0 + c < N) {
-                const float sw = sw_sm[c];
+                // The scales are read before the stores, by shared-space
+                // address: a generic read after a global store waits for it.
+                const float sw = ld_shared_f32(smem_u32(sw_sm + c));
+                float sa[kCols];
+#pragma unroll
+                for (int mm = 0; mm < kCols; mm += 4) {
+                    const float4 v = ld_shared_f4(smem_u32(sa_sm + m0 + mm));
+                    sa[mm] = v.x;
+                    sa[mm + 1] = v.y;
+                    sa[mm + 2] = v.z;
+                    sa[mm + 3] = v.w;
+                }
 #pragma unroll
                 for (int mm = 0; mm < kCols; ++mm)
                     if (m0 + mm < M)
                         args.Y[int64_t(m0 + mm) * N + n0 + c] =
-                            __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa_sm[m0 + mm] * sw);
+                            __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa[mm] * sw);
             }
         } else {
             // Partial row of channel c to its owner: slot [rank][c % CPR],
@@ -566,29 +576,36 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const Args args) {
             }
             if (have_partials) {
                 // One thread per (channel, group of 4 tokens): a 16-byte read
-                // per rank, consecutive channels across the warp, so the Y
-                // stores of each token row are contiguous.
+                // per rank (all issued together), consecutive channels across
+                // the warp, so the Y stores of each token row are contiguous.
+                // Shared memory is read by shared-space address: a generic
+                // read after a global store would wait for the store.
                 const int G = (M + 3) / 4;
+                const uint32_t recv_base = sbase + uint32_t(Smem::RECV_OFF);
                 for (int e = t; e < CPR * G; e += kQuantThreads) {
                     const int cl = e % CPR, g = e / CPR;
                     const int n = n0 + rank * CPR + cl;
+                    const uint32_t slot = recv_base + uint32_t((cl * MMA_N + 4 * (g ^ recv_swz(cl))) * 4);
+                    float4 p[kMaxCluster];
+#pragma unroll
+                    for (int i = 0; i < kMaxCluster; ++i)
+                        if (i < S) p[i] = ld_shared_f4(slot + uint32_t(i * CPR * MMA_N * 4));
                     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int i = 0; i < S; ++i) {
-                        const float4 p = *reinterpret_cast<const float4*>(recv + (i * CPR + cl) * MMA_N +
-                                                                          4 * (g ^ recv_swz(cl)));
-                        sum.x += p.x;
-                        sum.y += p.y;
-                        sum.z += p.z;
-                        sum.w += p.w;
-                    }
+#pragma unroll
+                    for (int i = 0; i < kMaxCluster; ++i)
+                        if (i < S) {
+                            sum.x += p[i].x;
+                            sum.y += p[i].y;
+                            sum.z += p[i].z;
+                            sum.w += p[i].w;
+                        }
                     if (n < N) {
-                        const float sw = sw_sm[rank * CPR + cl];
-                        const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+                        const float sw = ld_shared_f32(smem_u32(sw_sm + rank * CPR + cl));
+                        const float4 sa = ld_shared_f4(smem_u32(sa_sm + 4 * g));
+                        const float v[4] = {sum.x * sa.x, sum.y * sa.y, sum.z * sa.z, sum.w * sa.w};
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            if (4 * g + j < M)
-                                args.Y[int64_t(4 * g + j) * N + n] =
-                                    __float2bfloat16_rn(v[j] * sa_sm[4 * g + j] * sw);
+                            if (4 * g + j < M) args.Y[int64_t(4 * g + j) * N + n] = __float2bfloat16_rn(v[j] * sw);
                     }
                 }
             }
