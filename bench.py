@@ -301,12 +301,13 @@ def kernel_times(torch, mfp8, layer, steps, warmup):
     return out
 
 
-def stack_sweep(torch, mfp8, W, device, steps, warmup, dist_ctx):
+def stack_sweep(torch, mfp8, W, device, steps, warmup, dist_ctx, Ms=None):
     """The 252-Linear stack (36 self-attention layers x 7 projections, weight
-    std jittered per layer, seed 4) swept at M in {1, 16, 128, 1024, 8192}:
-    one CUDA graph per M runs the 252 Linears in order.  One X buffer per
-    (M, K) and one Y buffer per (M, N) are reused across layers.  Weight-read
-    GB/s for M <= 128, TFLOP/s (quantize included) above."""
+    std jittered per layer, seed 4) swept at M in {1, 16, 128, 1024, 8192}
+    (or the M values in `Ms`): one CUDA graph per M runs the 252 Linears in
+    order.  One X buffer per (M, K) and one Y buffer per (M, N) are reused
+    across layers.  Weight-read GB/s for M <= 128, TFLOP/s (quantize
+    included) above."""
     seed = 4
     jitter = W.layer_std_jitter(seed, len(W.SELF_LAYERS))
     weights = []
@@ -320,7 +321,7 @@ def stack_sweep(torch, mfp8, W, device, steps, warmup, dist_ctx):
     out = {"workload": "252-Linear stack (36 self-attention layers x 7, ~7 GB of e4m3 weights, per-layer std "
                        "jitter +-20%), seed 4", "weight_bytes": wbytes,
            "rates": "per GPU (under torchrun every rank sweeps the same stack)", "by_M": {}}
-    for M in W.WORKLOADS[4]["Ms"]:
+    for M in (Ms or W.WORKLOADS[4]["Ms"]):
         xs = {K: W.make_x(M, K, seed=seed, stream=K, device=device) for K in {lin.K for lin, _, _ in weights}}
         ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=device) for N in {lin.N for lin, _, _ in weights}}
         ws = torch.zeros((max(16, max(mfp8.mfp8_linear_workspace_bytes(M, lin.N, lin.K) for lin, _, _ in weights)),),
@@ -540,6 +541,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-packed", action="store_true")
     ap.add_argument("--no-stack", action="store_true")
+    ap.add_argument("--stack-m", default=None, help="comma-separated M values for the stack sweep")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -648,7 +650,8 @@ def main():
 
     stack = None
     if not args.no_stack:
-        stack = stack_sweep(torch, mfp8, W, device, max(3, min(args.steps, 10)), args.warmup, ctx)
+        stack_ms = tuple(int(v) for v in args.stack_m.split(",")) if args.stack_m else None
+        stack = stack_sweep(torch, mfp8, W, device, max(3, min(args.steps, 10)), args.warmup, ctx, stack_ms)
 
     cpu = None
     if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
