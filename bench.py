@@ -114,6 +114,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(mhz)}
 
 
+# Clock-event reasons that rule a timed region out (power capping is kept
+# and reported).
+DISQUALIFYING_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def clocks_disqualify(summary, floor=0.85):
+    """True when a timed region's clock record rules its number out: a
+    hardware or thermal slowdown was active, or the median SM clock sat below
+    `floor` of its maximum with no reason active (a clock lock)."""
+    reasons = summary.get("reasons") or []
+    if any(r in reasons for r in DISQUALIFYING_REASONS):
+        return True
+    mhz, mx = summary.get("sm_mhz"), summary.get("sm_max_mhz")
+    return bool(mhz and mx and not reasons and mhz < floor * mx)
+
+
 # ------------------------------------------------------------- workload --
 
 class Layer:
@@ -564,8 +580,20 @@ def main():
     layer = Layer(torch, mfp8, W, seed=rank_seed(1, ctx.rank), weight_sets=3, Ms=DECODE_MS, device=device,
                   x_kind="normal")
     wbytes = layer.weight_bytes_per_step()
-    with ClockSampler(ctx.local_rank) as clocks:
-        ms = time_graph(torch, lambda h: layer.step(mfp8, h), args.steps, args.warmup, ctx)
+
+    def timed_decode():
+        with ClockSampler(ctx.local_rank) as clocks:
+            t = time_graph(torch, lambda h: layer.step(mfp8, h), args.steps, args.warmup, ctx)
+        return t, clocks.summary()
+
+    ms, clk = timed_decode()
+    # A region that saw a slowdown or a clock lock is measured once more.  The
+    # decision is the max over ranks, so that every rank takes the same
+    # barriers.
+    if ctx.max(1.0 if clocks_disqualify(clk) else 0.0) > 0:
+        first = clk
+        ms, clk = timed_decode()
+        clk["remeasured_after"] = {"sm_mhz": first["sm_mhz"], "reasons": first["reasons"]}
     assert mfp8.device_status() == mfp8.OK
     step_ms = ms / args.steps
     value = job_throughput(wbytes * args.steps, ctx.world, ms) / 1e9
@@ -678,7 +706,7 @@ def main():
                 "steps": e2e_steps, "copies": "double-buffered on copy streams (step i+1 up, step i-1 down, "
                                               "during step i); host wall clock"},
         "gpu_launches": launches,
-        "clocks": clocks.summary(),
+        "clocks": clk,
         "prefill": prefill,
         "long_video": video,
         "stack": stack,
