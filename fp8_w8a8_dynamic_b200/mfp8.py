@@ -186,8 +186,10 @@ def quantize_act(X, stream=None):
 
 
 def workspace_for(M, N, K, device):
-    """A zero-filled workspace for mfp8_linear at these sizes (the split-K
-    counters in it must start at zero; every call leaves them zero)."""
+    """A workspace for mfp8_linear at these sizes: room for the activation
+    codes and scales of the quantize pass (none below 17 tokens, where one
+    kernel quantizes on chip).  The kernels need no particular contents; it
+    is zero-filled only so that a fresh buffer is deterministic."""
     import torch
     nbytes = mfp8_linear_workspace_bytes(M, N, K)
     return torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=device)

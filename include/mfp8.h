@@ -121,7 +121,7 @@ typedef enum {
     MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
     MFP8_PATH_SPLITK = 2, /* quantize pass, then the split-K GEMM on CTA clusters, partials summed on chip (M <= 128) */
     MFP8_PATH_PAIR = 3,   /* quantize pass, then the 256-row-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
-    MFP8_PATH_FUSED = 4   /* one kernel: quantizes X on chip and streams the weights, whole K per CTA (M <= 16) */
+    MFP8_PATH_FUSED = 4   /* one kernel: quantizes X on chip and streams the weights, K split over a CTA cluster (M <= 16) */
 } mfp8_path;
 
 /* The kernel MFP8_PATH_AUTO takes at these sizes (FUSED for M <= 16, SPLITK
@@ -143,8 +143,9 @@ MFP8_API int mfp8_choose_path(int64_t M, int64_t N, int64_t K);
  * x_scale_out [M]; pass NULL for none).  Used to test each kernel on the
  * same shapes, to check that the activation bytes of every path are
  * bit-identical to mfp8_quantize_act, and by callers with static weights.
- * MFP8_PATH_FUSED is one launch that quantizes X on chip (every CTA takes
- * the row scales itself) and owns whole output channels, so it keeps
+ * MFP8_PATH_FUSED is one launch that quantizes X on chip (the CTAs of a
+ * cluster share their slice maxima, so each has the full row scales) and
+ * sums the K-split partial rows in the cluster's shared memory, so it keeps
  * nothing in the workspace (it may be NULL with 0 bytes).  When
  * X_fp8_out is given, the codes are written there as well (the quantize
  * pass writes them there instead of the workspace).  Returns MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel
