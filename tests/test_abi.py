@@ -137,3 +137,48 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mfp8, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         mfp8.lib()
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "mfp8.h"
+
+int main(void) {
+    /* every entry point is a plain C function */
+    typedef void (*fn_t)(void);
+    fn_t fns[] = {%s};
+    size_t n = sizeof fns / sizeof fns[0];
+    for (size_t i = 0; i < n; ++i)
+        if (!fns[i]) return 10;
+    if (mfp8_version() < 100) return 11;
+    if (mfp8_linear_workspace_bytes(300, 4096, 4096) != (size_t)300 * 4096 + 1280) return 12;
+    if (mfp8_choose_path(8, 4096, 4096) != MFP8_PATH_FUSED) return 13;
+    /* argument errors come back before any device work */
+    if (mfp8_linear(NULL, 4, 64, NULL, NULL, 64, NULL, NULL, 0, NULL) != MFP8_ERR_INVALID_ARG) return 14;
+    if (mfp8_linear_noalloc((void*)4096, 4, 64, (void*)8192, (float*)12288, 12, (void*)16384, NULL)
+        != MFP8_ERR_UNSUPPORTED_SHAPE) return 15;
+    printf("%%s\n", mfp8_status_string(MFP8_ERR_MISALIGNED));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """A C99 program (no C++, no CUDA headers) includes mfp8.h, takes the
+    address of every declared entry point, links against libmfp8.so and gets
+    the host-side answers and argument errors without a GPU."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_mfp8.c"
+    src.write_text(C_PROGRAM % ", ".join(f"(fn_t){n}" for n in declared_symbols()))
+    exe = tmp_path / "use_mfp8"
+    libdir = os.path.dirname(mfp8.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                    "-L", libdir, "-l:libmfp8.so", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out
+    assert out.stdout.strip() == mfp8.mfp8_status_string(mfp8.ERR_MISALIGNED)
