@@ -1,6 +1,7 @@
 """Host logic of bench.py that needs no GPU: the clock record of a timed
-region and the rule that rules a number out, and the committed figures the
-roofline line reads (DRAM traffic per launch, measured peaks)."""
+region and the rule that rules a number out, the committed figures the
+roofline line reads (DRAM traffic per launch, measured peaks), and the JSON
+line of the reference arm (the CPU oracle)."""
 import json
 import os
 import sys
@@ -77,3 +78,39 @@ def test_peaks_are_the_measured_ones_when_present():
         assert p["hbm_gbs"] > 1000 and p["bf16_tflops"] > 100
     else:
         assert p["source"] == "fallback"
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    """`bench.py --impl reference` prints one JSON line with the keys the
+    driver reads.  The oracle's timing is replaced by a fixed sample here; the
+    line's layout is what is checked."""
+    calls = []
+
+    def fake_sample(budget_s=12.0):
+        calls.append(budget_s)
+        return 1.25, 8, "21 Linears of the decode step, 2.0 s of CPU time"
+
+    monkeypatch.setattr(bench, "oracle_decode_sample", fake_sample)
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+    args = bench.argparse.Namespace(gpus=1, steps=4, warmup=3, impl="reference")
+    bench.run_reference(args)
+    line = capsys.readouterr().out.strip().splitlines()
+    assert len(line) == 1
+    out = json.loads(line[0])
+    assert len(calls) == 7  # warm-up and timed steps
+    assert out["impl"] == "reference" and out["value"] == 1.25 and out["steps"] == 4 and out["warmup"] == 3
+    for key in ("metric", "unit", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in out
+    assert out["cpu_baseline"] == {"value": 1.25, "unit": "GB/s", "cores": 8, "kind": "oracle",
+                                   "sample": "21 Linears of the decode step, 2.0 s of CPU time"}
+    assert out["e2e"] == {"value": 1.25, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert "workload" in out["config"]
+
+
+def test_reference_arm_is_rank_zero_only(monkeypatch, capsys):
+    monkeypatch.setattr(bench, "oracle_decode_sample", lambda budget_s=12.0: pytest.fail("rank 1 ran the oracle"))
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    bench.run_reference(bench.argparse.Namespace(gpus=2, steps=2, warmup=3, impl="reference"))
+    assert capsys.readouterr().out == ""
