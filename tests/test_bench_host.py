@@ -81,9 +81,9 @@ def test_peaks_are_the_measured_ones_when_present():
 
 
 def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
-    """`bench.py --impl reference` prints one JSON line with the keys the
-    driver reads.  The oracle's timing is replaced by a fixed sample here; the
-    line's layout is what is checked."""
+    """`bench.py --impl reference` prints one JSON line with the keys of the
+    benchmark line.  The oracle's timing is replaced by a fixed sample here;
+    the line's layout is what is checked."""
     calls = []
 
     def fake_sample(budget_s=12.0):
