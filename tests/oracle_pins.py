@@ -168,6 +168,83 @@ def pin_scale_invariants(o, seed=5):
     assert qt[0, 3] != 0 and qt[0, 5] != 0 and np.all(np.delete(qt[0], [3, 5]) == 0)
 
 
+def _ieee_scale(amax_f32):
+    """fl32(amax / 448) by numpy's IEEE fp32 divide (correctly rounded),
+    raised to FLT_MIN: the scale reading of the "MOSS-VL quantization README"
+    FP8-Dynamic recipe (per-channel / per-token scale = absmax / 448)."""
+    s = np.asarray(amax_f32, np.float32) / np.float32(448.0)
+    # the same quotient through an fp64 divide rounded once to fp32 (an fp32
+    # quotient rounded via fp64 is still correctly rounded: 53 >= 2*24 + 2)
+    assert np.array_equal(s, (np.asarray(amax_f32, np.float64) / 448.0).astype(np.float32))
+    return np.maximum(s, FLT_MIN).astype(np.float32)
+
+
+def _ieee_codes(x_f32, s_f32):
+    """e4m3(fl32(x / s)): numpy's fp32 divide, then the library encoder
+    (ml_dtypes, round to nearest even) after saturating to +-448."""
+    q = np.asarray(x_f32, np.float32) / np.asarray(s_f32, np.float32)
+    return lib_encode(np.clip(q, np.float32(-448.0), np.float32(448.0)))
+
+
+def _divide_sensitive_rows(rng, n_rows=48, K=24):
+    """bf16 rows chosen so that a plausible rounding slip changes the bytes:
+      - rows whose absmax a has fl32(a * fl32(1/448)) != fl32(a / 448), so a
+        scale taken by reciprocal multiplication differs from the divide's;
+      - rows holding values x with e4m3(fl32(x * fl32(1/s))) !=
+        e4m3(fl32(x / s)), so codes taken by reciprocal multiplication differ.
+    Both sets are found here by exhaustive numpy search over bf16 values."""
+    pos = np.arange(1, 0x7F80, dtype=np.uint32)                  # positive finite bf16
+    a_all = (pos << 16).view(np.float32)
+    s_rec = (a_all * (np.float32(1.0) / np.float32(448.0))).astype(np.float32)
+    scale_sensitive = pos[(a_all / np.float32(448.0)) != s_rec]
+    rows = np.zeros((n_rows, K), np.uint16)
+    r = 0
+    # half the rows: a scale-sensitive absmax (normal range) and smaller values
+    cand = scale_sensitive[(scale_sensitive > 0x0100) & (scale_sensitive < 0x7E00)]
+    for ab in rng.choice(cand, n_rows // 2, replace=False):
+        lo = rng.integers(0, ab, K - 1, dtype=np.uint32)
+        rows[r, 0] = ab
+        rows[r, 1:] = lo | (rng.integers(0, 2, K - 1, dtype=np.uint32) << 15)
+        r += 1
+    # the other half: values whose quotient sits where the reciprocal form
+    # rounds to a different code
+    for ab in rng.permutation(np.arange(0x3000, 0x5000, dtype=np.uint32)):
+        if r == n_rows:
+            break
+        a = np.array([ab << 16], np.uint32).view(np.float32)[0]
+        s = _ieee_scale(np.array([a], np.float32))[0]
+        xb = np.arange(0, ab + 1, dtype=np.uint32)
+        x = (xb << 16).view(np.float32)
+        d = _ieee_codes(x, s) != lib_encode(np.clip(x * (np.float32(1.0) / s), -448, 448))
+        hits = xb[d]
+        if hits.size == 0:
+            continue
+        take = hits[:K - 1]
+        rows[r, 0] = ab | 0x8000  # the absmax element, negative
+        rows[r, 1:1 + take.size] = take | (rng.integers(0, 2, take.size, dtype=np.uint32) << 15).astype(np.uint32)
+        r += 1
+    assert r == n_rows, "not enough divide-sensitive values found"
+    return rows
+
+
+def pin_scale_and_quotient_rounding(o, seed=12):
+    """Scales and codes equal, bit for bit, the IEEE fp32 divide forms
+    s = fl32(max|x| / 448) (floored at FLT_MIN) and q = e4m3(fl32(x / s)),
+    computed here by numpy and ml_dtypes alone, on random rows (every
+    magnitude range, tiny rows included) and on rows where a reciprocal
+    multiplication would round the scale or a code differently."""
+    rng = np.random.default_rng(seed)
+    xb = np.concatenate([_random_rows(rng, 32, 96, -140, 60), _divide_sensitive_rows(rng)[:, :24].repeat(4, 1)])
+    x = bits_to_f32(xb)
+    q, s = o.quantize_rows(xb)
+    s_exp = _ieee_scale(np.abs(x).max(axis=1))
+    assert np.array_equal(s.view(np.uint32), s_exp.view(np.uint32)), \
+        f"scales differ from fl32(amax / 448) in {(s != s_exp).sum()} rows"
+    q_exp = _ieee_codes(x, s_exp[:, None])
+    bad = np.argwhere(q != q_exp)
+    assert bad.size == 0, f"{bad.shape[0]} codes differ from e4m3(fl32(x / s)), first at {bad[0].tolist()}"
+
+
 # ------------------------------------------------------------------- GEMM --
 
 def pin_gemm_bruteforce(o, seed=3):
@@ -232,5 +309,5 @@ def pin_onehot_closed_form(o, seed=6):
 
 
 ALL_PINS = [pin_decode_table, pin_roundtrip, pin_rounding_cases, pin_encode_vs_library,
-            pin_saturation, pin_scale_invariants, pin_gemm_bruteforce, pin_gemm_int_vs_fp,
-            pin_onehot_closed_form]
+            pin_saturation, pin_scale_invariants, pin_scale_and_quotient_rounding, pin_gemm_bruteforce,
+            pin_gemm_int_vs_fp, pin_onehot_closed_form]

@@ -24,6 +24,12 @@ MUTANTS = {
     "scale_240": ("float s = amax / 448.0f;", "float s = amax / 240.0f;"),
     # multiply instead of divide when quantizing
     "mul_not_div": ("float q = orc_bf16_to_f32(row[k]) / sr;", "float q = orc_bf16_to_f32(row[k]) * sr;"),
+    # quotient by reciprocal multiplication: fl32(x * fl32(1/s)) rounds
+    # differently from fl32(x / s) for some x
+    "recip_mul": ("float q = orc_bf16_to_f32(row[k]) / sr;", "float q = orc_bf16_to_f32(row[k]) * (1.0f / sr);"),
+    # scale by reciprocal multiplication: fl32(a * fl32(1/448)) != fl32(a / 448)
+    # for about half the bf16 absmax values
+    "scale_recip": ("float s = amax / 448.0f;", "float s = amax * (1.0f / 448.0f);"),
     # sign of zero dropped
     "zero_sign": ("if (r == 0.0) return sign;", "if (r == 0.0) return 0;"),
     # transposed output index
