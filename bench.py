@@ -272,8 +272,9 @@ def kernel_times(torch, mfp8, layer, steps, warmup):
     launching stream; the average includes the gaps between graph nodes, so
     it is an upper bound on a launch's own time.  Where every Linear takes
     the one-kernel decode path (quantization on chip), the graph of the
-    step's launches is that kernel's graph.  The split-K workspaces are
-    zero-filled once (every call leaves their counters at zero)."""
+    step's launches is that kernel's graph.  The GEMMs run on codes
+    quantized once before the timing (mfp8_gemm); no kernel keeps anything in
+    a workspace."""
     keys = [(mi, M, i, lin) for mi, M in enumerate(layer.Ms) for i, lin in enumerate(layer.lins)]
     paths = sorted({mfp8.mfp8_choose_path(M, lin.N, lin.K) for (mi, M, i, lin) in keys})
     n = len(keys)
@@ -315,6 +316,65 @@ def kernel_times(torch, mfp8, layer, steps, warmup):
                             for (mi, M, i, lin) in keys) / n
     out["quant_bytes"] = sum(3 * M * lin.K + 4 * M for (mi, M, i, lin) in keys) / n
     return out
+
+
+def q_proj_m16(torch, mfp8, W, device, steps, warmup, dist_ctx, peaks):
+    """The single q_proj-shaped Linear at M = 16 (seed 0): 4096 -> 4096,
+    16.8 MB of e4m3 weights.  One weight set fits in L2, so the graph cycles
+    through 16 copies of it (268 MB, more than twice the 126 MB L2): every
+    call reads its weights from HBM.  Weight-read GB/s and the average
+    launch time of the one-kernel decode Linear."""
+    lin, M, copies = W.LAYER_LINEARS[0], 16, 16
+    x = W.make_x(M, lin.K, seed=0, stream=M, device=device)
+    w8, sw = mfp8.quantize_weight(W.make_w(lin.N, lin.K, seed=0, stream=lin.N, device=device))
+    w8s = [w8] + [w8.clone() for _ in range(copies - 1)]
+    y = torch.empty((M, lin.N), dtype=torch.bfloat16, device=device)
+    ws = mfp8.workspace_for(M, lin.N, lin.K, device)
+    torch.cuda.synchronize()
+    calls = [(x.data_ptr(), M, lin.K, c.data_ptr(), sw.data_ptr(), lin.N, y.data_ptr(), ws.data_ptr(), ws.numel(),
+              mfp8.PATH_AUTO, mfp8.FLAG_STATIC_WEIGHTS, None, None) for c in w8s]
+
+    def fn(h):
+        for a in calls:
+            st = mfp8.lib().mfp8_linear_ex(*a, h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_linear_ex")
+
+    ms = time_graph(torch, fn, steps, warmup, dist_ctx)
+    assert mfp8.device_status() == mfp8.OK
+    us = ms * 1e3 / (steps * copies)
+    wb = lin.N * lin.K + 4 * lin.N
+    gbs = wb / (us * 1e-6) / 1e9
+    return {"workload": "q_proj 4096->4096 at M=16, X ~N(0,1) + 0.1% x50 outliers, W ~N(0,0.02), seed 0; "
+                        f"{copies} rotated weight copies ({copies * wb / 1e6:.0f} MB, > 2x L2)",
+            "value": round(gbs * dist_ctx.world, 1), "unit": "GB/s", "avg_launch_us": round(us, 3),
+            "kernel": mfp8.KERNEL_OF_PATH[mfp8.mfp8_choose_path(M, lin.N, lin.K)],
+            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "all_bytes_per_launch": wb + 2 * M * lin.K + 2 * M * lin.N}
+
+
+def fp8_ceiling_tflops(torch, device, n=8192, reps=10):
+    """The box's dense e4m3 GEMM ceiling, as a denominator only: cuBLASLt
+    through torch._scaled_mm on n x n x n, bf16 out, best of `reps` launches
+    timed alone with CUDA events after warm-up."""
+    g = torch.Generator(device=device).manual_seed(0)
+    a = torch.randn(n, n, device=device, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=device, generator=g).to(torch.float8_e4m3fn).t()  # column-major operand
+    one = torch.ones((), device=device, dtype=torch.float32)
+    for _ in range(3):
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1)
+        best = t if best is None else min(best, t)
+    del a, b
+    torch.cuda.empty_cache()
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
 def stack_sweep(torch, mfp8, W, device, steps, warmup, dist_ctx, Ms=None):
@@ -645,9 +705,15 @@ def main():
         pk = kernel_times(torch, mfp8, pl, steps=5, warmup=args.warmup)
         g_tf = pk["gemm_flops"] / (pk["gemm_us"] * 1e-6) / 1e12
         fp8_peak = 2.0 * peaks["bf16_tflops"]
+        fp8_ceiling = fp8_ceiling_tflops(torch, device)
         prefill = {"metric": "FP8-dynamic Linear TFLOPS (M=2048, 7 Linears, quantize included)",
                    "value": round(tflops, 1), "unit": "TFLOP/s", "ms_per_step": round(pms / psteps, 4),
                    "frac_of_fp8_peak": round(tflops / ctx.world / fp8_peak, 4),
+                   "fp8_ceiling": {"value": round(fp8_ceiling, 1), "unit": "TFLOP/s",
+                                   "how": "cuBLASLt e4m3 8192^3 via torch._scaled_mm, bf16 out, best of 10, "
+                                          "timed alone in this run (a denominator only)",
+                                   "frac_end_to_end": round(tflops / ctx.world / fp8_ceiling, 4),
+                                   "frac_gemms": round(g_tf / fp8_ceiling, 4)},
                    "roofline": {"bound": "tensor", "achieved": round(g_tf, 1), "peak": round(fp8_peak, 1),
                                 "unit": "TFLOP/s", "frac": round(g_tf / fp8_peak, 4),
                                 # DRAM bytes per launch of the pair kernel, which runs 5 of
@@ -675,6 +741,10 @@ def main():
                                            / (2.0 * peaks["bf16_tflops"]), 4)}
         del vl
         torch.cuda.empty_cache()
+
+    # The single q_proj Linear at M = 16 (seed 0), weights rotated past L2.
+    config0 = q_proj_m16(torch, mfp8, W, device, max(5, args.steps), args.warmup, ctx, peaks)
+    torch.cuda.empty_cache()
 
     stack = None
     if not args.no_stack:
@@ -707,6 +777,7 @@ def main():
                                               "during step i); host wall clock"},
         "gpu_launches": launches,
         "clocks": clk,
+        "q_proj_m16": config0,
         "prefill": prefill,
         "long_video": video,
         "stack": stack,

@@ -615,20 +615,61 @@ int sm_count_for_sizing() {
 constexpr size_t kStaticWsBytes = MFP8_STATIC_WORKSPACE_BYTES;
 static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
 
-void* g_static_ws_ptr[kMaxDevices] = {};
+// The array's device address, looked up once per device and context.  In
+// host code `g_static_ws` names a host-side stand-in, not device memory; the
+// address kernels need comes from cudaGetSymbolAddress with the device
+// current.  It is cached together with the context's unique ID: a context
+// that was destroyed and created again (cudaDeviceReset) reloads the module,
+// which may place the array elsewhere, and the new ID forces a new lookup.
+struct StaticWs {
+    unsigned long long ctx_id = 0;
+    void* ptr = nullptr;
+};
+StaticWs g_static_ws_cache[kMaxDevices];
+PFN_cuCtxGetCurrent_v4000 g_ctx_get_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_get_id = nullptr;
 
-// Once per device: the array's device address.
+// Unique ID of the calling thread's current context (0 when none is bound).
+mfp8_status current_context_id(unsigned long long* id) {
+    if (!g_ctx_get_current || !g_ctx_get_id) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2) {
+            cudaGetLastError();
+            return MFP8_ERR_CUDA;
+        }
+        g_ctx_get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+        g_ctx_get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return MFP8_ERR_CUDA;
+    *id = 0;
+    if (ctx && g_ctx_get_id(ctx, id) != CUDA_SUCCESS) return MFP8_ERR_CUDA;
+    return MFP8_OK;
+}
+
 mfp8_status static_workspace(int dev, void** out) {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_static_ws_ptr[dev]) {
+    unsigned long long id = 0;
+    mfp8_status st = current_context_id(&id);
+    if (st != MFP8_OK) return st;
+    StaticWs& c = g_static_ws_cache[dev];
+    if (id == 0 || c.ptr == nullptr || c.ctx_id != id) {
+        // cudaGetSymbolAddress also binds the device's primary context to
+        // this thread if none was bound yet; the ID is read after it.
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) {
             cudaGetLastError();
             return MFP8_ERR_CUDA;
         }
-        g_static_ws_ptr[dev] = p;
+        if ((st = current_context_id(&id)) != MFP8_OK) return st;
+        c.ptr = p;
+        c.ctx_id = id;
     }
-    *out = g_static_ws_ptr[dev];
+    *out = c.ptr;
     return MFP8_OK;
 }
 

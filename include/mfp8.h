@@ -170,7 +170,9 @@ MFP8_API mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K,
  *   MFP8_STATIC_WORKSPACE_BYTES are rejected with MFP8_ERR_WORKSPACE before
  *   any device work (the quantized activations need about M * K bytes:
  *   every projection up to K = 12288 fits for M <= 1300).
- *   Set-up: the first call on each device looks up the array's address.
+ *   Set-up: the first call on each device (and again after the device's
+ *   context was reset) looks up the array's address; that first call should
+ *   come before any stream capture.
  *   Concurrency: every call on a device shares the one scratch array.  Calls
  *   that may be in flight at the same time (different streams, or host
  *   threads) race and give wrong results; serialise them, e.g. on one stream. */

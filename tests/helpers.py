@@ -41,3 +41,13 @@ def assert_linear_parity(y_gpu: torch.Tensor, x8: np.ndarray, s_a: np.ndarray, w
             f"{what}: {bad.shape[0]} of {ok.size} outputs outside tolerance; first at (row {m}, col {n}): "
             f"gpu {y[m, n]!r} ref {y_ref[m, n]!r} s_abs {s_abs[m, n]!r}")
     assert np.isfinite(y).all()
+
+
+def rows_in_every_tile(M, tile=256, seed=0):
+    """One random row in every `tile`-row block of M rows, plus rows 0 and
+    M - 1, sorted."""
+    rng = np.random.default_rng(seed)
+    starts = np.arange(0, M, tile)
+    picks = starts + rng.integers(0, tile, starts.size)
+    picks = np.minimum(picks, M - 1)
+    return np.union1d(picks, [0, M - 1])

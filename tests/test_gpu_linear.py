@@ -10,7 +10,7 @@ import torch
 import oracle
 from fp8_w8a8_dynamic_b200 import mfp8
 from fp8_w8a8_dynamic_b200 import workloads as W
-from helpers import assert_linear_parity, bits16, f32, u8
+from helpers import assert_linear_parity, bits16, f32, rows_in_every_tile, u8
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -263,6 +263,13 @@ def sampled_rows(M, n=48, seed=0):
     return np.array(sorted(r))
 
 
+def rows_per_tile(M, tile=256, seed=0):
+    """One random row in every `tile`-row block of M (the 256-row tiles of
+    the CTA-pair kernel, so every tile and every lap of its persistent
+    schedule meets the oracle), plus the first and last rows."""
+    return rows_in_every_tile(M, tile, seed)
+
+
 @pytest.mark.parametrize("lin", W.LAYER_LINEARS, ids=lambda l: l.name)
 @pytest.mark.parametrize("path", [mfp8.PATH_AUTO, mfp8.PATH_FUSED])
 def test_decode_layer_full_size(lin, path):
@@ -275,13 +282,16 @@ def test_decode_layer_full_size(lin, path):
 def test_prefill_layer_full_size_sampled(lin):
     """Prefill M=2048: every code and scale, sampled output rows."""
     M = 2048
-    run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=2, kind="rowscale", rows=sampled_rows(M, 32, lin.N))
+    run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=2, kind="rowscale",
+             rows=np.union1d(sampled_rows(M, 16, lin.N), rows_per_tile(M, seed=lin.N)))
 
 
 @pytest.mark.parametrize("lin", W.MLP_LINEARS, ids=lambda l: l.name)
 def test_long_video_full_size_sampled(lin):
+    """M = 16384: every code and scale, and one output row in each of the 64
+    row tiles."""
     M = 16384
-    run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=3, kind="rowscale", rows=sampled_rows(M, 16, lin.K))
+    run_case(M, lin.N, lin.K, mfp8.PATH_AUTO, seed=3, kind="rowscale", rows=rows_per_tile(M, seed=lin.K))
 
 
 def test_workspace_reused_across_calls_and_shapes():
@@ -300,3 +310,56 @@ def test_workspace_reused_across_calls_and_shapes():
         x8_ref, xs_ref = oracle.quantize_rows(bits16(x))
         assert_linear_parity(y, x8_ref, xs_ref, u8(W8), f32(sw), what=f"reuse {i}")
     assert mfp8.device_status() == mfp8.OK
+
+
+# ------------------------------------------------------ packed projections --
+
+PACKS = {"qkv_proj": W.LAYER_LINEARS[0:3], "gate_up_proj": W.LAYER_LINEARS[4:6]}
+
+
+@pytest.mark.parametrize("pack", sorted(PACKS))
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 64, 2048])
+def test_packed_projection_equals_the_separate_ones(pack, M):
+    """The README's packed modules (qkv_proj, gate_up_proj) are exact under
+    per-channel weight scales: quantizing the stacked weight rows gives the
+    stacked codes and scales, the activation codes and scales are those of
+    the separate calls, and each block of the packed output is the separate
+    projection's output.  Where the kernel sums K in the same order for
+    both (the tile kernels at M = 2048) the blocks are equal bit for bit;
+    the split-K kernels choose their K split from N, so there the blocks are
+    each within tolerance of the oracle."""
+    parts = PACKS[pack]
+    K = parts[0].K
+    ws = [W.make_w(p.N, K, seed=5, stream=i, device=DEV) for i, p in enumerate(parts)]
+    q = [mfp8.quantize_weight(w) for w in ws]
+    W8p, swp = mfp8.quantize_weight(torch.cat(ws, 0))
+    torch.cuda.synchronize()
+    assert torch.equal(W8p, torch.cat([a for a, _ in q], 0))
+    assert torch.equal(swp.view(torch.int32), torch.cat([b for _, b in q], 0).view(torch.int32))
+    x = W.make_x(M, K, seed=5, stream=M, kind="rowscale", device=DEV)
+    paths = [mfp8.PATH_AUTO] + ([mfp8.PATH_PAIR, mfp8.PATH_TILED] if M >= 256 else [])
+    rows = rows_per_tile(M, seed=M) if M > 64 else None
+    x8_ref, xs_ref = oracle.quantize_rows(bits16(x))
+    for path in paths:
+        def run(W8, sw):
+            x8 = torch.empty((M, K), dtype=torch.uint8, device=DEV)
+            xs = torch.empty((M,), dtype=torch.float32, device=DEV)
+            y = mfp8.linear(x, W8, sw, path=path, x8_out=x8, xs_out=xs, flags=mfp8.FLAG_STATIC_WEIGHTS)
+            return y, x8, xs
+        yp, x8p, xsp = run(W8p, swp)
+        sep = [run(a, b) for a, b in q]
+        torch.cuda.synchronize()
+        assert mfp8.device_status() == mfp8.OK
+        assert np.array_equal(u8(x8p), x8_ref) and np.array_equal(f32(xsp).view(np.uint32), xs_ref.view(np.uint32))
+        off = 0
+        for p, (a, b), (y, x8, xs) in zip(parts, q, sep):
+            assert torch.equal(x8, x8p) and torch.equal(xs.view(torch.int32), xsp.view(torch.int32))
+            blk = yp[:, off:off + p.N]
+            if path in (mfp8.PATH_PAIR, mfp8.PATH_TILED):
+                assert torch.equal(blk.contiguous().view(torch.int16), y.view(torch.int16)), \
+                    f"{pack} M={M} path={path}: block {p.name} differs from the separate call"
+            else:
+                assert_linear_parity(blk.contiguous(), x8_ref, xs_ref, u8(a), f32(b), rows=rows,
+                                     what=f"{pack} block {p.name} M={M}")
+                assert_linear_parity(y, x8_ref, xs_ref, u8(a), f32(b), rows=rows, what=f"{p.name} M={M}")
+            off += p.N

@@ -15,7 +15,7 @@ import torch
 import oracle
 from fp8_w8a8_dynamic_b200 import mfp8
 from fp8_w8a8_dynamic_b200 import workloads as W
-from helpers import assert_linear_parity, bits16, f32, u8
+from helpers import assert_linear_parity, bits16, f32, rows_in_every_tile, u8
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -44,6 +44,10 @@ def test_stack_layers_at_every_m(M):
             x8_ref, xs_ref = oracle.quantize_rows(bits16(x))
             assert np.array_equal(u8(x8), x8_ref), f"layer {W.SELF_LAYERS[li]} {lin.name} M={M}: codes"
             assert np.array_equal(f32(xs).view(np.uint32), xs_ref.view(np.uint32))
-            rows = None if M <= 128 else np.unique(np.concatenate([[0, M - 1], rng.choice(M, 14, replace=False)]))
+            # every output row up to M = 128; above, one row in each row tile
+            # of the kernel that runs (128 rows at M = 1024, the CTA-pair
+            # kernel's 256 at M = 8192: every tile and persistent lap)
+            rows = None if M <= 128 else rows_in_every_tile(M, 128 if M <= 1024 else 256,
+                                                            seed=int(rng.integers(1 << 30)))
             assert_linear_parity(y, x8_ref, xs_ref, w8_ref, sw_ref, rows=rows,
                                  what=f"layer {W.SELF_LAYERS[li]} {lin.name} M={M}")
