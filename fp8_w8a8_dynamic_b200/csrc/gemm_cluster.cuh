@@ -1,4 +1,4 @@
-// gemm_cluster.cuh — the FP8 GEMM for small and middle M (up to 128 token
+// gemm_cluster.cuh — the FP8 GEMM for small and middle M (up to 256 token
 // rows) on activation codes already quantized (the quantize pass of
 // mfp8_linear, or the caller's codes in mfp8_gemm):
 //
@@ -20,12 +20,16 @@
 //     weights before the dependency wait when they are static;
 //   - one thread issues 4 MMAs per K block;
 //   - with S > 1, once every CTA of the cluster has its accumulator (a
-//     cluster barrier), each channel's partial row goes with plain remote
-//     stores to the CTA that owns the channel, into that CTA's ring (free by
-//     then), followed by one releasing arrival on the owner's barrier; the
-//     owner adds the S partials in rank order (deterministic), scales and
-//     stores BF16.  With S = 1 the epilogue stores directly.
-// About 98 KB of shared memory and at most 128 TMEM columns, so two CTAs
+//     cluster barrier), the partial rows are exchanged in rounds of TC
+//     token columns: each CTA copies its accumulator columns from TMEM into
+//     its own ring (free by then), one slot per owning rank (rank r owns
+//     128/S of the channels), and one thread sends each slot to its owner
+//     with a single bulk shared-memory copy across the cluster, counted on
+//     the owner's barrier; the owner adds the S partials in rank order
+//     (deterministic), scales and stores BF16; a cluster barrier ends the
+//     round, after which the slots are reused.  With S = 1 the epilogue
+//     stores directly.
+// About 98 KB of shared memory and at most 256 TMEM columns, so two CTAs
 // fit on an SM and the next kernel's CTAs can start alongside.
 //
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA
@@ -47,7 +51,7 @@ constexpr int kThreads = 192;
 constexpr int TILE = 128;                   // output channels per cluster (MMA M)
 constexpr int SUB = 128;                    // K bytes per block: swizzle atom, TMA box width
 constexpr int MMA_K = 32;
-constexpr int kMaxM = 128;                  // token rows (MMA N up to 128)
+constexpr int kMaxM = 256;                  // token rows (MMA N up to 256)
 constexpr int kMaxCluster = 8;
 constexpr int kMaxStages = 8;
 constexpr int kWBlockBytes = TILE * SUB;    // one weight K block of the tile: 16 KB
@@ -60,17 +64,26 @@ struct Geometry {
     int S;       // CTAs per cluster (K split)
     int mp;      // token columns of the MMA: M rounded up to 16
     int stages;  // ring depth; a stage is a weight block and a code block
+    int tc;      // token columns per exchange round (S > 1): a multiple of 16, <= mp
 };
 
 __host__ __device__ constexpr int stage_bytes(int mp) { return kWBlockBytes + mp * SUB; }
 
-__host__ __device__ constexpr uint32_t tmem_cols(int mp) { return mp <= 32 ? 32u : mp <= 64 ? 64u : 128u; }
+__host__ __device__ constexpr uint32_t tmem_cols(int mp) {
+    return mp <= 32 ? 32u : mp <= 64 ? 64u : mp <= 128 ? 128u : 256u;
+}
+
+// Ring bytes one exchange round of tc token columns takes (S > 1): the
+// receive slots [S][128/S][tc] fp32 of the channels this CTA owns, then the
+// send slots [S-1][128/S][tc] fp32 of the channels the other ranks own.
+__host__ __device__ constexpr int exchange_bytes(int S, int tc) {
+    return (TILE * tc * 4 / S) * (2 * S - 1);
+}
 
 // Shared memory, from a 1024-byte aligned base:
 //   [ring] kRingBytes: stage s at s * stage_bytes(mp) (weights, then codes);
-//          with S > 1 it later receives the partial rows this CTA owns,
-//          [S][128/S][mp] fp32 (at most 64 KB)
-//   [sa] [128] f32, [sw] [128] f32, barriers, TMEM base and abort flag
+//          with S > 1 it later holds the exchange slots (exchange_bytes)
+//   [sa] [256] f32, [sw] [128] f32, barriers, TMEM base and abort flag
 struct Smem {
     static constexpr int SA_OFF = kRingBytes;
     static constexpr int SW_OFF = SA_OFF + kMaxM * 4;
@@ -80,7 +93,7 @@ struct Smem {
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int USED = MISC_OFF + 16;
     static constexpr int BYTES = USED + 1024;  // alignment slack
-    static_assert(TILE * kMaxM * 4 <= kRingBytes, "partial rows fit in the ring");
+    static_assert(exchange_bytes(2, 16) <= kRingBytes, "one round of the narrowest exchange fits in the ring");
     static_assert(kMinStages * stage_bytes(kMaxM) <= kRingBytes, "ring room");
 };
 
@@ -93,12 +106,13 @@ struct Args {
     Geometry g;
 };
 
-// Position of 16-byte token group g of a partial row in the receive slot of
-// channel cl: g ^ swz(cl), so that the owner's 16-byte reads of one group
-// across consecutive channels hit distinct banks.  A slot has mp / 4 groups
-// (a multiple of 4); the XOR stays inside an aligned run of 8 groups when
-// mp is a multiple of 32, of 4 otherwise.
-__device__ __forceinline__ int recv_swz(int cl, int mp) { return (mp & 31) == 0 ? (cl & 7) : ((cl >> 1) & 3); }
+// Position of 16-byte token group g in channel cl's row of an exchange slot
+// (tc token columns, tc / 4 groups, a multiple of 4): g ^ swz(cl), so that
+// 16-byte accesses of one group across consecutive channels (the TMEM
+// copy-out, one channel per thread, and the owner's sum) hit distinct banks.
+// The XOR stays inside an aligned run of 8 groups when tc is a multiple of
+// 32, of 4 otherwise.
+__device__ __forceinline__ int recv_swz(int cl, int tc) { return (tc & 31) == 0 ? (cl & 7) : ((cl >> 1) & 3); }
 
 __global__ void __launch_bounds__(kThreads, 2)
 gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -138,12 +152,13 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(tfull_bar, 1);
-        // (S > 1) one arrival from each thread, in every CTA, whose channel
-        // this CTA owns: S ranks x 128/S channels
-        mbar_init(rbar, S > 1 ? TILE : 1);
+        // (S > 1) each round, the S - 1 slots sent to this CTA: one arrival
+        // (this thread's, below and at the end of each round) and the bytes
+        mbar_init(rbar, 1);
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
+        if (S > 1) mbar_arrive_expect_tx(rbar, uint32_t((S - 1) * CPR * args.g.tc * 4));
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
     }
@@ -248,7 +263,7 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const int t = int(threadIdx.x) - 64;  // 0..127
         sw_sm[t] = (n0 + t < N) ? __ldg(args.s_w + n0 + t) : 0.f;
         grid_dependency_wait();  // s_a comes from the quantize pass
-        sa_sm[t] = t < M ? __ldg(args.s_a + t) : 0.f;
+        for (int m = t; m < kMaxM; m += 128) sa_sm[m] = m < M ? __ldg(args.s_a + m) : 0.f;
         have_acc = mbar_wait(tfull_bar, 0, abort_flag);
         named_bar_sync(1, 128);  // sa_sm, sw_sm complete
     }
@@ -263,13 +278,12 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         tc_fence_after();
     }
 
-    if (warp >= 2) {
-        // -------------------------------------------- epilogue, part 2 --
-        const int t = int(threadIdx.x) - 64;
-        const int q = int(warp & 3u);       // TMEM lane quarter of this warp
-        const int c = q * 32 + int(lane);  // channel within the tile
-        if (have_acc) tc_fence_after();
-        if (S == 1) {
+    if (S == 1) {
+        if (warp >= 2) {
+            // -------------------------------------- epilogue, one CTA --
+            const int q = int(warp & 3u);       // TMEM lane quarter of this warp
+            const int c = q * 32 + int(lane);  // channel within the tile
+            if (have_acc) tc_fence_after();
             for (int c0 = 0; c0 < MP && have_acc; c0 += 16) {
                 uint32_t acc[16];
                 tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(c0), acc);
@@ -293,82 +307,117 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                                 __float2bfloat16_rn(__uint_as_float(acc[mm]) * sa[mm] * sw);
                 }
             }
-        } else {
-            // Partial row of channel c to its owner: slot [rank][c % CPR],
-            // MP token columns in 16-byte groups, group g at position
-            // g ^ recv_swz(c % CPR).  Plain remote stores, then one arrival
-            // on the owner's barrier that releases them (per-store
-            // transaction counting made each store a round trip).
-            const int owner = c / CPR;
-            const int cl = c % CPR;
-            const int swz = recv_swz(cl, MP);
-            const uint32_t local = sbase + uint32_t(((rank * CPR + cl) * MP) * 4);
-            const uint32_t dst = mapa_shared(local, uint32_t(owner));
-            const uint32_t bar = mapa_shared(rbar, uint32_t(owner));
-            for (int c0 = 0; c0 < MP && have_acc; c0 += 16) {
-                uint32_t acc[16];
-                tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(c0), acc);
-                tmem_wait_ld();
+        }
+    } else {
+        // ---------------------------------- partial-row exchange, S > 1 --
+        // Rounds of TC token columns.  Slot layout (fp32): receive slot s =
+        // partials from rank s of the 128/S channels this CTA owns, at
+        // s * SLOT; send slot of owner o != rank at (S + o') * SLOT, o' = o
+        // or o - 1 (this rank's own slot is written straight into receive
+        // slot `rank`).  A slot row is one channel's TC columns in 16-byte
+        // groups, group g at position g ^ recv_swz(channel, TC).  Every warp
+        // takes part in the round's closing cluster barrier.
+        const int TC = args.g.tc;
+        const int rounds = (MP + TC - 1) / TC;
+        const uint32_t SLOT = uint32_t(CPR * TC * 4);
+        const uint32_t row_bytes = uint32_t(TC * 4);
+        for (int j = 0; j < rounds; ++j) {
+            const int tok0 = j * TC;
+            const int tcj = MP - tok0 < TC ? MP - tok0 : TC;  // columns this round (a multiple of 16)
+            if (warp >= 2) {
+                const int t = int(threadIdx.x) - 64;
+                const int q = int(warp & 3u);
+                const int c = q * 32 + int(lane);
+                const int o = c / CPR, cl = c % CPR;
+                const int swz = recv_swz(cl, TC);
+                const uint32_t slot = o == rank ? uint32_t(rank) * SLOT : uint32_t(S + (o < rank ? o : o - 1)) * SLOT;
+                const uint32_t row = sbase + slot + uint32_t(cl) * row_bytes;
+                if (have_acc) {
+                    if (j == 0) tc_fence_after();
+                    for (int c0 = 0; c0 < tcj; c0 += 16) {
+                        uint32_t acc[16];
+                        tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(tok0 + c0), acc);
+                        tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int g = c0 / 4 + h;
-                    st_cluster_v4(dst + 16u * uint32_t(g ^ swz),
-                                  make_uint4(acc[4 * h], acc[4 * h + 1], acc[4 * h + 2], acc[4 * h + 3]));
+                        for (int h = 0; h < 4; ++h)
+                            st_shared_v4(row + 16u * uint32_t((c0 / 4 + h) ^ swz), acc[4 * h], acc[4 * h + 1],
+                                         acc[4 * h + 2], acc[4 * h + 3]);
+                    }
                 }
-            }
-            if (have_acc) mbar_arrive_remote_release(bar);
-            // Sum the S partials of the channels this rank owns, in rank order.
-            const bool have_partials = mbar_wait_cluster(rbar, 0, abort_flag);
-            if (!have_partials && t == 0) {
-                volatile int no_abort = 0;
-                mbar_wait_cluster(rbar, 0, &no_abort, 20000000ull);
-            }
-            if (have_partials) {
-                // One thread per (channel, group of 4 tokens): a 16-byte read
-                // per rank (all S issued together), consecutive channels
-                // across the warp, so the Y stores of each token row are
-                // contiguous.  Thread t keeps channel t % CPR and walks the
-                // groups t / CPR, t / CPR + 128 / CPR, ...
-                // Shared memory is read by shared-space address (ld_shared_*)
-                // so that the reads are not ordered behind the Y stores.
-                const int G = (M + 3) / 4;
-                const int cl2 = t % CPR;
-                const int n = n0 + rank * CPR + cl2;
-                const float sw = ld_shared_f32(smem_u32(sw_sm + rank * CPR + cl2));
-                const int swz2 = recv_swz(cl2, MP);
-                const uint32_t base = sbase + uint32_t(cl2 * MP * 4);
-                const uint32_t sa_base = smem_u32(sa_sm);
-                for (int g = t / CPR; g < G && n < N; g += 128 / CPR) {
-                    const int pos = g ^ swz2;
-                    float4 p[kMaxCluster];
-#pragma unroll
-                    for (int i = 0; i < kMaxCluster; ++i)
-                        if (i < S) p[i] = ld_shared_f4(base + uint32_t((i * CPR * MP + 4 * pos) * 4));
-                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int i = 0; i < kMaxCluster; ++i)
-                        if (i < S) {
-                            sum.x += p[i].x;
-                            sum.y += p[i].y;
-                            sum.z += p[i].z;
-                            sum.w += p[i].w;
-                        }
-                    const float v[4] = {sum.x, sum.y, sum.z, sum.w};
-                    const float4 sa4 = ld_shared_f4(sa_base + uint32_t(16 * g));
-                    const float sa[4] = {sa4.x, sa4.y, sa4.z, sa4.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        if (4 * g + j < M)
-                            args.Y[int64_t(4 * g + j) * N + n] = __float2bfloat16_rn(v[j] * sa[j] * sw);
+                fence_proxy_async_smem();  // slot writes -> the bulk copies' reads
+                named_bar_sync(1, 128);
+                if (t == 0 && have_acc) {
+                    for (int o2 = 0; o2 < S; ++o2) {
+                        if (o2 == rank) continue;
+                        const uint32_t src = sbase + uint32_t(S + (o2 < rank ? o2 : o2 - 1)) * SLOT;
+                        bulk_copy_to_cluster(mapa_shared(sbase + uint32_t(rank) * SLOT, uint32_t(o2)), src, SLOT,
+                                             mapa_shared(rbar, uint32_t(o2)));
+                    }
                 }
+                // Sum the S partials of the channels this rank owns, in rank
+                // order, for this round's token columns.
+                const bool have_partials = mbar_wait_cluster(rbar, uint32_t(j & 1), abort_flag);
+                if (!have_partials && t == 0) {
+                    volatile int no_abort = 0;
+                    mbar_wait_cluster(rbar, uint32_t(j & 1), &no_abort, 20000000ull);
+                }
+                // Rows of this round that exist: M - tok0 (when positive).
+                const int mj = M - tok0 < tcj ? M - tok0 : tcj;
+                if (have_partials && mj > 0) {
+                    // One thread per (channel, group of 4 tokens): a 16-byte
+                    // read per rank (all S issued together), consecutive
+                    // channels across the warp, so the Y stores of each token
+                    // row are contiguous.  Shared memory is read by
+                    // shared-space address (ld_shared_*) so that the reads are
+                    // not ordered behind the Y stores.
+                    const int G = (mj + 3) / 4;
+                    const int cl2 = t % CPR;
+                    const int n = n0 + rank * CPR + cl2;
+                    const float sw = ld_shared_f32(smem_u32(sw_sm + rank * CPR + cl2));
+                    const int swz2 = recv_swz(cl2, TC);
+                    const uint32_t base = sbase + uint32_t(cl2) * row_bytes;
+                    const uint32_t sa_base = smem_u32(sa_sm + tok0);
+                    for (int g = t / CPR; g < G && n < N; g += 128 / CPR) {
+                        const uint32_t pos = 16u * uint32_t(g ^ swz2);
+                        float4 p[kMaxCluster];
+#pragma unroll
+                        for (int i = 0; i < kMaxCluster; ++i)
+                            if (i < S) p[i] = ld_shared_f4(base + uint32_t(i) * SLOT + pos);
+                        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int i = 0; i < kMaxCluster; ++i)
+                            if (i < S) {
+                                sum.x += p[i].x;
+                                sum.y += p[i].y;
+                                sum.z += p[i].z;
+                                sum.w += p[i].w;
+                            }
+                        const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+                        const float4 sa4 = ld_shared_f4(sa_base + uint32_t(16 * g));
+                        const float sa[4] = {sa4.x, sa4.y, sa4.z, sa4.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if (4 * g + i < mj)
+                                args.Y[int64_t(tok0 + 4 * g + i) * N + n] = __float2bfloat16_rn(v[i] * sa[i] * sw);
+                    }
+                }
+                // Arm the barrier for the next round's slots before any rank
+                // can send them (they go only after the cluster barrier below).
+                if (t == 0 && j + 1 < rounds) mbar_arrive_expect_tx(rbar, (uint32_t(S) - 1u) * SLOT);
             }
+            // Every slot sent this round has landed (each owner waited for its
+            // own) and been summed: the slots are free, and after the last
+            // round no copy is in flight from or into this CTA.
+            __syncwarp();
+            cluster_arrive_release();
+            cluster_wait_acquire();
         }
     }
 
-    // A CTA receives remote stores only into its own ring after the cluster
-    // barrier above, and has waited for all of them (the senders' releasing
-    // arrivals on rbar) before it gets here.  After a timeout the waiting thread gave the late bytes a second
-    // bounded wait.
+    // With S > 1 a CTA receives bulk copies only into its own ring, after the
+    // cluster barrier above, and every copy from or into it completed before
+    // the last round's cluster barrier.  After a timeout the waiting thread
+    // gave the late bytes a second bounded wait.
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

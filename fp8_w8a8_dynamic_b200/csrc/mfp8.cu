@@ -534,6 +534,18 @@ bool cluster_geometry(int64_t M, int64_t N, int64_t K, int sm_count, cluster::Ge
     g->mp = int((M + 15) / 16 * 16);
     const int st = cluster::kRingBytes / cluster::stage_bytes(g->mp);
     g->stages = st > cluster::kMaxStages ? cluster::kMaxStages : st;
+    // Exchange rounds: as few as the ring allows, of equal width (a multiple
+    // of 32 token columns where the round is that wide, else of 16).
+    g->tc = g->mp;
+    if (S > 1) {
+        int rounds = 1;
+        auto width = [&](int r) {
+            const int w = (g->mp + r - 1) / r;
+            return w > 16 ? (w + 31) / 32 * 32 : 16;
+        };
+        while (cluster::exchange_bytes(S, width(rounds)) > cluster::kRingBytes) ++rounds;
+        g->tc = width(rounds) < g->mp ? width(rounds) : g->mp;
+    }
     return g->stages >= cluster::kMinStages;
 }
 

@@ -450,6 +450,22 @@ __device__ __forceinline__ void mbar_arrive_remote_release(uint32_t remote_bar) 
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from this CTA's shared memory to a CTA of the cluster (`dst_cluster`, a
+// shared::cluster address from mapa), counted as transaction bytes on that
+// CTA's mbarrier `bar_cluster`.  The source must have been written before
+// with a fence.proxy.async.shared::cta between the writes and this copy;
+// the copy has finished reading it once the destination's phase completes.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                     uint32_t bar_cluster) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst_cluster), "r"(src), "r"(bytes), "r"(bar_cluster) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 // 16 bytes into another CTA's shared memory of the cluster, counted as
 // transaction bytes on that CTA's mbarrier `remote_bar`.
 __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint4 v, uint32_t remote_bar) {

@@ -119,7 +119,7 @@ MFP8_API mfp8_status mfp8_linear(const void* X_bf16, int64_t M, int64_t K,
 typedef enum {
     MFP8_PATH_AUTO = 0,   /* what mfp8_linear does: chosen from M, N, K */
     MFP8_PATH_TILED = 1,  /* quantize pass, then the persistent 128-row-tile tcgen05 GEMM */
-    MFP8_PATH_SPLITK = 2, /* quantize pass, then the split-K GEMM on CTA clusters, partials summed on chip (M <= 128) */
+    MFP8_PATH_SPLITK = 2, /* quantize pass, then the split-K GEMM on CTA clusters, partials summed on chip (M <= 256) */
     MFP8_PATH_PAIR = 3,   /* quantize pass, then the 256-row-tile GEMM on CTA pairs (tcgen05 cta_group::2) */
     MFP8_PATH_FUSED = 4   /* one kernel: quantizes X on chip and streams the weights, K split over a CTA cluster (M <= 16) */
 } mfp8_path;

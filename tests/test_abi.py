@@ -112,7 +112,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert call(path=5) == mfp8.ERR_INVALID_ARG
     assert call(path=mfp8.PATH_FUSED, M=17) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(ws=None, path=mfp8.PATH_SPLITK) == mfp8.ERR_WORKSPACE  # the quantize pass's codes
-    assert call(path=mfp8.PATH_SPLITK, M=129) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(path=mfp8.PATH_SPLITK, M=257) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(x8=FAKE * 6) == mfp8.ERR_INVALID_ARG  # codes without scales
     assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X
     assert call(M=0) == mfp8.OK
@@ -124,8 +124,8 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     G = mfp8.mfp8_gemm
     assert G(None, FAKE, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_INVALID_ARG
     assert G(FAKE, FAKE * 9 + 4, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, 0, None) == mfp8.ERR_MISALIGNED
-    assert G(FAKE, FAKE * 9, 129, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, mfp8.PATH_SPLITK,
-             None) == mfp8.ERR_UNSUPPORTED_SHAPE  # split-K kernel: M <= 128
+    assert G(FAKE, FAKE * 9, 257, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, mfp8.PATH_SPLITK,
+             None) == mfp8.ERR_UNSUPPORTED_SHAPE  # split-K kernel: M <= 256
     assert G(FAKE, FAKE * 9, 4, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None, 0, mfp8.PATH_FUSED, None) == mfp8.ERR_INVALID_ARG
     assert mfp8.mfp8_e4m3_encode_f32(FAKE, -1, FAKE * 2, None) == mfp8.ERR_INVALID_ARG
     assert mfp8.mfp8_debug_bounded_wait(0, None) == mfp8.ERR_INVALID_ARG

@@ -39,14 +39,14 @@ class Guarded:
 CASES = [  # (M, N, K): ragged in M and N, several tiles
     (1, 136, 272), (5, 264, 400), (13, 1032, 528), (16, 392, 1040),      # one-kernel decode path
     (17, 136, 272), (37, 264, 400), (100, 520, 528), (128, 1160, 400),   # cluster split-K
-    (130, 264, 384), (201, 776, 528),                                    # 1-CTA tiles
+    (130, 264, 384), (201, 776, 528), (256, 1032, 400),                  # 1-CTA tiles, split-K
     (300, 520, 400), (513, 1032, 528),                                   # CTA pairs
 ]
 
 
 def _paths(M):
     p = [mfp8.PATH_AUTO, mfp8.PATH_TILED, mfp8.PATH_PAIR]
-    if M <= 128:
+    if M <= 256:
         p.append(mfp8.PATH_SPLITK)
     if M <= 16:
         p.append(mfp8.PATH_FUSED)
@@ -97,7 +97,7 @@ def test_quantize_and_gemm_write_nothing_outside_their_buffers(M, N, K):
     for g in (gx8, gxs, gw8, gsw):
         assert g.guards_intact()
     x8, xs = gx8.view(torch.uint8, (M, K)), gxs.view(torch.float32, (M,))
-    for path in [mfp8.PATH_TILED, mfp8.PATH_PAIR] + ([mfp8.PATH_SPLITK] if M <= 128 else []):
+    for path in [mfp8.PATH_TILED, mfp8.PATH_PAIR] + ([mfp8.PATH_SPLITK] if M <= 256 else []):
         gy = Guarded(M * N * 2)
         st = mfp8.mfp8_gemm(x8.data_ptr(), xs.data_ptr(), M, K, W8.data_ptr(), sw.data_ptr(), N,
                             gy.body.data_ptr(), None, 0, path, h)

@@ -91,13 +91,15 @@ def test_fused_stream_geometry(M, N, K):
     run_case(M, N, K, mfp8.PATH_FUSED, seed=M * 5 + K, flags=mfp8.FLAG_STATIC_WEIGHTS if M % 2 else 0)
 
 
-# The cluster split-K kernel on codes: token columns 16..128 (M rounded up
+# The cluster split-K kernel on codes: token columns 16..256 (M rounded up
 # to 16, with ragged M), cluster sizes 1..8, a ragged last K block, a K
 # shorter than one block, a partial last channel tile (N % 128 != 0), grids
 # of many tiles, and long K.
 CLUSTER = [
     (17, 8, 16), (24, 136, 272), (48, 1032, 4112), (64, 6144, 4096), (80, 264, 4992), (96, 4096, 12288),
     (112, 520, 1040), (128, 12296, 2064), (33, 40960, 256), (127, 1024, 8320), (65, 24576, 4096),
+    (129, 1032, 4112), (160, 264, 400), (192, 4096, 4096), (200, 12296, 2064), (255, 136, 272),
+    (256, 1024, 8320), (176, 24576, 512), (240, 4096, 12288),
 ]
 
 
@@ -140,8 +142,8 @@ def test_fused_back_to_back_on_one_stream():
     assert torch.isfinite(a.float()).all()
 
 
-@pytest.mark.parametrize("M,path", [(32, mfp8.PATH_SPLITK), (112, mfp8.PATH_SPLITK), (200, mfp8.PATH_TILED),
-                                    (512, mfp8.PATH_PAIR)])
+@pytest.mark.parametrize("M,path", [(32, mfp8.PATH_SPLITK), (112, mfp8.PATH_SPLITK), (200, mfp8.PATH_SPLITK),
+                                    (200, mfp8.PATH_TILED), (512, mfp8.PATH_PAIR)])
 def test_dependent_chain_every_path(M, path):
     """Each call is a quantize pass that lets its GEMM start early and a GEMM
     that waits for the codes; consecutive calls overlap the same way.  A
@@ -180,8 +182,8 @@ def test_linear_tiled_ragged(M, N, K, path):
 def test_gemm_entry_point(M, N, K, path):
     """mfp8_gemm on codes from mfp8_quantize_act: within tolerance of the
     oracle, and bit-identical to mfp8_linear through the same kernel."""
-    if path == mfp8.PATH_SPLITK and M > 128:
-        pytest.skip("split-K takes M <= 128")
+    if path == mfp8.PATH_SPLITK and M > 256:
+        pytest.skip("split-K takes M <= 256")
     x = W.make_x(M, K, seed=5, device=DEV)
     W8, sw = mfp8.quantize_weight(W.make_w(N, K, seed=5, device=DEV))
     x8, xs = mfp8.quantize_act(x)
