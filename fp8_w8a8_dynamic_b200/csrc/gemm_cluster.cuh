@@ -74,8 +74,8 @@ __host__ __device__ constexpr uint32_t tmem_cols(int mp) {
 }
 
 // Ring bytes one exchange round of tc token columns takes (S > 1): the
-// receive slots [S][128/S][tc] fp32 of the channels this CTA owns, then the
-// send slots [S-1][128/S][tc] fp32 of the channels the other ranks own.
+// receive slots [S][tc][128/S] fp32 of the channels this CTA owns, then the
+// send slots [S-1][tc][128/S] fp32 of the channels the other ranks own.
 __host__ __device__ constexpr int exchange_bytes(int S, int tc) {
     return (TILE * tc * 4 / S) * (2 * S - 1);
 }
@@ -105,14 +105,6 @@ struct Args {
     int weights_static;
     Geometry g;
 };
-
-// Position of 16-byte token group g in channel cl's row of an exchange slot
-// (tc token columns, tc / 4 groups, a multiple of 4): g ^ swz(cl), so that
-// 16-byte accesses of one group across consecutive channels (the TMEM
-// copy-out, one channel per thread, and the owner's sum) hit distinct banks.
-// The XOR stays inside an aligned run of 8 groups when tc is a multiple of
-// 32, of 4 otherwise.
-__device__ __forceinline__ int recv_swz(int cl, int tc) { return (tc & 31) == 0 ? (cl & 7) : ((cl >> 1) & 3); }
 
 __global__ void __launch_bounds__(kThreads, 2)
 gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -310,17 +302,17 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         }
     } else {
         // ---------------------------------- partial-row exchange, S > 1 --
-        // Rounds of TC token columns.  Slot layout (fp32): receive slot s =
-        // partials from rank s of the 128/S channels this CTA owns, at
-        // s * SLOT; send slot of owner o != rank at (S + o') * SLOT, o' = o
-        // or o - 1 (this rank's own slot is written straight into receive
-        // slot `rank`).  A slot row is one channel's TC columns in 16-byte
-        // groups, group g at position g ^ recv_swz(channel, TC).  Every warp
-        // takes part in the round's closing cluster barrier.
+        // Rounds of TC token columns.  Slot layout (fp32, token-major):
+        // receive slot s = partials from rank s of the 128/S channels this
+        // CTA owns, at s * SLOT; send slot of owner o != rank at (S + o') *
+        // SLOT, o' = o or o - 1 (this rank's own slot is written straight
+        // into receive slot `rank`).  Row r of a slot is token tok0 + r, its
+        // 128/S channels contiguous.  Every warp takes part in the round's
+        // closing cluster barrier.
         const int TC = args.g.tc;
         const int rounds = (MP + TC - 1) / TC;
-        const uint32_t SLOT = uint32_t(CPR * TC * 4);
-        const uint32_t row_bytes = uint32_t(TC * 4);
+        const uint32_t row_bytes = uint32_t(CPR * 4);
+        const uint32_t SLOT = row_bytes * uint32_t(TC);
         for (int j = 0; j < rounds; ++j) {
             const int tok0 = j * TC;
             const int tcj = MP - tok0 < TC ? MP - tok0 : TC;  // columns this round (a multiple of 16)
@@ -329,19 +321,31 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const int q = int(warp & 3u);
                 const int c = q * 32 + int(lane);
                 const int o = c / CPR, cl = c % CPR;
-                const int swz = recv_swz(cl, TC);
                 const uint32_t slot = o == rank ? uint32_t(rank) * SLOT : uint32_t(S + (o < rank ? o : o - 1)) * SLOT;
-                const uint32_t row = sbase + slot + uint32_t(cl) * row_bytes;
+                // This thread's channel in every row of its slot: the 32 lanes
+                // of a warp write consecutive words of a row.
+                const uint32_t col = sbase + slot + uint32_t(cl) * 4u;
                 if (have_acc) {
                     if (j == 0) tc_fence_after();
-                    for (int c0 = 0; c0 < tcj; c0 += 16) {
-                        uint32_t acc[16];
-                        tmem_ld_32x32b_x16(tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(tok0 + c0), acc);
+                    const uint32_t taddr = tmem_base + ((uint32_t(q) * 32u) << 16) + uint32_t(tok0);
+                    int c0 = 0;
+                    for (; c0 + 32 <= tcj; c0 += 32) {
+                        uint32_t acc[32];
+                        tmem_ld_32x32b_x32(taddr + uint32_t(c0), acc);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < 4; ++h)
-                            st_shared_v4(row + 16u * uint32_t((c0 / 4 + h) ^ swz), acc[4 * h], acc[4 * h + 1],
-                                         acc[4 * h + 2], acc[4 * h + 3]);
+                        for (int i = 0; i < 32; ++i)
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(col + uint32_t(c0 + i) * row_bytes), "r"(acc[i])
+                                         : "memory");
+                    }
+                    if (c0 < tcj) {  // a last 16 columns
+                        uint32_t acc[16];
+                        tmem_ld_32x32b_x16(taddr + uint32_t(c0), acc);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(col + uint32_t(c0 + i) * row_bytes), "r"(acc[i])
+                                         : "memory");
                     }
                 }
                 fence_proxy_async_smem();  // slot writes -> the bulk copies' reads
@@ -364,25 +368,25 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 // Rows of this round that exist: M - tok0 (when positive).
                 const int mj = M - tok0 < tcj ? M - tok0 : tcj;
                 if (have_partials && mj > 0) {
-                    // One thread per (channel, group of 4 tokens): a 16-byte
-                    // read per rank (all S issued together), consecutive
-                    // channels across the warp, so the Y stores of each token
-                    // row are contiguous.  Shared memory is read by
-                    // shared-space address (ld_shared_*) so that the reads are
-                    // not ordered behind the Y stores.
-                    const int G = (mj + 3) / 4;
-                    const int cl2 = t % CPR;
-                    const int n = n0 + rank * CPR + cl2;
-                    const float sw = ld_shared_f32(smem_u32(sw_sm + rank * CPR + cl2));
-                    const int swz2 = recv_swz(cl2, TC);
-                    const uint32_t base = sbase + uint32_t(cl2) * row_bytes;
+                    // One thread per (token row, group of 4 channels): a
+                    // 16-byte read per rank (all S issued together; the warp
+                    // reads 512 contiguous bytes), the rescale, and one 8-byte
+                    // store of 4 bf16 (the warp's stores cover whole row
+                    // segments).  Shared memory is read by shared-space
+                    // address (ld_shared_*) so that the reads are not ordered
+                    // behind the Y stores.
+                    const int GPR = CPR / 4;  // 4-channel groups per row
                     const uint32_t sa_base = smem_u32(sa_sm + tok0);
-                    for (int g = t / CPR; g < G && n < N; g += 128 / CPR) {
-                        const uint32_t pos = 16u * uint32_t(g ^ swz2);
+                    const uint32_t sw_base = smem_u32(sw_sm + rank * CPR);
+                    for (int e = t; e < mj * GPR; e += 128) {
+                        const int r = e / GPR, g4 = e % GPR;
+                        const int n = n0 + rank * CPR + 4 * g4;
+                        if (n >= N) continue;  // N % 8 == 0: a group of 4 is all in or all out
+                        const uint32_t off = uint32_t(r) * row_bytes + uint32_t(16 * g4);
                         float4 p[kMaxCluster];
 #pragma unroll
                         for (int i = 0; i < kMaxCluster; ++i)
-                            if (i < S) p[i] = ld_shared_f4(base + uint32_t(i) * SLOT + pos);
+                            if (i < S) p[i] = ld_shared_f4(sbase + uint32_t(i) * SLOT + off);
                         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                         for (int i = 0; i < kMaxCluster; ++i)
@@ -392,13 +396,14 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                                 sum.z += p[i].z;
                                 sum.w += p[i].w;
                             }
-                        const float v[4] = {sum.x, sum.y, sum.z, sum.w};
-                        const float4 sa4 = ld_shared_f4(sa_base + uint32_t(16 * g));
-                        const float sa[4] = {sa4.x, sa4.y, sa4.z, sa4.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            if (4 * g + i < mj)
-                                args.Y[int64_t(tok0 + 4 * g + i) * N + n] = __float2bfloat16_rn(v[i] * sa[i] * sw);
+                        const float sa = ld_shared_f32(sa_base + uint32_t(4 * r));
+                        const float4 sw = ld_shared_f4(sw_base + uint32_t(16 * g4));
+                        const __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x * sa * sw.x, sum.y * sa * sw.y);
+                        const __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z * sa * sw.z, sum.w * sa * sw.w);
+                        uint2 packed;
+                        packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+                        packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+                        *reinterpret_cast<uint2*>(args.Y + int64_t(tok0 + r) * N + n) = packed;
                     }
                 }
                 // Arm the barrier for the next round's slots before any rank

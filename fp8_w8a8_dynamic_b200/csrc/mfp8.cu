@@ -379,10 +379,11 @@ int sm_count_for_sizing();
 int choose_path(int64_t M, int64_t N, int64_t K) {
     (void)K;
     if (M <= kStreamMaxM) return MFP8_PATH_FUSED;
-    // The cluster split-K kernel up to 112 rows: at 128 its 32 KB stages
-    // (a weight block and 128 code rows) leave a 3-deep ring and the 128-row
-    // tiles were measured faster on the layer's shapes.
-    if (M <= 112) return MFP8_PATH_SPLITK;
+    // The cluster split-K kernel up to 128 rows (measured ahead of the
+    // 128-row tiles there on the layer's shapes); above, its stages of a
+    // weight block and up to 256 code rows leave too shallow a ring and the
+    // tiles are faster.
+    if (M <= 128) return MFP8_PATH_SPLITK;
     if (M < 256) return MFP8_PATH_TILED;
     // Too few 256 x 256 pair tiles to occupy half the CTA pairs (the k/v
     // projections at M = 2048 make 32): narrower single-CTA tiles fill the
@@ -535,7 +536,8 @@ bool cluster_geometry(int64_t M, int64_t N, int64_t K, int sm_count, cluster::Ge
     const int st = cluster::kRingBytes / cluster::stage_bytes(g->mp);
     g->stages = st > cluster::kMaxStages ? cluster::kMaxStages : st;
     // Exchange rounds: as few as the ring allows, of equal width (a multiple
-    // of 32 token columns where the round is that wide, else of 16).
+    // of 32 token columns where the round is that wide, else of 16: whole
+    // 32-column TMEM loads).
     g->tc = g->mp;
     if (S > 1) {
         int rounds = 1;

@@ -125,7 +125,7 @@ typedef enum {
 } mfp8_path;
 
 /* The kernel MFP8_PATH_AUTO takes at these sizes (FUSED for M <= 16, SPLITK
- * up to 112, TILED below 256, PAIR above); MFP8_PATH_AUTO itself for sizes
+ * up to 128, TILED below 256, PAIR above); MFP8_PATH_AUTO itself for sizes
  * no kernel takes. */
 MFP8_API int mfp8_choose_path(int64_t M, int64_t N, int64_t K);
 

@@ -63,12 +63,13 @@ def test_workspace_bytes(lib):
     assert mfp8.mfp8_gemm_workspace_bytes(16, 4096, 4096) == 0
     assert mfp8.mfp8_gemm_workspace_bytes(300, 4096, 4096) == 0
     # the AUTO choice: the one-kernel path up to 16 tokens, the cluster
-    # split-K kernel to 112, 128-row tiles for mid M, pairs above
+    # split-K kernel to 128, 128-row tiles for mid M, pairs above
     assert mfp8.mfp8_choose_path(8, 12288, 4096) == mfp8.PATH_FUSED
     assert mfp8.mfp8_choose_path(16, 4096, 12288) == mfp8.PATH_FUSED
     assert mfp8.mfp8_choose_path(17, 4096, 4096) == mfp8.PATH_SPLITK
     assert mfp8.mfp8_choose_path(112, 4096, 4096) == mfp8.PATH_SPLITK
-    assert mfp8.mfp8_choose_path(128, 4096, 4096) == mfp8.PATH_TILED
+    assert mfp8.mfp8_choose_path(128, 4096, 4096) == mfp8.PATH_SPLITK
+    assert mfp8.mfp8_choose_path(129, 4096, 4096) == mfp8.PATH_TILED
     assert mfp8.mfp8_choose_path(200, 4096, 4096) == mfp8.PATH_TILED
     assert mfp8.mfp8_choose_path(2048, 4096, 4096) == mfp8.PATH_PAIR
     assert mfp8.mfp8_choose_path(0, 4096, 4096) == mfp8.PATH_AUTO
