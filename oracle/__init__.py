@@ -22,6 +22,16 @@ module only marshals numpy arrays into it.  What each function follows:
   s_a[m] * s_w[n]; ``dot_int64`` is the same contraction in integers.
 * ``within_tolerance`` - the acceptance rule for BF16 outputs:
   |y - y_ref| <= 2^-7 |y_ref| + 1e-5 * s_abs.
+* ``kv_quantize`` / ``kv_dequantize`` - the FP8 e4m3 KV cache that the
+  README's SGLang paragraph turns on with --kv-cache-dtype fp8_e4m3 (the
+  pages give only the flag).  Reading: one scale per (token, head) row of a
+  [T, H, D] tensor by the activation rule; dequantize = bf16(fl32(dec * s)).
+  ``f32_to_bf16`` is round-to-nearest-even on the dropped 16 bits.
+* ``rmsnorm`` / ``silu_mul`` - the producers of the quantized Linears'
+  inputs, exactly in fp64: RMSNorm before q/k/v and gate/up (named by the
+  "MOSS-VL-Realtime-FP8 mixed-precision strategy" article, norms kept in high
+  precision), and SiLU(gate) * up on the packed gate_up output before down
+  (the activation is not named on the pages: a reading).
 """
 import ctypes
 
@@ -53,6 +63,12 @@ class Oracle:
         L.orc_linear_ref.argtypes = [P, P, i64, P, P, i64, i64, P, P]
         L.orc_dot_int64.argtypes = [P, i64, P, i64, i64, P]
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_f32_to_bf16.restype = ctypes.c_uint16
+        L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.orc_kv_quantize.argtypes = [P, i64, i64, i64, P, P]
+        L.orc_kv_dequantize.argtypes = [P, P, i64, i64, i64, P]
+        L.orc_rmsnorm.argtypes = [P, P, i64, i64, ctypes.c_double, P]
+        L.orc_silu_mul.argtypes = [P, i64, i64, P]
         self.L = L
         self.path = path
 
@@ -107,6 +123,47 @@ class Oracle:
         self.L.orc_linear_ref(_ptr(x8), _ptr(s_a), M, _ptr(w8), _ptr(s_w), N, K,
                               _ptr(y), _ptr(sa) if want_abs else None)
         return y, sa
+
+    def f32_to_bf16(self, values):
+        """bf16 bit patterns of fp32 values (round to nearest even)."""
+        values = _c(values, np.float32)
+        return np.array([self.L.orc_f32_to_bf16(float(v)) for v in values.ravel()],
+                        dtype=np.uint16).reshape(values.shape)
+
+    def kv_quantize(self, kv_bits):
+        """kv_bits: uint16 bf16 patterns [T, H, D] -> (codes u8 [T, H, D], scales f32 [T, H])."""
+        kv_bits = _c(kv_bits, np.uint16)
+        T, H, D = kv_bits.shape
+        q = np.empty((T, H, D), dtype=np.uint8)
+        s = np.empty((T, H), dtype=np.float32)
+        self.L.orc_kv_quantize(_ptr(kv_bits), T, H, D, _ptr(q), _ptr(s))
+        return q, s
+
+    def kv_dequantize(self, codes, scales):
+        """codes u8 [T, H, D], scales f32 [T, H] -> bf16 bit patterns [T, H, D]."""
+        codes = _c(codes, np.uint8)
+        scales = _c(scales, np.float32)
+        T, H, D = codes.shape
+        out = np.empty((T, H, D), dtype=np.uint16)
+        self.L.orc_kv_dequantize(_ptr(codes), _ptr(scales), T, H, D, _ptr(out))
+        return out
+
+    def rmsnorm(self, x_bits, g_bits, eps):
+        """x_bits uint16 [M, K], g_bits uint16 [K] -> fp64 [M, K], exact."""
+        x_bits = _c(x_bits, np.uint16)
+        g_bits = _c(g_bits, np.uint16)
+        M, K = x_bits.shape
+        y = np.empty((M, K), dtype=np.float64)
+        self.L.orc_rmsnorm(_ptr(x_bits), _ptr(g_bits), M, K, float(eps), _ptr(y))
+        return y
+
+    def silu_mul(self, gu_bits):
+        """gu_bits uint16 [M, 2I] (gate, then up) -> fp64 [M, I], exact."""
+        gu_bits = _c(gu_bits, np.uint16)
+        M, I2 = gu_bits.shape
+        y = np.empty((M, I2 // 2), dtype=np.float64)
+        self.L.orc_silu_mul(_ptr(gu_bits), M, I2 // 2, _ptr(y))
+        return y
 
     def dot_int64(self, x8, w8):
         """Integer form of the contraction: sum_k (2^9 dec(x)) * (2^9 dec(w))."""
@@ -163,6 +220,26 @@ def quantize_rows(x_bits):
 
 def linear_ref(x8, s_a, w8, s_w, want_abs: bool = True):
     return default().linear_ref(x8, s_a, w8, s_w, want_abs)
+
+
+def kv_quantize(kv_bits):
+    return default().kv_quantize(kv_bits)
+
+
+def kv_dequantize(codes, scales):
+    return default().kv_dequantize(codes, scales)
+
+
+def f32_to_bf16(values):
+    return default().f32_to_bf16(values)
+
+
+def rmsnorm(x_bits, g_bits, eps):
+    return default().rmsnorm(x_bits, g_bits, eps)
+
+
+def silu_mul(gu_bits):
+    return default().silu_mul(gu_bits)
 
 
 def dot_int64(x8, w8):

@@ -170,6 +170,85 @@ void orc_quantize_rows(const uint16_t* X, int64_t R, int64_t K, uint8_t* Q, floa
     }
 }
 
+/* ---------------------------------------------------- FP8 KV cache -- */
+
+/* fp32 -> bf16: round to nearest, ties to even, on the 16 low bits dropped
+ * (a carry out of the mantissa moves into the exponent, up to infinity); a
+ * NaN stays a NaN (its quiet bit set). */
+uint16_t orc_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if (isnan(f)) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t lower = u & 0xFFFFu, upper = u >> 16;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+    return (uint16_t)upper;
+}
+
+/* The FP8 e4m3 KV cache ("MOSS-VL quantization README", SGLang paragraph:
+ * --kv-cache-dtype fp8_e4m3; the pages give only the flag).  Reading: a K or
+ * V tensor [T tokens][H heads][D] in bf16 gets one scale per (token, head)
+ * row of D values, by the same rule as the activations (orc_quantize_rows):
+ * s = fl32(absmax / 448) floored at FLT_MIN, q = e4m3(fl32(x / s)). */
+void orc_kv_quantize(const uint16_t* KV, int64_t T, int64_t H, int64_t D, uint8_t* Q, float* s) {
+    orc_quantize_rows(KV, T * H, D, Q, s);
+}
+
+/* Dequantize (reading): out = bf16(fl32(dec(q) * s)), the product rounded
+ * to fp32 (the decoded value is exact in fp32) and then to bf16. */
+void orc_kv_dequantize(const uint8_t* Q, const float* s, int64_t T, int64_t H, int64_t D, uint16_t* out) {
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < T * H; ++r) {
+        int64_t k;
+        for (k = 0; k < D; ++k) {
+            float v = (float)orc_e4m3_decode(Q[r * D + k]) * s[r];
+            out[r * D + k] = orc_f32_to_bf16(v);
+        }
+    }
+}
+
+/* ------------------------------------- producers of the activations -- */
+
+/* RMSNorm, the producer of the q/k/v and gate/up inputs ("MOSS-VL-Realtime-FP8
+ * mixed-precision strategy" article: the norms stay in high precision and
+ * feed the FP8 Linears).  The pages fix neither the formula's rounding nor
+ * eps; reading: y = x * g / sqrt(mean_k(x^2) + eps), computed exactly here
+ * (fp64; the result is the unrounded value the bf16 output approximates).
+ * X [M, K] and g [K] are bf16 bit patterns; y [M, K] fp64. */
+void orc_rmsnorm(const uint16_t* X, const uint16_t* g, int64_t M, int64_t K, double eps, double* y) {
+    int64_t m;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        const uint16_t* row = X + m * K;
+        double ss = 0.0;
+        int64_t k;
+        for (k = 0; k < K; ++k) {
+            double v = (double)orc_bf16_to_f32(row[k]);
+            ss += v * v;
+        }
+        double r = 1.0 / sqrt(ss / (double)K + eps);
+        for (k = 0; k < K; ++k)
+            y[m * K + k] = (double)orc_bf16_to_f32(row[k]) * r * (double)orc_bf16_to_f32(g[k]);
+    }
+}
+
+/* The gated MLP activation before down_proj (not named on the pages;
+ * reading: SiLU(gate) * up, SiLU(v) = v / (1 + e^-v)), on the packed
+ * gate_up output GU [M, 2I] (gate in columns 0 .. I-1, up in I .. 2I-1, the
+ * README's packed gate_up_proj), exactly in fp64: y [M, I]. */
+void orc_silu_mul(const uint16_t* GU, int64_t M, int64_t I, double* y) {
+    int64_t m;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        int64_t k;
+        for (k = 0; k < I; ++k) {
+            double gv = (double)orc_bf16_to_f32(GU[m * 2 * I + k]);
+            double uv = (double)orc_bf16_to_f32(GU[m * 2 * I + I + k]);
+            y[m * I + k] = gv / (1.0 + exp(-gv)) * uv;
+        }
+    }
+}
+
 /* ----------------------------------------------------------------- GEMM -- */
 
 /* y_ref[m,n] = (sum_k dec(X8[m,k]) * dec(W8[n,k])) * s_a[m] * s_w[n]

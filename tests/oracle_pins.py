@@ -308,6 +308,87 @@ def pin_onehot_closed_form(o, seed=6):
             assert y[m, n] == expect, (m, n)
 
 
+# ------------------------------------------------------------ KV cache --
+
+def pin_bf16_rounding(o, seed=13):
+    """fp32 -> bf16 against two library conversions (torch, ml_dtypes) on
+    values over the whole range, exact ties both ways, and specials."""
+    rng = np.random.default_rng(seed)
+    v = (rng.standard_normal(6000) * np.exp2(rng.uniform(-130, 127, 6000))).astype(np.float32)
+    base = rng.integers(0, 1 << 15, 2000, dtype=np.uint32) << 16
+    ties = np.concatenate([base | 0x8000, base | 0x18000 & 0xFFFF8000, base | 0x7FFF, base | 0x8001]).astype(np.uint32)
+    ties = ties[(ties & 0x7F800000) != 0x7F800000].view(np.float32)
+    v = np.concatenate([v, ties, np.float32([0.0, -0.0, np.inf, -np.inf, 3.3895314e38])]).astype(np.float32)
+    got = o.f32_to_bf16(v)
+    ref_t = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    ref_m = v.astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert np.array_equal(got, ref_t), f"{(got != ref_t).sum()} values differ from torch"
+    assert np.array_equal(got, ref_m), f"{(got != ref_m).sum()} values differ from ml_dtypes"
+    n = o.f32_to_bf16(np.float32([np.nan]))[0]
+    assert (n & 0x7F80) == 0x7F80 and (n & 0x7F) != 0, "NaN must stay NaN"
+
+
+def pin_kv_cache(o, seed=14):
+    """KV-cache quantize is the activation rule on (token, head) rows;
+    dequantize equals numpy's fp32 product rounded by ml_dtypes, and, with
+    power-of-two scales, the exact product."""
+    rng = np.random.default_rng(seed)
+    T, H, D = 7, 8, 128
+    kv = _random_rows(rng, T * H, D, -6, 6).reshape(T, H, D)
+    q, s = o.kv_quantize(kv)
+    q2, s2 = o.quantize_rows(kv.reshape(T * H, D))
+    assert np.array_equal(q.reshape(T * H, D), q2) and np.array_equal(s.reshape(-1), s2)
+    # heads are independent rows: permuting them permutes codes and scales
+    perm = rng.permutation(H)
+    qp, sp = o.kv_quantize(kv[:, perm, :])
+    assert np.array_equal(qp, q[:, perm, :]) and np.array_equal(sp, s[:, perm])
+    out = o.kv_dequantize(q, s)
+    prod = (lib_decode(q).astype(np.float32) * s[:, :, None]).astype(np.float32)
+    ref = prod.astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert np.array_equal(out, ref), f"{(out != ref).sum()} dequantized values differ"
+    # power-of-two scales: the product is exact in bf16 (codes have 4 significant bits)
+    s_pow2 = np.exp2(rng.integers(-20, 20, (T, H))).astype(np.float32)
+    out2 = o.kv_dequantize(q, s_pow2)
+    exact = lib_decode(q) * s_pow2[:, :, None].astype(np.float64)
+    assert np.array_equal(bits_to_f32(out2).astype(np.float64), exact)
+
+
+# ------------------------------------------------------------ producers --
+
+def pin_rmsnorm(o, seed=15):
+    """RMSNorm against torch's rms_norm in float64 (a library routine), and
+    the closed form of a constant row: c * g / sqrt(c^2 + eps)."""
+    rng = np.random.default_rng(seed)
+    M, K, eps = 6, 384, 1e-6
+    xb = _random_rows(rng, M, K, -4, 4)
+    gb = bf16_bits((1.0 + 0.3 * rng.standard_normal(K)).astype(np.float32))
+    y = o.rmsnorm(xb, gb, eps)
+    xt = torch.from_numpy(bits_to_f32(xb).astype(np.float64))
+    gt = torch.from_numpy(bits_to_f32(gb).astype(np.float64))
+    ref = torch.nn.functional.rms_norm(xt, (K,), gt, eps).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=0.0), "rmsnorm differs from torch"
+    c = np.float32(-2.5)
+    yc = o.rmsnorm(bf16_bits(np.full((1, 64), c, np.float32)), bf16_bits(np.ones(64, np.float32)), 0.25)
+    cd = float(c)
+    assert np.allclose(yc, cd / np.sqrt(cd * cd + 0.25), rtol=1e-15, atol=0.0)
+
+
+def pin_silu_mul(o, seed=16):
+    """SiLU(gate) * up against torch's silu in float64, on the packed
+    [gate | up] layout (a transposed half would fail), and silu(0) = 0."""
+    rng = np.random.default_rng(seed)
+    M, I = 5, 200
+    gu = _random_rows(rng, M, 2 * I, -3, 3)
+    y = o.silu_mul(gu)
+    v = torch.from_numpy(bits_to_f32(gu).astype(np.float64))
+    ref = (torch.nn.functional.silu(v[:, :I]) * v[:, I:]).numpy()
+    assert np.allclose(y, ref, rtol=1e-13, atol=0.0), "silu_mul differs from torch"
+    z = np.zeros((1, 8), np.uint16)
+    z[0, 4:] = bf16_bits(np.float32([1, 2, 3, 4]))
+    assert np.all(o.silu_mul(z) == 0.0)
+
+
 ALL_PINS = [pin_decode_table, pin_roundtrip, pin_rounding_cases, pin_encode_vs_library,
             pin_saturation, pin_scale_invariants, pin_scale_and_quotient_rounding, pin_gemm_bruteforce,
-            pin_gemm_int_vs_fp, pin_onehot_closed_form]
+            pin_gemm_int_vs_fp, pin_onehot_closed_form, pin_bf16_rounding, pin_kv_cache,
+            pin_rmsnorm, pin_silu_mul]

@@ -38,6 +38,25 @@ MUTANTS = {
     "dropped_term": ("for (k = 0; k < K; ++k) {\n                    double p", "for (k = 1; k < K; ++k) {\n                    double p"),
     # the activation scale is not applied
     "no_sa": ("double sc = (double)s_a[m] * (double)s_w[n];", "double sc = (double)s_w[n];"),
+    # bf16 by truncation instead of round-to-nearest-even
+    "bf16_truncate": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;",
+                      "if (lower > 0xFFFFu) upper += 1u;"),
+    # bf16 ties away from zero
+    "bf16_ties_away": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;",
+                       "if (lower >= 0x8000u) upper += 1u;"),
+    # KV dequantize without the scale
+    "kv_no_scale": ("float v = (float)orc_e4m3_decode(Q[r * D + k]) * s[r];",
+                    "float v = (float)orc_e4m3_decode(Q[r * D + k]);"),
+    # RMSNorm over the sum instead of the mean
+    "rms_sum": ("double r = 1.0 / sqrt(ss / (double)K + eps);", "double r = 1.0 / sqrt(ss + eps);"),
+    # RMSNorm without the gain
+    "rms_no_gain": ("y[m * K + k] = (double)orc_bf16_to_f32(row[k]) * r * (double)orc_bf16_to_f32(g[k]);",
+                    "y[m * K + k] = (double)orc_bf16_to_f32(row[k]) * r;"),
+    # SiLU with the wrong sign in the exponent
+    "silu_sign": ("y[m * I + k] = gv / (1.0 + exp(-gv)) * uv;", "y[m * I + k] = gv / (1.0 + exp(gv)) * uv;"),
+    # gate and up swapped
+    "silu_swap": ("double gv = (double)orc_bf16_to_f32(GU[m * 2 * I + k]);",
+                  "double gv = (double)orc_bf16_to_f32(GU[m * 2 * I + I + k]);"),
     # saturation missing (values above 448 become NaN)
     "no_satfinite": ("if (a >= 448.0) return (uint8_t)(sign | 0x7E);", "if (a >= 464.0) return (uint8_t)(sign | 0x7F);"),
 }
