@@ -352,6 +352,90 @@ def q_proj_m16(torch, mfp8, W, device, steps, warmup, dist_ctx, peaks):
             "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "all_bytes_per_launch": wb + 2 * M * lin.K + 2 * M * lin.N}
 
 
+def kv_cache_line(torch, mfp8, W, device, steps, warmup, peaks):
+    """The FP8 e4m3 KV cache (the README's SGLang --kv-cache-dtype fp8_e4m3):
+    quantize and dequantize K and V of T = 16384 tokens (the long video
+    context), 8 KV heads x 128, one scale per (token, head).  Four buffer sets
+    (4 x 96 MB, more than L2) are cycled so every call reads from HBM.
+    GB/s of algorithmic bytes: quantize 2 + 1 bytes per value + 4 per row,
+    dequantize 1 + 2 per value + 4 per row."""
+    T, H, D, sets = 16384, 8, 128, 4
+    kv = [W.make_x(T * H, D, seed=5, stream=i, kind="rowscale", device=device).view(T, H, D) for i in range(2 * sets)]
+    q = [torch.empty((T, H, D), dtype=torch.uint8, device=device) for _ in kv]
+    sc = [torch.empty((T, H), dtype=torch.float32, device=device) for _ in kv]
+    out = [torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for _ in kv]
+    torch.cuda.synchronize()
+
+    def quant(h):
+        for a, b, c in zip(kv, q, sc):
+            st = mfp8.mfp8_kv_quantize(a.data_ptr(), T, H, D, b.data_ptr(), c.data_ptr(), h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_kv_quantize")
+
+    def dequant(h):
+        for b, c, o in zip(q, sc, out):
+            st = mfp8.mfp8_kv_dequantize(b.data_ptr(), c.data_ptr(), T, H, D, o.data_ptr(), h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_kv_dequantize")
+
+    n = len(kv)
+    res = {"workload": "K and V of T=16384 tokens x 8 KV heads x 128 (long video context), one scale per "
+                       "(token, head); 4 buffer sets cycled (> L2)"}
+    for name, fn, per in (("quantize", quant, 3), ("dequantize", dequant, 3)):
+        ms = time_graph(torch, fn, steps, warmup, None)
+        us = ms * 1e3 / (steps * n)
+        nbytes = T * H * D * per + T * H * 4
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"GB/s": round(gbs, 1), "avg_launch_us": round(us, 3), "bytes_per_launch": nbytes,
+                     "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    assert mfp8.device_status() == mfp8.OK
+    del kv, q, sc, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def producers_line(torch, mfp8, W, device, steps, warmup, peaks):
+    """The activation quantization fused into its producers at the prefill
+    size M = 2048: RMSNorm + quantize (hidden 4096; reads the bf16 rows and
+    the gain, writes codes and scales only) and SiLU(gate) * up + quantize on
+    the packed gate_up output (I = 12288).  Buffer sets are cycled past L2.
+    GB/s of algorithmic bytes."""
+    M, H, I = 2048, 4096, 12288
+    res = {"workload": "prefill M=2048: RMSNorm+quantize (4096) and SiLU(gate)*up+quantize on the packed gate_up "
+                       "output (2 x 12288); codes and scales written, no bf16 copy"}
+    g = (1.0 + 0.1 * torch.randn(H, device=device)).to(torch.bfloat16)
+    xs = [W.make_x(M, H, seed=6, stream=i, kind="rowscale", device=device) for i in range(10)]
+    gus = [W.make_x(M, 2 * I, seed=7, stream=i, kind="rowscale", device=device) for i in range(3)]
+    cq = torch.empty((M, I), dtype=torch.uint8, device=device)
+    cs = torch.empty((M,), dtype=torch.float32, device=device)
+    torch.cuda.synchronize()
+
+    def norm(h):
+        for x in xs:
+            st = mfp8.mfp8_rmsnorm_quantize(x.data_ptr(), g.data_ptr(), 1e-6, M, H, None, cq.data_ptr(),
+                                            cs.data_ptr(), h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_rmsnorm_quantize")
+
+    def silu(h):
+        for gu in gus:
+            st = mfp8.mfp8_silu_mul_quantize(gu.data_ptr(), M, I, None, cq.data_ptr(), cs.data_ptr(), h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_silu_mul_quantize")
+
+    for name, fn, n, nbytes in (("rmsnorm_quantize", norm, len(xs), 3 * M * H + 2 * H + 4 * M),
+                                ("silu_mul_quantize", silu, len(gus), 5 * M * I + 4 * M)):
+        ms = time_graph(torch, fn, steps, warmup, None)
+        us = ms * 1e3 / (steps * n)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"GB/s": round(gbs, 1), "avg_launch_us": round(us, 3), "bytes_per_launch": nbytes,
+                     "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    assert mfp8.device_status() == mfp8.OK
+    del xs, gus
+    torch.cuda.empty_cache()
+    return res
+
+
 def fp8_ceiling_tflops(torch, device, n=8192, reps=10):
     """The box's dense e4m3 GEMM ceiling, as a denominator only: cuBLASLt
     through torch._scaled_mm on n x n x n, bf16 out, best of `reps` launches
@@ -745,6 +829,8 @@ def main():
     # The single q_proj Linear at M = 16 (seed 0), weights rotated past L2.
     config0 = q_proj_m16(torch, mfp8, W, device, max(5, args.steps), args.warmup, ctx, peaks)
     torch.cuda.empty_cache()
+    kv_cache = kv_cache_line(torch, mfp8, W, device, max(5, min(args.steps, 20)), args.warmup, peaks)
+    producers = producers_line(torch, mfp8, W, device, max(5, min(args.steps, 20)), args.warmup, peaks)
 
     stack = None
     if not args.no_stack:
@@ -778,6 +864,8 @@ def main():
         "gpu_launches": launches,
         "clocks": clk,
         "q_proj_m16": config0,
+        "kv_cache_fp8": kv_cache,
+        "fused_producers": producers,
         "prefill": prefill,
         "long_video": video,
         "stack": stack,

@@ -19,6 +19,7 @@
 #include "gemm_pair.cuh"
 #include "gemm_stream.cuh"
 #include "gemm_cluster.cuh"
+#include "producer.cuh"
 
 namespace mfp8 {
 namespace {
@@ -702,6 +703,43 @@ __global__ void bounded_wait_kernel(uint64_t limit_ns) {
     }
 }
 
+// Launch of a fused producer kernel: one block per row, VPT vectors of 8
+// values per thread (rows up to 16384 values), as a programmatic dependent.
+template <template <int> class Pick, class... A>
+mfp8_status launch_producer(int64_t nvec, int64_t M, cudaStream_t stream, A... args) {
+    auto launch = [&](auto kern) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(M));
+        cfg.blockDim = dim3(producer::kThreads);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) {
+            cudaGetLastError();
+            return MFP8_ERR_CUDA;
+        }
+        return MFP8_OK;
+    };
+    if (nvec <= 256) return launch(Pick<1>::kern());
+    if (nvec <= 512) return launch(Pick<2>::kern());
+    if (nvec <= 1024) return launch(Pick<4>::kern());
+    if (nvec <= 1536) return launch(Pick<6>::kern());
+    if (nvec <= 2048) return launch(Pick<8>::kern());
+    return MFP8_ERR_UNSUPPORTED_SHAPE;
+}
+
+template <int VPT>
+struct PickRmsnorm {
+    static auto kern() { return producer::rmsnorm_quant_kernel<VPT>; }
+};
+template <int VPT>
+struct PickSiluMul {
+    static auto kern() { return producer::silu_mul_quant_kernel<VPT>; }
+};
+
 }  // namespace
 }  // namespace mfp8
 
@@ -836,6 +874,107 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, /*weights_static=*/false,
                     /*dependent=*/false, dev, info, s);
+}
+
+mfp8_status mfp8_rmsnorm_quantize(const void* X_bf16, const void* gamma_bf16, float eps, int64_t M, int64_t K,
+                                  void* Y_bf16, void* X_fp8, float* x_scale, void* stream) {
+    mfp8_status st = check_quant_args(X_bf16, M, K, X_fp8, x_scale);
+    if (st != MFP8_OK) return st;
+    if (K > 16384) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (!(eps >= 0.0f) || eps > 1.0f) return MFP8_ERR_INVALID_ARG;
+    if (M == 0) return MFP8_OK;
+    if (!gamma_bf16) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(gamma_bf16) || !aligned16(Y_bf16)) return MFP8_ERR_MISALIGNED;
+    if (Y_bf16 && (ranges_overlap(Y_bf16, size_t(M * K * 2), X_bf16, size_t(M * K * 2)) ||
+                   ranges_overlap(Y_bf16, size_t(M * K * 2), X_fp8, size_t(M * K)) ||
+                   ranges_overlap(Y_bf16, size_t(M * K * 2), x_scale, size_t(M * 4))))
+        return MFP8_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
+    return launch_producer<PickRmsnorm>(K / 8, M, static_cast<cudaStream_t>(stream),
+                                        static_cast<const uint4*>(X_bf16), static_cast<const uint4*>(gamma_bf16),
+                                        K, eps, static_cast<uint4*>(Y_bf16), static_cast<uint2*>(X_fp8), x_scale);
+}
+
+mfp8_status mfp8_silu_mul_quantize(const void* GU_bf16, int64_t M, int64_t I, void* Y_bf16, void* X_fp8,
+                                   float* x_scale, void* stream) {
+    if (M < 0 || I < 0) return MFP8_ERR_INVALID_ARG;
+    if (I == 0 || I % 16 != 0 || I > 16384 || M > kMaxDim) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return MFP8_OK;
+    if (!GU_bf16 || !X_fp8 || !x_scale) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(GU_bf16) || !aligned16(X_fp8) || !aligned16(x_scale) || !aligned16(Y_bf16))
+        return MFP8_ERR_MISALIGNED;
+    const size_t in_bytes = size_t(M) * size_t(2 * I) * 2;
+    if (ranges_overlap(GU_bf16, in_bytes, X_fp8, size_t(M * I)) ||
+        ranges_overlap(GU_bf16, in_bytes, x_scale, size_t(M * 4)) ||
+        ranges_overlap(X_fp8, size_t(M * I), x_scale, size_t(M * 4)) ||
+        (Y_bf16 && (ranges_overlap(Y_bf16, size_t(M * I * 2), GU_bf16, in_bytes) ||
+                    ranges_overlap(Y_bf16, size_t(M * I * 2), X_fp8, size_t(M * I)) ||
+                    ranges_overlap(Y_bf16, size_t(M * I * 2), x_scale, size_t(M * 4)))))
+        return MFP8_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    return launch_producer<PickSiluMul>(I / 8, M, static_cast<cudaStream_t>(stream),
+                                        static_cast<const uint4*>(GU_bf16), I, static_cast<uint4*>(Y_bf16),
+                                        static_cast<uint2*>(X_fp8), x_scale);
+}
+
+mfp8_status mfp8_kv_quantize(const void* KV_bf16, int64_t T, int64_t H, int64_t D, void* KV_fp8, float* kv_scale,
+                             void* stream) {
+    if (T < 0 || H < 0 || D < 0) return MFP8_ERR_INVALID_ARG;
+    if (H == 0 || D == 0 || D % 16 != 0 || D > kMaxDim || H > kMaxDim || T > kMaxDim) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t R = T * H;
+    if (R > kMaxDim) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    mfp8_status st = check_quant_args(KV_bf16, R, D, KV_fp8, kv_scale);
+    if (st != MFP8_OK || R == 0) return st;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (D > 256) return quantize_weight_rows(KV_bf16, R, D, KV_fp8, kv_scale, s);  // long rows: the row kernels
+    const int vpr = int(D / 8);
+    const int lpr = vpr <= 2 ? 2 : vpr <= 4 ? 4 : vpr <= 8 ? 8 : vpr <= 16 ? 16 : 32;
+    const int64_t rows_per_block = int64_t(kQuantThreads / 32) * (32 / lpr);
+    const int64_t blocks = (R + rows_per_block - 1) / rows_per_block;
+    if (blocks > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    const uint4* x = static_cast<const uint4*>(KV_bf16);
+    uint2* q = static_cast<uint2*>(KV_fp8);
+    switch (lpr) {
+        case 2: quant_small_rows_kernel<2><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
+        case 4: quant_small_rows_kernel<4><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
+        case 8: quant_small_rows_kernel<8><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
+        case 16: quant_small_rows_kernel<16><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
+        default: quant_small_rows_kernel<32><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
+    }
+    return launch_status();
+}
+
+mfp8_status mfp8_kv_dequantize(const void* KV_fp8, const float* kv_scale, int64_t T, int64_t H, int64_t D,
+                               void* KV_bf16, void* stream) {
+    if (T < 0 || H < 0 || D < 0) return MFP8_ERR_INVALID_ARG;
+    if (H == 0 || D == 0 || D % 16 != 0 || D > kMaxDim || H > kMaxDim || T > kMaxDim) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t R = T * H;
+    if (R > kMaxDim) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (R == 0) return MFP8_OK;
+    if (!KV_fp8 || !kv_scale || !KV_bf16) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(KV_fp8) || !aligned16(kv_scale) || !aligned16(KV_bf16)) return MFP8_ERR_MISALIGNED;
+    if (ranges_overlap(KV_bf16, size_t(R * D * 2), KV_fp8, size_t(R * D)) ||
+        ranges_overlap(KV_bf16, size_t(R * D * 2), kv_scale, size_t(R * 4)))
+        return MFP8_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    const int64_t n16 = R * D / 16;
+    int64_t blocks = (n16 + kQuantThreads - 1) / kQuantThreads;
+    const int64_t cap = int64_t(info.sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    kv_dequant_kernel<<<unsigned(blocks), kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(KV_fp8), kv_scale, n16, int(D), static_cast<uint4*>(KV_bf16));
+    return launch_status();
 }
 
 mfp8_status mfp8_e4m3_encode_f32(const float* in, int64_t n, uint8_t* out, void* stream) {

@@ -19,6 +19,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "ptx.cuh"
 
@@ -271,6 +272,71 @@ quant_rows_loop_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict
     if (threadIdx.x == 0) S[row] = s;
     uint2* qr = Q + row * nvec;
     for (int64_t j = threadIdx.x; j < nvec; j += kQuantThreads) qr[j] = quantize8(__ldg(xr + j), s, r);
+}
+
+// ------------------------------------------------------- FP8 KV cache --
+// "MOSS-VL quantization README", SGLang paragraph (--kv-cache-dtype
+// fp8_e4m3; the pages give only the flag).  A K or V tensor [T, H, D] in
+// bf16 gets one scale per (token, head) row of D values, by the activation
+// rule above; dequantize is bf16(fl32(dec(q) * s)).
+
+// Rows of D <= 256 values (D % 16 == 0): LPR lanes per row (a power of two
+// >= D / 8), each holding one 16-byte vector of 8 values, 32 / LPR rows per
+// warp, so a warp's loads and stores are contiguous.  The absmax is a
+// shuffle reduction over the row's lanes.
+template <int LPR>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_small_rows_kernel(const uint4* __restrict__ X, int64_t R, int D, uint2* __restrict__ Q,
+                        float* __restrict__ S) {
+    constexpr int kRowsPerWarp = 32 / LPR;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp +
+                        lane / LPR;
+    const int v = lane % LPR;
+    const int vpr = D >> 3;  // vectors per row
+    const bool live = row < R && v < vpr;
+    const uint4 x = live ? __ldg(X + row * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t acc = absmax_bits_u4(x, 0u);
+    uint32_t amax = max(acc & 0xffffu, acc >> 16);
+#pragma unroll
+    for (int off = 1; off < LPR; off <<= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (!live) return;
+    const float s = scale_from_absmax_bits(amax);
+    const float r = __frcp_rn(s);
+    if (v == 0) S[row] = s;
+    Q[row * vpr + v] = quantize8(x, s, r);
+}
+
+// Dequantize: each thread turns 16 codes (16 bytes) into 16 bf16 (32 bytes).
+// e4m3 -> f16 is exact, f16 -> f32 is exact, the product with the row scale
+// rounds once to fp32 and the cast to bf16 rounds to nearest even.
+__device__ __forceinline__ uint32_t dequant2(uint16_t codes2, float s) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes2));
+    const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+    const float2 f = __half22float2(h);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+kv_dequant_kernel(const uint4* __restrict__ Q, const float* __restrict__ S, int64_t n16, int D,
+                  uint4* __restrict__ out) {
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    const int g16 = D >> 4;  // 16-code groups per row
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride) {
+        const uint4 q = __ldg(Q + i);
+        const float s = __ldg(S + i / g16);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            o[2 * j] = dequant2(uint16_t(w[j] & 0xffffu), s);
+            o[2 * j + 1] = dequant2(uint16_t(w[j] >> 16), s);
+        }
+        out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+        out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
 }
 
 // Diagnostic: for every absmax a (a positive finite bf16, or zero) the

@@ -57,6 +57,10 @@ def lib():
             "mfp8_choose_path": (i32, [i64, i64, i64]),
             "mfp8_gemm_workspace_bytes": (sz, [i64, i64, i64]),
             "mfp8_gemm": (i32, [P, P, i64, i64, P, P, i64, P, P, sz, i32, P]),
+            "mfp8_rmsnorm_quantize": (i32, [P, P, ctypes.c_float, i64, i64, P, P, P, P]),
+            "mfp8_silu_mul_quantize": (i32, [P, i64, i64, P, P, P, P]),
+            "mfp8_kv_quantize": (i32, [P, i64, i64, i64, P, P, P]),
+            "mfp8_kv_dequantize": (i32, [P, P, i64, i64, i64, P, P]),
             "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
             "mfp8_debug_quantize_check": (i32, [P, P]),
             "mfp8_debug_bounded_wait": (i32, [i64, P]),
@@ -119,6 +123,22 @@ def mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, workspace, worksp
               stream=0):
     return lib().mfp8_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, workspace, workspace_bytes, path,
                            stream)
+
+
+def mfp8_rmsnorm_quantize(X_bf16, gamma_bf16, eps, M, K, Y_bf16, X_fp8, x_scale, stream=0):
+    return lib().mfp8_rmsnorm_quantize(X_bf16, gamma_bf16, eps, M, K, Y_bf16, X_fp8, x_scale, stream)
+
+
+def mfp8_silu_mul_quantize(GU_bf16, M, I, Y_bf16, X_fp8, x_scale, stream=0):
+    return lib().mfp8_silu_mul_quantize(GU_bf16, M, I, Y_bf16, X_fp8, x_scale, stream)
+
+
+def mfp8_kv_quantize(KV_bf16, T, H, D, KV_fp8, kv_scale, stream=0):
+    return lib().mfp8_kv_quantize(KV_bf16, T, H, D, KV_fp8, kv_scale, stream)
+
+
+def mfp8_kv_dequantize(KV_fp8, kv_scale, T, H, D, KV_bf16, stream=0):
+    return lib().mfp8_kv_dequantize(KV_fp8, kv_scale, T, H, D, KV_bf16, stream)
 
 
 def mfp8_e4m3_encode_f32(inp, n, out, stream=0):
@@ -224,6 +244,52 @@ def gemm(X8, x_scale, W8, w_scale, out=None, path=PATH_AUTO, workspace=None, str
                                 device=X8.device)
     _check(mfp8_gemm(_ptr(X8), _ptr(x_scale), M, K, _ptr(W8), _ptr(w_scale), N, _ptr(out), _ptr(workspace),
                      workspace.numel(), path, _stream_handle(stream)), "mfp8_gemm")
+    return out
+
+
+def rmsnorm_quantize(X, gamma, eps, want_y=True, stream=None):
+    """X bf16 [M, K], gamma bf16 [K] -> (y bf16 [M, K] or None, codes uint8 [M, K], scales fp32 [M])."""
+    import torch
+    M, K = X.shape
+    y = torch.empty((M, K), dtype=torch.bfloat16, device=X.device) if want_y else None
+    codes = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    scales = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _check(mfp8_rmsnorm_quantize(_ptr(X), _ptr(gamma), float(eps), M, K, _ptr(y), _ptr(codes), _ptr(scales),
+                                 _stream_handle(stream)), "mfp8_rmsnorm_quantize")
+    return y, codes, scales
+
+
+def silu_mul_quantize(GU, want_y=True, stream=None):
+    """GU bf16 [M, 2I] (gate | up) -> (y bf16 [M, I] or None, codes uint8 [M, I], scales fp32 [M])."""
+    import torch
+    M, I2 = GU.shape
+    I = I2 // 2
+    y = torch.empty((M, I), dtype=torch.bfloat16, device=GU.device) if want_y else None
+    codes = torch.empty((M, I), dtype=torch.uint8, device=GU.device)
+    scales = torch.empty((M,), dtype=torch.float32, device=GU.device)
+    _check(mfp8_silu_mul_quantize(_ptr(GU), M, I, _ptr(y), _ptr(codes), _ptr(scales), _stream_handle(stream)),
+           "mfp8_silu_mul_quantize")
+    return y, codes, scales
+
+
+def kv_quantize(KV, stream=None):
+    """KV: bf16 [T, H, D] CUDA tensor -> (codes uint8 [T, H, D], scales fp32 [T, H])."""
+    import torch
+    T, H, D = KV.shape
+    codes = torch.empty((T, H, D), dtype=torch.uint8, device=KV.device)
+    scales = torch.empty((T, H), dtype=torch.float32, device=KV.device)
+    _check(mfp8_kv_quantize(_ptr(KV), T, H, D, _ptr(codes), _ptr(scales), _stream_handle(stream)),
+           "mfp8_kv_quantize")
+    return codes, scales
+
+
+def kv_dequantize(codes, scales, stream=None):
+    """codes uint8 [T, H, D], scales fp32 [T, H] -> bf16 [T, H, D]."""
+    import torch
+    T, H, D = codes.shape
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=codes.device)
+    _check(mfp8_kv_dequantize(_ptr(codes), _ptr(scales), T, H, D, _ptr(out), _stream_handle(stream)),
+           "mfp8_kv_dequantize")
     return out
 
 

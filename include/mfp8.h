@@ -194,6 +194,57 @@ MFP8_API mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t 
                       void* Y_bf16, void* workspace, size_t workspace_bytes,
                       int path, void* stream);
 
+/* The activation quantization fused into its producer: RMSNorm, the
+ * producer of the q/k/v and gate/up inputs ("MOSS-VL-Realtime-FP8
+ * mixed-precision strategy" article: the norms stay in high precision and
+ * feed the FP8 Linears).  Per token row of X [M, K] (bf16):
+ *   y = bf16(x * r * gamma),  r = 1 / sqrt(mean(x^2) + eps)   (fp32)
+ *   x_scale[m], X_fp8[m, :] = the mfp8_quantize_act codes of the bf16 y
+ * so the codes and scales are bit-identical to mfp8_quantize_act on the
+ * bf16 y that Y_bf16 receives (Y_bf16 may be NULL when only the codes are
+ * wanted).  The codes feed mfp8_gemm.  The pages fix neither eps nor the
+ * norm's rounding; y is within one bf16 unit of the exact value.
+ *   gamma_bf16 [K]; X_fp8 [M, K] u8; x_scale [M] fp32; caller-owned,
+ *   16-byte aligned, outputs not overlapping inputs.  K % 16 == 0 and
+ *   K <= 16384 (else MFP8_ERR_UNSUPPORTED_SHAPE); 0 <= eps <= 1
+ *   (else MFP8_ERR_INVALID_ARG); M == 0 is a no-op. */
+MFP8_API mfp8_status mfp8_rmsnorm_quantize(const void* X_bf16, const void* gamma_bf16, float eps,
+                                  int64_t M, int64_t K, void* Y_bf16, void* X_fp8, float* x_scale,
+                                  void* stream);
+
+/* The same for the gated MLP activation before down_proj, on the packed
+ * gate_up_proj output ("MOSS-VL quantization README", packed modules):
+ * GU_bf16 [M, 2I] holds gate in columns 0 .. I-1 and up in I .. 2I-1;
+ *   y = bf16(silu(gate) * up),  silu(v) = v / (1 + e^-v)   (fp32; for
+ *   v < 0 as v e^v / (1 + e^v), which cannot overflow)
+ * and X_fp8 [M, I], x_scale [M] are the mfp8_quantize_act codes and scales of
+ * y.  The pages do not name the activation: SiLU(gate) * up is this
+ * library's reading.  Y_bf16 [M, I] optional; I % 16 == 0, I <= 16384. */
+MFP8_API mfp8_status mfp8_silu_mul_quantize(const void* GU_bf16, int64_t M, int64_t I, void* Y_bf16,
+                                   void* X_fp8, float* x_scale, void* stream);
+
+/* FP8 e4m3 KV cache.  "MOSS-VL quantization README", SGLang paragraph
+ * (--kv-cache-dtype fp8_e4m3); the pages give only the flag, so the scale
+ * rule is this library's reading: a K or V tensor [T tokens][H heads][D]
+ * (bf16, row-major, contiguous) gets one fp32 scale per (token, head) row of
+ * D values, s = fl32(max |x| / 448) raised to FLT_MIN, and codes
+ * e4m3(fl32(x / s)) with round-to-nearest-even and saturation: the
+ * activation rule of mfp8_quantize_act, so the bytes are identical to
+ * mfp8_quantize_act on the [T*H, D] view.
+ *   KV_fp8 [T][H][D] u8 and kv_scale [T][H] fp32 are written; caller-owned,
+ *   16-byte aligned, not overlapping the input.  D % 16 == 0 (else
+ *   MFP8_ERR_UNSUPPORTED_SHAPE); T == 0 is a no-op. */
+MFP8_API mfp8_status mfp8_kv_quantize(const void* KV_bf16, int64_t T, int64_t H, int64_t D,
+                             void* KV_fp8, float* kv_scale, void* stream);
+
+/* The inverse of mfp8_kv_quantize for reading the cache:
+ * KV_bf16[t][h][d] = bf16(fl32(dec(KV_fp8[t][h][d]) * kv_scale[t][h])), the
+ * product rounded to fp32, then to bf16 (round to nearest even).  Same
+ * shapes, alignment and errors as mfp8_kv_quantize; KV_bf16 must not overlap
+ * the codes or scales. */
+MFP8_API mfp8_status mfp8_kv_dequantize(const void* KV_fp8, const float* kv_scale, int64_t T, int64_t H,
+                               int64_t D, void* KV_bf16, void* stream);
+
 /* Diagnostic: checks the quantizer's divide-free arithmetic against IEEE
  * divides.  The scale fl32(absmax / 448) of every absmax (0 and each positive
  * finite bf16) is computed as a corrected quotient by 7 times 2^-6, and each

@@ -91,6 +91,31 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert q(FAKE, 0, 64, None, None, None) == mfp8.OK  # empty: nothing to do
     w = mfp8.mfp8_quantize_weight
     assert w(FAKE, 8, 24, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+    rq, sq = mfp8.mfp8_rmsnorm_quantize, mfp8.mfp8_silu_mul_quantize
+    assert rq(FAKE, FAKE * 5, 1e-6, 4, 40, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # K % 16
+    assert rq(FAKE, FAKE * 5, 1e-6, 4, 32768, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert rq(FAKE, FAKE * 5, -1.0, 4, 64, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_INVALID_ARG  # eps
+    assert rq(FAKE, None, 1e-6, 4, 64, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_INVALID_ARG  # no gain
+    assert rq(FAKE, FAKE * 5 + 2, 1e-6, 4, 64, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_MISALIGNED
+    assert rq(FAKE, FAKE * 5, 1e-6, 4, 64, FAKE + 16, FAKE * 2, FAKE * 3, None) == mfp8.ERR_INVALID_ARG
+    assert rq(FAKE, FAKE * 5, 1e-6, 0, 64, None, FAKE * 2, FAKE * 3, None) == mfp8.OK
+    assert sq(FAKE, 4, 40, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert sq(FAKE, -1, 64, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_INVALID_ARG
+    assert sq(FAKE, 4, 64, None, FAKE + 32, FAKE * 3, None) == mfp8.ERR_INVALID_ARG  # codes overlap input
+    assert sq(FAKE + 4, 4, 64, None, FAKE * 2, FAKE * 3, None) == mfp8.ERR_MISALIGNED
+    assert sq(FAKE, 0, 64, None, FAKE * 2, FAKE * 3, None) == mfp8.OK
+    kq, kd = mfp8.mfp8_kv_quantize, mfp8.mfp8_kv_dequantize
+    assert kq(FAKE, 2, 8, 40, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # D % 16
+    assert kq(FAKE, 2, 0, 128, FAKE * 2, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # no heads
+    assert kq(FAKE, -1, 8, 128, FAKE * 2, FAKE * 3, None) == mfp8.ERR_INVALID_ARG
+    assert kq(FAKE + 8, 2, 8, 128, FAKE * 2, FAKE * 3, None) == mfp8.ERR_MISALIGNED
+    assert kq(FAKE, 2, 8, 128, FAKE + 64, FAKE * 3, None) == mfp8.ERR_INVALID_ARG  # codes overlap input
+    assert kq(FAKE, 0, 8, 128, None, None, None) == mfp8.OK
+    assert kd(FAKE, FAKE * 2, 2, 8, 40, FAKE * 3, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert kd(None, FAKE * 2, 2, 8, 128, FAKE * 3, None) == mfp8.ERR_INVALID_ARG
+    assert kd(FAKE, FAKE * 2 + 4, 2, 8, 128, FAKE * 3, None) == mfp8.ERR_MISALIGNED
+    assert kd(FAKE, FAKE * 2, 2, 8, 128, FAKE + 16, None) == mfp8.ERR_INVALID_ARG  # output overlaps codes
+    assert kd(FAKE, FAKE * 2, 0, 8, 128, FAKE * 3, None) == mfp8.OK
 
     L = mfp8.mfp8_linear_ex
     args = dict(X=FAKE, M=4, K=64, W=FAKE * 2, sw=FAKE * 3, N=64, Y=FAKE * 4, ws=FAKE * 5, wsb=1 << 16)
