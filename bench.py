@@ -36,15 +36,18 @@ DECODE_MS = (1, 4, 8)
 PREFILL_M = 2048
 
 
-def load_traffic(kernel):
-    """DRAM bytes per launch of `kernel` on the bench's workload, from the
-    committed ncu summary (profiles/roofline_traffic.json), or None."""
+def load_traffic(kernel, bytes_per_launch):
+    """DRAM bytes per launch of `kernel`: the ratio of DRAM traffic to
+    algorithmic bytes from the committed one-kernel ncu captures
+    (profiles/roofline_traffic.json) times this run's algorithmic bytes per
+    launch, or None."""
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "roofline_traffic.json")
     try:
         with open(path) as f:
-            return json.load(f).get(kernel, {}).get("dram_bytes_per_launch")
+            ratio = json.load(f).get(kernel, {}).get("dram_over_algorithmic")
     except (OSError, ValueError):
         return None
+    return None if ratio is None else round(ratio * bytes_per_launch)
 
 
 def load_peaks():
@@ -802,8 +805,8 @@ def main():
                                 "unit": "TFLOP/s", "frac": round(g_tf / fp8_peak, 4),
                                 # DRAM bytes per launch of the pair kernel, which runs 5 of
                                 # the 7 Linears and 96% of the FLOPs
-                                "traffic": load_traffic("gemm_pair_kernel") if "gemm_pair_kernel" in pk["kernel"]
-                                else None,
+                                "traffic": load_traffic("gemm_pair_kernel", pk["gemm_bytes"])
+                                if "gemm_pair_kernel" in pk["kernel"] else None,
                                 "kernel": pk["kernel"], "avg_launch_us": round(pk["gemm_us"], 3),
                                 "peak_source": f"{peaks['source']} bf16 x 2 (fp8/bf16 nominal ratio)"}}
         del pl
@@ -850,7 +853,7 @@ def main():
         "data": "synthetic", "config": decode_config(),
         "frac_of_hbm": round(value / ctx.world / peaks["hbm_gbs"], 4),
         "roofline": {"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": load_traffic(kt["kernel"]),
+                     "frac": round(gemm_gbs / peaks["hbm_gbs"], 4), "traffic": load_traffic(kt["kernel"], kt["gemm_bytes"]),
                      "kernel": kt["kernel"], "launches_timed": kt["launches"],
                      "avg_launch_us": round(kt["gemm_us"], 3),
                      "bytes_per_launch": round(kt["gemm_bytes"]),

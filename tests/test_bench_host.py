@@ -61,14 +61,18 @@ def test_hardware_slowdown_disqualifies_whatever_the_clock():
 
 
 def test_traffic_figures_come_from_the_committed_summary():
+    """The committed ratio is the captured bytes over the algorithmic bytes
+    of the captured launches, within a few per cent of 1, and the bench
+    scales it by a launch's algorithmic bytes."""
     with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
         committed = json.load(f)
     for kernel, entry in committed.items():
-        got = bench.load_traffic(kernel)
-        assert got == entry["dram_bytes_per_launch"]
-        # measured traffic is within a few per cent of the algorithmic bytes
-        assert 0.8 < got / entry["algorithmic_bytes_per_launch"] < 1.1
-    assert bench.load_traffic("no_such_kernel") is None
+        cap = sum(entry["captured_bytes"].values()) / len(entry["captured_bytes"])
+        alg = sum(entry["algorithmic_bytes"].values()) / len(entry["algorithmic_bytes"])
+        assert abs(entry["dram_over_algorithmic"] - cap / alg) < 0.02
+        assert 0.9 < entry["dram_over_algorithmic"] < 1.1
+        assert bench.load_traffic(kernel, 27678622) == round(entry["dram_over_algorithmic"] * 27678622)
+    assert bench.load_traffic("no_such_kernel", 1000) is None
 
 
 def test_peaks_are_the_measured_ones_when_present():
