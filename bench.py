@@ -321,6 +321,78 @@ def kernel_times(torch, mfp8, layer, steps, warmup):
     return out
 
 
+def layer_prefill_fused(torch, mfp8, W, device, steps, warmup, dist_ctx):
+    """One layer's seven Linears at M = 2048 (seed 2) in the model's
+    dataflow, with the activation quantization fused into the producers:
+    RMSNorm + quantize for the packed qkv_proj, a
+    quantize pass for o (its input comes from attention, outside this
+    library), RMSNorm + quantize for the packed gate_up_proj (one GEMM writing
+    [gate | up]), and SiLU(gate) * up + quantize on that output for down.  TFLOP/s of the seven GEMMs
+    over the whole sequence (producers and quantize included)."""
+    M, H, I = 2048, W.HIDDEN, W.INTERMEDIATE
+    lins = {l.name: l for l in W.LAYER_LINEARS}
+    w = {}
+    for i, name in enumerate(("o_proj", "down_proj")):
+        l = lins[name]
+        w[name] = mfp8.quantize_weight(W.make_w(l.N, l.K, seed=2, stream=3 + 3 * i, device=device))
+    # q/k/v as the packed qkv_proj
+    wq = torch.cat([W.make_w(lins[n].N, H, seed=2, stream=i, device=device)
+                    for i, n in enumerate(("q_proj", "k_proj", "v_proj"))])
+    w["qkv_proj"] = mfp8.quantize_weight(wq)
+    del wq
+    # gate and up as the packed gate_up_proj: one GEMM writes [gate | up]
+    wg = torch.cat([W.make_w(I, H, seed=2, stream=4, device=device), W.make_w(I, H, seed=2, stream=5, device=device)])
+    w["gate_up_proj"] = mfp8.quantize_weight(wg)
+    del wg
+    lins = dict(lins, qkv_proj=W.PACKED_LAYER_LINEARS[0], gate_up_proj=W.PACKED_LAYER_LINEARS[2])
+    h_attn = W.make_x(M, H, seed=2, stream=1, kind="rowscale", device=device)   # RMSNorm input (residual stream)
+    h_mlp = W.make_x(M, H, seed=2, stream=2, kind="rowscale", device=device)
+    attn = W.make_x(M, H, seed=2, stream=3, kind="rowscale", device=device)     # attention output, o_proj input
+    g1 = (1.0 + 0.1 * torch.randn(H, device=device)).to(torch.bfloat16)
+    g2 = (1.0 + 0.1 * torch.randn(H, device=device)).to(torch.bfloat16)
+    c_h, s_h = torch.empty((M, H), dtype=torch.uint8, device=device), torch.empty((M,), dtype=torch.float32, device=device)
+    c_i, s_i = torch.empty((M, I), dtype=torch.uint8, device=device), torch.empty((M,), dtype=torch.float32, device=device)
+    y = {n: torch.empty((M, lins[n].N), dtype=torch.bfloat16, device=device) for n in w}
+    gu = y["gate_up_proj"]  # gate | up
+    gws = torch.zeros((max(16, max(mfp8.mfp8_gemm_workspace_bytes(M, lins[n].N, lins[n].K) for n in w)),),
+                      dtype=torch.uint8, device=device)
+    torch.cuda.synchronize()
+
+    def gemm(codes, scales, name, out, h):
+        l = lins[name]
+        st = mfp8.mfp8_gemm(codes.data_ptr(), scales.data_ptr(), M, l.K, w[name][0].data_ptr(), w[name][1].data_ptr(),
+                            l.N, out.data_ptr(), gws.data_ptr(), gws.numel(), mfp8.PATH_AUTO, h)
+        if st != mfp8.OK:
+            raise mfp8.Mfp8Error(st, "mfp8_gemm")
+
+    def check(st, what):
+        if st != mfp8.OK:
+            raise mfp8.Mfp8Error(st, what)
+
+    def layer(h):
+        check(mfp8.mfp8_rmsnorm_quantize(h_attn.data_ptr(), g1.data_ptr(), 1e-6, M, H, None, c_h.data_ptr(),
+                                         s_h.data_ptr(), h), "mfp8_rmsnorm_quantize")
+        gemm(c_h, s_h, "qkv_proj", y["qkv_proj"], h)
+        check(mfp8.mfp8_quantize_act(attn.data_ptr(), M, H, c_h.data_ptr(), s_h.data_ptr(), h), "mfp8_quantize_act")
+        gemm(c_h, s_h, "o_proj", y["o_proj"], h)
+        check(mfp8.mfp8_rmsnorm_quantize(h_mlp.data_ptr(), g2.data_ptr(), 1e-6, M, H, None, c_h.data_ptr(),
+                                         s_h.data_ptr(), h), "mfp8_rmsnorm_quantize")
+        gemm(c_h, s_h, "gate_up_proj", gu, h)
+        check(mfp8.mfp8_silu_mul_quantize(gu.data_ptr(), M, I, None, c_i.data_ptr(), s_i.data_ptr(), h),
+              "mfp8_silu_mul_quantize")
+        gemm(c_i, s_i, "down_proj", y["down_proj"], h)
+
+    n = max(5, steps // 2)
+    ms = time_graph(torch, layer, n, warmup, dist_ctx) / n
+    flops = sum(2 * M * l.N * l.K for l in W.LAYER_LINEARS)
+    assert mfp8.device_status() == mfp8.OK
+    return {"workload": "one layer's 7 Linears at M=2048 (seed 2) in the model's dataflow, packed as the README's "
+                        "qkv_proj and gate_up_proj: RMSNorm+quantize for each packed projection, a quantize pass for "
+                        "o, SiLU(gate)*up+quantize on the gate_up output for down",
+            "value": round(flops / (ms * 1e-3) / 1e12 * dist_ctx.world, 1), "unit": "TFLOP/s",
+            "ms_per_layer": round(ms, 4), "launches_per_layer": 8}
+
+
 def q_proj_m16(torch, mfp8, W, device, steps, warmup, dist_ctx, peaks):
     """The single q_proj-shaped Linear at M = 16 (seed 0): 4096 -> 4096,
     16.8 MB of e4m3 weights.  One weight set fits in L2, so the graph cycles
@@ -812,6 +884,12 @@ def main():
         del pl
         torch.cuda.empty_cache()
 
+    fused_layer = None
+    if not args.no_prefill:
+        fused_layer = layer_prefill_fused(torch, mfp8, W, device, args.steps, args.warmup, ctx)
+        fused_layer["frac_of_fp8_ceiling"] = round(fused_layer["value"] / ctx.world / prefill["fp8_ceiling"]["value"], 4)
+        torch.cuda.empty_cache()
+
     # Long video-context prefill: gate/up/down at M = 16384 (seed 3).
     video = None
     if not args.no_prefill:
@@ -870,6 +948,7 @@ def main():
         "kv_cache_fp8": kv_cache,
         "fused_producers": producers,
         "prefill": prefill,
+        "layer_prefill_fused_producers": fused_layer,
         "long_video": video,
         "stack": stack,
         "cpu_baseline": cpu,
