@@ -27,6 +27,14 @@ module only marshals numpy arrays into it.  What each function follows:
   pages give only the flag).  Reading: one scale per (token, head) row of a
   [T, H, D] tensor by the activation rule; dequantize = bf16(fl32(dec * s)).
   ``f32_to_bf16`` is round-to-nearest-even on the dropped 16 bits.
+* ``kv8_quantize`` / ``kv8_read`` / ``kv8_history_tokens`` - the INT8 KV
+  cache of the README's KV8 section (hqq backend, nbits 8, q_group_size 64,
+  axis 0, residual_length 128; the pages do not give HQQ's optimizer).
+  Readings: groups of 64 consecutive tokens per (head, channel) column of a
+  [T, H, D] tensor; the asymmetric min-max fit with an integer zero point in
+  fp32 (each rounding stated in the C source); the read dequantizes the
+  history and appends the bf16 tail; the latest 128 positions stay bf16 and
+  older ones are quantized in whole groups of 64.
 * ``rmsnorm`` / ``silu_mul`` - the producers of the quantized Linears'
   inputs, exactly in fp64: RMSNorm before q/k/v and gate/up (named by the
   "MOSS-VL-Realtime-FP8 mixed-precision strategy" article, norms kept in high
@@ -68,6 +76,10 @@ class Oracle:
         L.orc_kv_quantize.argtypes = [P, i64, i64, i64, P, P]
         L.orc_kv_dequantize.argtypes = [P, P, i64, i64, i64, P]
         L.orc_rmsnorm.argtypes = [P, P, i64, i64, ctypes.c_double, P]
+        L.orc_kv8_quantize.argtypes = [P, i64, i64, i64, P, P, P]
+        L.orc_kv8_read.argtypes = [P, P, P, i64, P, i64, i64, i64, P]
+        L.orc_kv8_history_tokens.restype = i64
+        L.orc_kv8_history_tokens.argtypes = [i64]
         L.orc_silu_mul.argtypes = [P, i64, i64, P]
         self.L = L
         self.path = path
@@ -147,6 +159,32 @@ class Oracle:
         out = np.empty((T, H, D), dtype=np.uint16)
         self.L.orc_kv_dequantize(_ptr(codes), _ptr(scales), T, H, D, _ptr(out))
         return out
+
+    def kv8_quantize(self, kv_bits):
+        """kv_bits uint16 [T, H, D], T % 64 == 0 -> (codes u8 [T, H, D],
+        scale f32 [T/64, H, D], zero f32 [T/64, H, D])."""
+        kv_bits = _c(kv_bits, np.uint16)
+        T, H, D = kv_bits.shape
+        if T % 64:
+            raise ValueError("kv8_quantize: T must be a multiple of 64")
+        q = np.empty((T, H, D), dtype=np.uint8)
+        sc = np.empty((T // 64, H, D), dtype=np.float32)
+        z = np.empty((T // 64, H, D), dtype=np.float32)
+        self.L.orc_kv8_quantize(_ptr(kv_bits), T, H, D, _ptr(q), _ptr(sc), _ptr(z))
+        return q, sc, z
+
+    def kv8_read(self, codes, scale, zero, resid_bits):
+        """Dequantized codes [Tq, H, D] followed by the bf16 residual [Tr, H, D] -> bf16 bits [Tq + Tr, H, D]."""
+        codes, scale, zero = _c(codes, np.uint8), _c(scale, np.float32), _c(zero, np.float32)
+        resid_bits = _c(resid_bits, np.uint16)
+        Tq, H, D = codes.shape
+        Tr = resid_bits.shape[0]
+        out = np.empty((Tq + Tr, H, D), dtype=np.uint16)
+        self.L.orc_kv8_read(_ptr(codes), _ptr(scale), _ptr(zero), Tq, _ptr(resid_bits), Tr, H, D, _ptr(out))
+        return out
+
+    def kv8_history_tokens(self, T):
+        return int(self.L.orc_kv8_history_tokens(int(T)))
 
     def rmsnorm(self, x_bits, g_bits, eps):
         """x_bits uint16 [M, K], g_bits uint16 [K] -> fp64 [M, K], exact."""
@@ -236,6 +274,18 @@ def f32_to_bf16(values):
 
 def rmsnorm(x_bits, g_bits, eps):
     return default().rmsnorm(x_bits, g_bits, eps)
+
+
+def kv8_quantize(kv_bits):
+    return default().kv8_quantize(kv_bits)
+
+
+def kv8_read(codes, scale, zero, resid_bits):
+    return default().kv8_read(codes, scale, zero, resid_bits)
+
+
+def kv8_history_tokens(T):
+    return default().kv8_history_tokens(T)
 
 
 def silu_mul(gu_bits):

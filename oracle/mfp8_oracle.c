@@ -207,6 +207,98 @@ void orc_kv_dequantize(const uint8_t* Q, const float* s, int64_t T, int64_t H, i
     }
 }
 
+/* ------------------------------------------------- INT8 KV cache (HQQ) -- */
+
+/* The INT8 KV cache of the "MOSS-VL quantization README", KV8 section: the
+ * cache_config of generation_config.json names the hqq backend with nbits 8,
+ * axis_key = axis_value = 0, q_group_size 64 and residual_length 128, and the
+ * text says the history is kept quantized while a short bf16 tail of recent
+ * positions is not.  The pages give these settings, not HQQ's optimizer.
+ *
+ * Readings (all of them this project's):
+ *  - a K or V tensor of one layer is [T tokens][H heads][D]; axis 0 is the
+ *    token axis, so a group is 64 consecutive tokens of one (head, channel)
+ *    column, and a tensor of T tokens (T % 64 == 0) has T/64 groups per
+ *    column: scale and zero are [T/64][H][D];
+ *  - the fit is the asymmetric min-max one with an integer zero point,
+ *    in fp32 with each rounding stated (rint = nearest, ties to even):
+ *      range = fl32(max - min)
+ *      s = max(fl32(range / 255), FLT_MIN)     when range > 0
+ *      s = max(|min|, FLT_MIN)                 for a constant group
+ *      z = rint(fl32(-min / s)) + 0            (+0, never -0)
+ *      q = min(255, max(0, rint(fl32(fl32(x / s) + z))))   (NaN -> 0)
+ *    so the group's minimum gets code 0, its maximum 255 or 254 (the
+ *    rounded zero point moves the grid by at most half a step), and a
+ *    constant group is reproduced exactly;
+ *  - dequantize: x' = bf16(fl32(fl32(q - z) * s)) (q - z is exact).
+ * The values must be finite with max - min finite in fp32. */
+static void kv8_fit(float mn, float mx, float* s_out, float* z_out) {
+    float range = mx - mn, s;
+    if (range > 0.0f) {
+        s = range / 255.0f;
+        if (s < FLT_MIN) s = FLT_MIN;
+    } else {
+        s = fabsf(mn);
+        if (s < FLT_MIN) s = FLT_MIN;
+    }
+    *s_out = s;
+    *z_out = rintf(-mn / s) + 0.0f;
+}
+
+static uint8_t kv8_code(float x, float s, float z) {
+    float t = x / s;
+    t = t + z;
+    float q = rintf(t);
+    q = fmaxf(q, 0.0f); /* NaN -> 0 */
+    q = fminf(q, 255.0f);
+    return (uint8_t)q;
+}
+
+void orc_kv8_quantize(const uint16_t* KV, int64_t T, int64_t H, int64_t D, uint8_t* Q, float* scale, float* zero) {
+    const int64_t C = H * D, G = T / 64;
+    int64_t gc;
+#pragma omp parallel for schedule(static)
+    for (gc = 0; gc < G * C; ++gc) {
+        const int64_t g = gc / C, c = gc % C;
+        const uint16_t* x = KV + g * 64 * C + c; /* token 64g, column c */
+        float mn = orc_bf16_to_f32(x[0]), mx = mn, s, z;
+        int t;
+        for (t = 1; t < 64; ++t) {
+            float v = orc_bf16_to_f32(x[t * C]);
+            if (v < mn) mn = v;
+            if (v > mx) mx = v;
+        }
+        kv8_fit(mn, mx, &s, &z);
+        for (t = 0; t < 64; ++t) Q[(g * 64 + t) * C + c] = kv8_code(orc_bf16_to_f32(x[t * C]), s, z);
+        scale[gc] = s;
+        zero[gc] = z;
+    }
+}
+
+/* The cache read (the README's KV8 caveat: the quantized history is
+ * dequantized and the bf16 tail appended): out [Tq + Tr][H][D] holds the Tq
+ * quantized tokens dequantized, then the Tr residual tokens as they are. */
+void orc_kv8_read(const uint8_t* Q, const float* scale, const float* zero, int64_t Tq, const uint16_t* resid,
+                  int64_t Tr, int64_t H, int64_t D, uint16_t* out) {
+    const int64_t C = H * D;
+    int64_t i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < Tq * C; ++i) {
+        const int64_t t = i / C, c = i % C, gc = (t / 64) * C + c;
+        const float d = (float)Q[i] - zero[gc];
+        out[i] = orc_f32_to_bf16(d * scale[gc]);
+    }
+    memcpy(out + Tq * C, resid, (size_t)(Tr * C) * sizeof(uint16_t));
+}
+
+/* How many of the T positions a cache holds quantized (reading of
+ * residual_length 128 with groups of 64 along the tokens): the latest 128
+ * positions always stay bf16, and older ones are quantized in whole groups,
+ * so Tq = 64 * floor((T - 128) / 64) for T >= 128, else 0. */
+int64_t orc_kv8_history_tokens(int64_t T) {
+    return T < 128 ? 0 : 64 * ((T - 128) / 64);
+}
+
 /* ------------------------------------- producers of the activations -- */
 
 /* RMSNorm, the producer of the q/k/v and gate/up inputs ("MOSS-VL-Realtime-FP8

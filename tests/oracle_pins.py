@@ -353,6 +353,134 @@ def pin_kv_cache(o, seed=14):
     assert np.array_equal(bits_to_f32(out2).astype(np.float64), exact)
 
 
+# ------------------------------------------------------- INT8 KV cache --
+
+def _kv8_grid_case(rng, H=3, D=8):
+    """128 tokens x H x D values on exact grids: in every column and group,
+    token values (k - m) * 2^-e for a permutation k of 64 distinct codes that
+    include 0 and 255, with m in [0, 255] and e per column and group.  Every
+    value has at most 8 significant bits (bf16-exact), the range is 255 * 2^-e,
+    so the fit is s = 2^-e, z = m, and the codes are k: no rounding anywhere."""
+    G = 2
+    k = np.empty((G * 64, H, D), np.int64)
+    m = rng.integers(0, 256, (G, H, D))
+    e = rng.integers(-20, 30, (G, H, D))
+    for g in range(G):
+        for h in range(H):
+            for d in range(D):
+                pick = np.concatenate([[0, 255], rng.choice(np.arange(1, 255), 62, replace=False)])
+                k[g * 64:(g + 1) * 64, h, d] = rng.permutation(pick)
+    mt = np.repeat(m, 64, axis=0)
+    et = np.repeat(e, 64, axis=0)
+    x = (k - mt) * np.exp2(-et.astype(np.float64))
+    xb = bf16_bits(x.astype(np.float32))
+    assert np.array_equal(bits_to_f32(xb).astype(np.float64), x), "grid values must be bf16-exact"
+    return xb, k, np.exp2(-e.astype(np.float64)).astype(np.float32), m.astype(np.float32)
+
+
+def pin_kv8_grid(o, seed=17):
+    """Closed form of the min-max fit on grid-valued groups (a group is 64
+    tokens of one column): scale 2^-e, zero m, codes k, and the read returns
+    the inputs exactly.  A group formed along another axis, another divisor
+    than 255, a flipped zero or a wrong dequantize formula all fail it."""
+    rng = np.random.default_rng(seed)
+    xb, k, s_ref, z_ref = _kv8_grid_case(rng)
+    q, s, z = o.kv8_quantize(xb)
+    assert np.array_equal(s, s_ref), "scale is not 2^-e"
+    assert np.array_equal(z, z_ref), "zero is not m"
+    assert np.array_equal(q.astype(np.int64), k), f"{(q != k).sum()} codes differ from the grid index"
+    out = o.kv8_read(q, s, z, np.zeros((0,) + xb.shape[1:], np.uint16))
+    assert np.array_equal(out, xb), "the read does not return grid values exactly"
+
+
+def pin_kv8_ties(o, seed=18):
+    """Half-way values round to the even code: groups of one column hold the
+    minimum -m s, the maximum (255 - m) s and values (j + 1/2) s in between
+    (s a power of two, |j + 1/2| < 128, so x / s + m is exact)."""
+    rng = np.random.default_rng(seed)
+    H, D = 2, 4
+    x = np.empty((64, H, D), np.float64)
+    want = np.empty((64, H, D), np.int64)
+    for h in range(H):
+        for d in range(D):
+            m = int(rng.integers(64, 192))
+            s = 2.0 ** int(rng.integers(-10, 10))
+            lo, hi = max(-m, -127), min(255 - m - 1, 126)
+            j = rng.integers(lo, hi + 1, 62)
+            x[:, h, d] = np.concatenate([[-m * s, (255 - m) * s], (j + 0.5) * s])
+            # x / s + m = j + m + 1/2 rounds to the even one of j + m and j + m + 1
+            want[:, h, d] = np.concatenate([[0, 255], np.where((j + m) % 2 == 0, j + m, j + m + 1)])
+    xb = bf16_bits(x.astype(np.float32))
+    assert np.array_equal(bits_to_f32(xb).astype(np.float64), x), "tie values must be bf16-exact"
+    q, _, _ = o.kv8_quantize(xb)
+    assert np.array_equal(q.astype(np.int64), want), f"{(q != want).sum()} half-way codes not rounded to even"
+
+
+def pin_kv8_invariants(o, seed=19):
+    """Random groups: the minimum takes code 0 and the maximum 254 or 255 (the
+    rounded zero point shifts the grid by at most half a step), codes are
+    monotone in x within a group, the read is within half a step (s / 2) plus
+    half a bf16 unit of x, permuting tokens inside a group permutes the codes
+    and keeps the fit, a change to one value moves only its own group, and a
+    constant group (0, small, negative, huge) is reproduced exactly."""
+    rng = np.random.default_rng(seed)
+    T, H, D = 192, 4, 16
+    x = (rng.standard_normal((T, H, D)) * np.exp2(rng.uniform(-6, 6, (1, H, D)))
+         + rng.uniform(-3, 3, (1, H, D))).astype(np.float32)
+    xb = bf16_bits(x)
+    xf = bits_to_f32(xb).astype(np.float64)
+    q, s, z = o.kv8_quantize(xb)
+    qi = q.astype(np.int64)
+    for g in range(T // 64):
+        blk, qb = xf[g * 64:(g + 1) * 64], qi[g * 64:(g + 1) * 64]
+        amin, amax = blk.argmin(axis=0), blk.argmax(axis=0)
+        assert np.all(np.take_along_axis(qb, amin[None], 0) == 0), "minimum is not code 0"
+        top = np.take_along_axis(qb, amax[None], 0)
+        assert np.all((top == 255) | (top == 254)), "maximum is not code 254 or 255"
+        order = np.argsort(blk, axis=0, kind="stable")
+        assert np.all(np.diff(np.take_along_axis(qb, order, 0), axis=0) >= 0), "codes not monotone in x"
+    out = bits_to_f32(o.kv8_read(q, s, z, np.zeros((0, H, D), np.uint16))).astype(np.float64)
+    srep = np.repeat(s, 64, axis=0).astype(np.float64)
+    bound = 0.5 * srep * (1 + 2.0 ** -12) + np.abs(out) * 2.0 ** -8  # half a step + half a bf16 unit
+    assert np.all(np.abs(out - xf) <= bound), "read farther than half a step from x"
+    perm = np.concatenate([rng.permutation(64) + 64 * g for g in range(T // 64)])
+    qp, sp, zp = o.kv8_quantize(xb[perm])
+    assert np.array_equal(qp, q[perm]) and np.array_equal(sp, s) and np.array_equal(zp, z)
+    xb2 = xb.copy()
+    xb2[70, 1, 3] = bf16_bits(np.float32([1e4]))[0]
+    q2, s2, z2 = o.kv8_quantize(xb2)
+    changed = np.argwhere(s2 != s)
+    assert changed.tolist() == [[1, 1, 3]], f"one value changed groups {changed.tolist()}"
+    mask = np.ones_like(q, bool)
+    mask[64:128, 1, 3] = False
+    assert np.array_equal(q2[mask], q[mask])
+    for c in (0.0, 1.5, -3.0e-30, -7.0, 2.0e30):
+        cb = bf16_bits(np.full((64, 1, 2), c, np.float32))
+        qc, sc, zc = o.kv8_quantize(cb)
+        assert np.all(qc == qc.flat[0]), f"constant group {c}: codes differ"
+        assert np.array_equal(o.kv8_read(qc, sc, zc, np.zeros((0, 1, 2), np.uint16)), cb), f"constant {c} not exact"
+
+
+def pin_kv8_read_and_tail(o, seed=20):
+    """The read is the dequantized history followed by the bf16 tail,
+    bit for bit; the number of quantized positions keeps the latest 128
+    positions in bf16 and quantizes older ones in whole groups of 64, no
+    more than 191 positions staying bf16."""
+    rng = np.random.default_rng(seed)
+    H, D = 2, 8
+    xb, k, s_ref, z_ref = _kv8_grid_case(rng, H, D)
+    tail = bf16_bits(rng.standard_normal((37, H, D)).astype(np.float32))
+    q, s, z = o.kv8_quantize(xb)
+    out = o.kv8_read(q, s, z, tail)
+    assert out.shape == (128 + 37, H, D)
+    assert np.array_equal(out[:128], xb) and np.array_equal(out[128:], tail), "history or tail misplaced"
+    for T in range(0, 1200):
+        tq = o.kv8_history_tokens(T)
+        assert tq % 64 == 0 and 0 <= tq <= T, (T, tq)
+        assert T - tq >= min(T, 128), f"T={T}: fewer than the latest 128 positions in bf16"
+        assert T - tq < 192, f"T={T}: a whole group older than the latest 128 is left in bf16"
+
+
 # ------------------------------------------------------------ producers --
 
 def pin_rmsnorm(o, seed=15):
@@ -391,4 +519,4 @@ def pin_silu_mul(o, seed=16):
 ALL_PINS = [pin_decode_table, pin_roundtrip, pin_rounding_cases, pin_encode_vs_library,
             pin_saturation, pin_scale_invariants, pin_scale_and_quotient_rounding, pin_gemm_bruteforce,
             pin_gemm_int_vs_fp, pin_onehot_closed_form, pin_bf16_rounding, pin_kv_cache,
-            pin_rmsnorm, pin_silu_mul]
+            pin_rmsnorm, pin_silu_mul, pin_kv8_grid, pin_kv8_ties, pin_kv8_invariants, pin_kv8_read_and_tail]

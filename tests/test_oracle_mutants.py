@@ -57,6 +57,24 @@ MUTANTS = {
     # gate and up swapped
     "silu_swap": ("double gv = (double)orc_bf16_to_f32(GU[m * 2 * I + k]);",
                   "double gv = (double)orc_bf16_to_f32(GU[m * 2 * I + I + k]);"),
+    # INT8 KV cache: another divisor than 255 for the scale
+    "kv8_div256": ("        s = range / 255.0f;", "        s = range / 256.0f;"),
+    # INT8 KV cache: zero point with the wrong sign
+    "kv8_zero_sign": ("*z_out = rintf(-mn / s) + 0.0f;", "*z_out = rintf(mn / s) + 0.0f;"),
+    # INT8 KV cache: ties away from zero
+    "kv8_ties_away": ("    float q = rintf(t);", "    float q = roundf(t);"),
+    # INT8 KV cache: truncation instead of rounding
+    "kv8_trunc": ("    float q = rintf(t);", "    float q = truncf(t);"),
+    # INT8 KV cache: groups along head_dim instead of the tokens
+    "kv8_axis": ("float v = orc_bf16_to_f32(x[t * C]);", "float v = orc_bf16_to_f32(x[t]);"),
+    # INT8 KV cache: a constant group with scale 1
+    "kv8_const": ("        s = fabsf(mn);", "        s = 1.0f;"),
+    # INT8 KV cache: dequantize adds the zero point
+    "kv8_read_sign": ("const float d = (float)Q[i] - zero[gc];", "const float d = (float)Q[i] + zero[gc];"),
+    # INT8 KV cache: the tail written over the history
+    "kv8_tail_place": ("memcpy(out + Tq * C, resid,", "memcpy(out, resid,"),
+    # INT8 KV cache: partial groups quantized
+    "kv8_partial_group": ("return T < 128 ? 0 : 64 * ((T - 128) / 64);", "return T < 128 ? 0 : T - 128;"),
     # saturation missing (values above 448 become NaN)
     "no_satfinite": ("if (a >= 448.0) return (uint8_t)(sign | 0x7E);", "if (a >= 464.0) return (uint8_t)(sign | 0x7F);"),
 }
