@@ -469,6 +469,56 @@ def kv_cache_line(torch, mfp8, W, device, steps, warmup, peaks):
     return res
 
 
+def kv8_cache_line(torch, mfp8, W, device, steps, warmup, peaks):
+    """The INT8 KV cache (the README's KV8 section: hqq backend, nbits 8,
+    group 64 along the tokens, residual 128): a cache of T = 16384 positions,
+    8 KV heads x 128, holds 16256 positions quantized and the latest 128 in
+    bf16.  Timed: quantizing the 16256-position history (a prefill filling the
+    cache) and reading the whole cache back (dequantize + the bf16 tail).
+    Eight tensors (K and V of four layers, 8 x 32 MB, more than L2) and
+    eight outputs are cycled.  GB/s of algorithmic bytes: quantize 2 + 1 bytes per value + 8 per
+    group and column, read 1 + 2 per history value + 8 per group and column +
+    2 + 2 per tail value."""
+    T, H, D, n = 16384, 8, 128, 8
+    Tq = mfp8.mfp8_kv8_history_tokens(T)
+    Tr, C = T - Tq, H * D
+    kv = [W.make_kv(T, H, D, seed=8, stream=i, device=device) for i in range(n)]
+    q = [torch.empty((Tq, H, D), dtype=torch.uint8, device=device) for _ in kv]
+    sc = [torch.empty((Tq // 64, H, D), dtype=torch.float32, device=device) for _ in kv]
+    zp = [torch.empty((Tq // 64, H, D), dtype=torch.float32, device=device) for _ in kv]
+    out = [torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for _ in range(n)]
+    torch.cuda.synchronize()
+
+    def quant(h):
+        for a, b, c, z in zip(kv, q, sc, zp):
+            st = mfp8.mfp8_kv8_quantize(a.data_ptr(), Tq, H, D, b.data_ptr(), c.data_ptr(), z.data_ptr(), h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_kv8_quantize")
+
+    def read(h):
+        for i, (a, b, c, z) in enumerate(zip(kv, q, sc, zp)):
+            st = mfp8.mfp8_kv8_read(b.data_ptr(), c.data_ptr(), z.data_ptr(), Tq, a[Tq:].data_ptr(), Tr, H, D,
+                                    out[i].data_ptr(), h)
+            if st != mfp8.OK:
+                raise mfp8.Mfp8Error(st, "mfp8_kv8_read")
+
+    res = {"workload": f"K and V of a cache of T={T} positions x 8 KV heads x 128 (long video context): "
+                       f"{Tq} positions quantized in groups of 64 tokens, the latest {Tr} in bf16; 8 tensors "
+                       "cycled (> L2)"}
+    fits = (Tq // 64) * C * 8
+    for name, fn, nbytes in (("quantize", quant, Tq * C * 3 + fits),
+                             ("read", read, Tq * C * 3 + fits + Tr * C * 4)):
+        ms = time_graph(torch, fn, steps, warmup, None)
+        us = ms * 1e3 / (steps * n)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"GB/s": round(gbs, 1), "avg_launch_us": round(us, 3), "bytes_per_launch": nbytes,
+                     "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    assert mfp8.device_status() == mfp8.OK
+    del kv, q, sc, zp, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def producers_line(torch, mfp8, W, device, steps, warmup, peaks):
     """The activation quantization fused into its producers at the prefill
     size M = 2048: RMSNorm + quantize (hidden 4096; reads the bf16 rows and
@@ -911,6 +961,7 @@ def main():
     config0 = q_proj_m16(torch, mfp8, W, device, max(5, args.steps), args.warmup, ctx, peaks)
     torch.cuda.empty_cache()
     kv_cache = kv_cache_line(torch, mfp8, W, device, max(5, min(args.steps, 20)), args.warmup, peaks)
+    kv8_cache = kv8_cache_line(torch, mfp8, W, device, max(5, min(args.steps, 20)), args.warmup, peaks)
     producers = producers_line(torch, mfp8, W, device, max(5, min(args.steps, 20)), args.warmup, peaks)
 
     stack = None
@@ -946,6 +997,7 @@ def main():
         "clocks": clk,
         "q_proj_m16": config0,
         "kv_cache_fp8": kv_cache,
+        "kv_cache_int8": kv8_cache,
         "fused_producers": producers,
         "prefill": prefill,
         "layer_prefill_fused_producers": fused_layer,

@@ -20,6 +20,7 @@
 #include "gemm_stream.cuh"
 #include "gemm_cluster.cuh"
 #include "producer.cuh"
+#include "kv8.cuh"
 
 namespace mfp8 {
 namespace {
@@ -731,6 +732,29 @@ mfp8_status launch_producer(int64_t nvec, int64_t M, cudaStream_t stream, A... a
     return MFP8_ERR_UNSUPPORTED_SHAPE;
 }
 
+// A launch that may begin while the previous kernel on the stream drains
+// (programmatic dependent launch); the kernel waits for that kernel's
+// results with griddepcontrol.wait before its first global load.
+template <typename... KArgs, typename... A>
+mfp8_status launch_pdl(void (*kern)(KArgs...), dim3 grid, int threads, cudaStream_t stream, int smem_bytes,
+                       A... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = size_t(smem_bytes);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return MFP8_ERR_CUDA;
+    }
+    return MFP8_OK;
+}
+
 template <int VPT>
 struct PickRmsnorm {
     static auto kern() { return producer::rmsnorm_quant_kernel<VPT>; }
@@ -968,12 +992,91 @@ mfp8_status mfp8_kv_dequantize(const void* KV_fp8, const float* kv_scale, int64_
     DeviceInfo info;
     mfp8_status st = current_device(&dev, &info);
     if (st != MFP8_OK) return st;
-    const int64_t n16 = R * D / 16;
-    int64_t blocks = (n16 + kQuantThreads - 1) / kQuantThreads;
-    const int64_t cap = int64_t(info.sm_count) * 8;
-    if (blocks > cap) blocks = cap;
-    kv_dequant_kernel<<<unsigned(blocks), kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4*>(KV_fp8), kv_scale, n16, int(D), static_cast<uint4*>(KV_bf16));
+    const int64_t n8 = R * D / 8;
+    const int64_t blocks = (n8 + kQuantThreads * kDequantItems - 1) / (kQuantThreads * kDequantItems);
+    if (blocks > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    return launch_pdl(kv_dequant_kernel, dim3(unsigned(blocks)), kQuantThreads, static_cast<cudaStream_t>(stream), 0,
+                      static_cast<const uint2*>(KV_fp8), kv_scale, n8, int(D), static_cast<uint4*>(KV_bf16));
+}
+
+mfp8_status mfp8_kv8_quantize(const void* KV_bf16, int64_t T, int64_t H, int64_t D, void* KV_u8, float* kv_scale,
+                              float* kv_zero, void* stream) {
+    if (T < 0 || H < 0 || D < 0) return MFP8_ERR_INVALID_ARG;
+    if (H == 0 || D == 0 || D % 16 != 0 || T % kv8::kGroup != 0 || D > kMaxDim || H > kMaxDim || T > kMaxDim)
+        return MFP8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t C = H * D;
+    if (C > kMaxDim || (T > 0 && C > (int64_t(1) << 40) / T)) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MFP8_OK;
+    if (!KV_bf16 || !KV_u8 || !kv_scale || !kv_zero) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(KV_bf16) || !aligned16(KV_u8) || !aligned16(kv_scale) || !aligned16(kv_zero))
+        return MFP8_ERR_MISALIGNED;
+    const int64_t G = T / kv8::kGroup;
+    const size_t nin = size_t(T * C) * 2, nq = size_t(T * C), nf = size_t(G * C) * 4;
+    if (ranges_overlap(KV_bf16, nin, KV_u8, nq) || ranges_overlap(KV_bf16, nin, kv_scale, nf) ||
+        ranges_overlap(KV_bf16, nin, kv_zero, nf) || ranges_overlap(KV_u8, nq, kv_scale, nf) ||
+        ranges_overlap(KV_u8, nq, kv_zero, nf) || ranges_overlap(kv_scale, nf, kv_zero, nf))
+        return MFP8_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    const int64_t tiles_per_group = (C + kv8::kTileCols - 1) / kv8::kTileCols;
+    const int64_t blocks = G * tiles_per_group;
+    if (blocks > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    return launch_pdl(kv8::quant_kernel, dim3(unsigned(blocks)), kv8::kQuantThreads, static_cast<cudaStream_t>(stream), 0,
+                      static_cast<const uint4*>(KV_bf16), C / 8, tiles_per_group, static_cast<uint2*>(KV_u8), kv_scale,
+                      kv_zero);
+}
+
+mfp8_status mfp8_kv8_read(const void* KV_u8, const float* kv_scale, const float* kv_zero, int64_t Tq,
+                          const void* tail_bf16, int64_t Tr, int64_t H, int64_t D, void* out_bf16, void* stream) {
+    if (Tq < 0 || Tr < 0 || H < 0 || D < 0) return MFP8_ERR_INVALID_ARG;
+    if (H == 0 || D == 0 || D % 16 != 0 || Tq % kv8::kGroup != 0 || D > kMaxDim || H > kMaxDim || Tq > kMaxDim ||
+        Tr > kMaxDim)
+        return MFP8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t C = H * D, T = Tq + Tr;
+    if (C > kMaxDim || (T > 0 && C > (int64_t(1) << 40) / T)) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MFP8_OK;
+    if (!out_bf16 || (Tq > 0 && (!KV_u8 || !kv_scale || !kv_zero)) || (Tr > 0 && !tail_bf16))
+        return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(out_bf16) || !aligned16(KV_u8) || !aligned16(kv_scale) || !aligned16(kv_zero) ||
+        !aligned16(tail_bf16))
+        return MFP8_ERR_MISALIGNED;
+    const size_t nout = size_t(T * C) * 2, nq = size_t(Tq * C), nf = size_t(Tq / kv8::kGroup * C) * 4,
+                 nt = size_t(Tr * C) * 2;
+    if ((Tq > 0 && (ranges_overlap(out_bf16, nout, KV_u8, nq) || ranges_overlap(out_bf16, nout, kv_scale, nf) ||
+                    ranges_overlap(out_bf16, nout, kv_zero, nf))) ||
+        (Tr > 0 && ranges_overlap(out_bf16, nout, tail_bf16, nt)))
+        return MFP8_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    const int64_t C8 = C / 8, n_tail16 = Tr * C / 8;
+    const int64_t items = Tq / kv8::kReadRows * C8 + n_tail16;
+    const int64_t blocks = (items + kv8::kReadThreads - 1) / kv8::kReadThreads;
+    if (blocks > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
+    return launch_pdl(kv8::read_kernel, dim3(unsigned(blocks)), kv8::kReadThreads, static_cast<cudaStream_t>(stream), 0,
+                      static_cast<const uint2*>(KV_u8), reinterpret_cast<const float4*>(kv_scale),
+                      reinterpret_cast<const float4*>(kv_zero), Tq, C8, static_cast<const uint4*>(tail_bf16),
+                      n_tail16, static_cast<uint4*>(out_bf16));
+}
+
+int64_t mfp8_kv8_history_tokens(int64_t T) {
+    if (T < 0) return -1;
+    return T < 128 ? 0 : kv8::kGroup * ((T - 128) / kv8::kGroup);
+}
+
+mfp8_status mfp8_debug_kv8_code_check(void* out_u64x2, int64_t n_scale_pairs, uint32_t seed, void* stream) {
+    if (!out_u64x2 || n_scale_pairs <= 0 || n_scale_pairs > INT32_MAX) return MFP8_ERR_INVALID_ARG;
+    if (!aligned16(out_u64x2)) return MFP8_ERR_MISALIGNED;
+    int dev;
+    DeviceInfo info;
+    mfp8_status st = current_device(&dev, &info);
+    if (st != MFP8_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(out_u64x2, 0, 16, s) != cudaSuccess) return MFP8_ERR_CUDA;
+    kv8::code_check_kernel<<<unsigned(n_scale_pairs), 256, 0, s>>>(static_cast<unsigned long long*>(out_u64x2), seed);
     return launch_status();
 }
 

@@ -319,23 +319,34 @@ __device__ __forceinline__ uint32_t dequant2(uint16_t codes2, float s) {
     return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// Dequantize: each thread takes kDequantItems items of 8 codes (an 8-byte
+// load) -> 8 bf16 (one 16-byte store), items blockDim.x apart, so a warp's
+// store covers 512 contiguous bytes, whole sectors; all of a thread's loads
+// are issued before its arithmetic.  n8 = R * D / 8.  A programmatic
+// dependent: the codes may be the previous kernel's output.
+constexpr int kDequantItems = 4;
+
 __global__ void __launch_bounds__(kQuantThreads)
-kv_dequant_kernel(const uint4* __restrict__ Q, const float* __restrict__ S, int64_t n16, int D,
+kv_dequant_kernel(const uint2* __restrict__ Q, const float* __restrict__ S, int64_t n8, int D,
                   uint4* __restrict__ out) {
-    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-    const int g16 = D >> 4;  // 16-code groups per row
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride) {
-        const uint4 q = __ldg(Q + i);
-        const float s = __ldg(S + i / g16);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-        uint32_t o[8];
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const int g8 = D >> 3;  // 8-code groups per row
+    const int64_t base = int64_t(blockIdx.x) * (kQuantThreads * kDequantItems) + threadIdx.x;
+    uint2 q[kDequantItems];
+    float s[kDequantItems];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            o[2 * j] = dequant2(uint16_t(w[j] & 0xffffu), s);
-            o[2 * j + 1] = dequant2(uint16_t(w[j] >> 16), s);
-        }
-        out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
-        out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    for (int k = 0; k < kDequantItems; ++k) {
+        const int64_t i = base + k * kQuantThreads;
+        q[k] = i < n8 ? __ldcs(Q + i) : make_uint2(0u, 0u);
+        s[k] = i < n8 ? __ldg(S + i / g8) : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < kDequantItems; ++k) {
+        const int64_t i = base + k * kQuantThreads;
+        if (i < n8)
+            __stcs(out + i, make_uint4(dequant2(uint16_t(q[k].x & 0xffffu), s[k]), dequant2(uint16_t(q[k].x >> 16), s[k]),
+                                       dequant2(uint16_t(q[k].y & 0xffffu), s[k]), dequant2(uint16_t(q[k].y >> 16), s[k])));
     }
 }
 

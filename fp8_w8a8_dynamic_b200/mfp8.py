@@ -61,6 +61,10 @@ def lib():
             "mfp8_silu_mul_quantize": (i32, [P, i64, i64, P, P, P, P]),
             "mfp8_kv_quantize": (i32, [P, i64, i64, i64, P, P, P]),
             "mfp8_kv_dequantize": (i32, [P, P, i64, i64, i64, P, P]),
+            "mfp8_kv8_quantize": (i32, [P, i64, i64, i64, P, P, P, P]),
+            "mfp8_kv8_read": (i32, [P, P, P, i64, P, i64, i64, i64, P, P]),
+            "mfp8_kv8_history_tokens": (i64, [i64]),
+            "mfp8_debug_kv8_code_check": (i32, [P, i64, ctypes.c_uint32, P]),
             "mfp8_e4m3_encode_f32": (i32, [P, i64, P, P]),
             "mfp8_debug_quantize_check": (i32, [P, P]),
             "mfp8_debug_bounded_wait": (i32, [i64, P]),
@@ -139,6 +143,22 @@ def mfp8_kv_quantize(KV_bf16, T, H, D, KV_fp8, kv_scale, stream=0):
 
 def mfp8_kv_dequantize(KV_fp8, kv_scale, T, H, D, KV_bf16, stream=0):
     return lib().mfp8_kv_dequantize(KV_fp8, kv_scale, T, H, D, KV_bf16, stream)
+
+
+def mfp8_kv8_quantize(KV_bf16, T, H, D, KV_u8, kv_scale, kv_zero, stream=0):
+    return lib().mfp8_kv8_quantize(KV_bf16, T, H, D, KV_u8, kv_scale, kv_zero, stream)
+
+
+def mfp8_kv8_read(KV_u8, kv_scale, kv_zero, Tq, tail_bf16, Tr, H, D, out_bf16, stream=0):
+    return lib().mfp8_kv8_read(KV_u8, kv_scale, kv_zero, Tq, tail_bf16, Tr, H, D, out_bf16, stream)
+
+
+def mfp8_kv8_history_tokens(T):
+    return lib().mfp8_kv8_history_tokens(T)
+
+
+def mfp8_debug_kv8_code_check(out, n_scale_pairs, seed, stream=0):
+    return lib().mfp8_debug_kv8_code_check(out, n_scale_pairs, seed, stream)
 
 
 def mfp8_e4m3_encode_f32(inp, n, out, stream=0):
@@ -291,6 +311,79 @@ def kv_dequantize(codes, scales, stream=None):
     _check(mfp8_kv_dequantize(_ptr(codes), _ptr(scales), T, H, D, _ptr(out), _stream_handle(stream)),
            "mfp8_kv_dequantize")
     return out
+
+
+def kv8_quantize(KV, stream=None):
+    """KV: bf16 [T, H, D] CUDA tensor, T % 64 == 0 -> (codes uint8 [T, H, D],
+    scale fp32 [T/64, H, D], zero fp32 [T/64, H, D])."""
+    import torch
+    T, H, D = KV.shape
+    codes = torch.empty((T, H, D), dtype=torch.uint8, device=KV.device)
+    scale = torch.empty((T // 64, H, D), dtype=torch.float32, device=KV.device)
+    zero = torch.empty((T // 64, H, D), dtype=torch.float32, device=KV.device)
+    _check(mfp8_kv8_quantize(_ptr(KV), T, H, D, _ptr(codes), _ptr(scale), _ptr(zero), _stream_handle(stream)),
+           "mfp8_kv8_quantize")
+    return codes, scale, zero
+
+
+def kv8_read(codes, scale, zero, tail, out=None, stream=None):
+    """History (codes [Tq, H, D], scale and zero [Tq/64, H, D]) and bf16 tail
+    [Tr, H, D] -> bf16 [Tq + Tr, H, D]: the history dequantized, then the
+    tail."""
+    import torch
+    Tq, H, D = codes.shape
+    Tr = tail.shape[0]
+    if out is None:
+        out = torch.empty((Tq + Tr, H, D), dtype=torch.bfloat16, device=codes.device)
+    _check(mfp8_kv8_read(_ptr(codes), _ptr(scale), _ptr(zero), Tq, _ptr(tail), Tr, H, D, _ptr(out),
+                         _stream_handle(stream)), "mfp8_kv8_read")
+    return out
+
+
+class Kv8Cache:
+    """One K or V tensor of a layer held as the INT8 cache: a history of
+    whole 64-token groups (codes, scale, zero) and the bf16 tail of the
+    latest positions.  Buffers are allocated once for `capacity` positions.
+    ``append`` stages the old tail and the new positions in one bf16 buffer,
+    quantizes the positions that mfp8_kv8_history_tokens moves into the
+    history (mfp8_kv8_quantize, written in place after the existing groups)
+    and keeps the rest as the tail; ``read`` returns every position as bf16
+    (mfp8_kv8_read).  Work is queued on the current torch stream."""
+
+    def __init__(self, capacity, H, D, device):
+        import torch
+        groups = (capacity + 63) // 64
+        self.capacity, self.H, self.D = capacity, H, D
+        self.codes = torch.empty((groups * 64, H, D), dtype=torch.uint8, device=device)
+        self.scale = torch.empty((groups, H, D), dtype=torch.float32, device=device)
+        self.zero = torch.empty((groups, H, D), dtype=torch.float32, device=device)
+        self.tail = torch.empty((0, H, D), dtype=torch.bfloat16, device=device)
+        self.T = 0
+
+    @property
+    def Tq(self):
+        return mfp8_kv8_history_tokens(self.T)
+
+    def append(self, kv):
+        import torch
+        n = kv.shape[0]
+        if kv.shape[1:] != (self.H, self.D) or kv.dtype != torch.bfloat16:
+            raise ValueError("Kv8Cache.append: expected bf16 [n, H, D]")
+        if self.T + n > self.capacity:
+            raise ValueError("Kv8Cache.append: capacity exceeded")
+        tq, tq2 = self.Tq, mfp8_kv8_history_tokens(self.T + n)
+        staged = torch.cat([self.tail, kv]) if self.tail.shape[0] else kv.contiguous()
+        f = tq2 - tq
+        if f:
+            g = tq // 64
+            _check(mfp8_kv8_quantize(_ptr(staged), f, self.H, self.D, _ptr(self.codes[tq]), _ptr(self.scale[g]),
+                                     _ptr(self.zero[g]), _stream_handle(None)), "mfp8_kv8_quantize")
+        self.tail = staged[f:].clone()
+        self.T += n
+
+    def read(self, out=None):
+        tq = self.Tq
+        return kv8_read(self.codes[:tq], self.scale[:tq // 64], self.zero[:tq // 64], self.tail, out=out)
 
 
 def e4m3_encode(values, stream=None):

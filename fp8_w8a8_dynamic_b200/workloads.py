@@ -88,6 +88,22 @@ def make_x(M: int, K: int, seed: int, stream: int = 0, kind: str = "normal",
     return x.to(torch.bfloat16)
 
 
+def make_kv(T: int, H: int, D: int, seed: int, stream: int = 0, device="cpu") -> torch.Tensor:
+    """Keys or values [T, H, D] BF16 for a cache whose groups run along the
+    tokens: per (head, channel) column an offset ~ U(-2, 2) and a log-uniform
+    spread in [0.1, 10] around it (so groups are asymmetric and of unequal
+    width), N(0, 1) per token, and 0.1% outliers x50."""
+    g = generator(seed, 20_000 + stream, device)
+    x = torch.randn(T, H, D, generator=g, device=device, dtype=torch.float32)
+    u = torch.rand(1, H, D, generator=g, device=device, dtype=torch.float32)
+    off = torch.rand(1, H, D, generator=g, device=device, dtype=torch.float32) * 4.0 - 2.0
+    lo, hi = math.log(0.1), math.log(10.0)
+    x = x * torch.exp(lo + u * (hi - lo)) + off
+    mask = torch.rand(T, H, D, generator=g, device=device, dtype=torch.float32) < 0.001
+    x = torch.where(mask, x * 50.0, x)
+    return x.to(torch.bfloat16)
+
+
 def make_w(N: int, K: int, seed: int, stream: int = 0, std: float = 0.02,
            device="cpu") -> torch.Tensor:
     """Weights [N, K] BF16 in the Linear's (out_features, in_features) layout."""

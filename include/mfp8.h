@@ -245,6 +245,57 @@ MFP8_API mfp8_status mfp8_kv_quantize(const void* KV_bf16, int64_t T, int64_t H,
 MFP8_API mfp8_status mfp8_kv_dequantize(const void* KV_fp8, const float* kv_scale, int64_t T, int64_t H,
                                int64_t D, void* KV_bf16, void* stream);
 
+/* ------------------------------------------------------ INT8 KV cache -- */
+
+/* The INT8 KV cache ("MOSS-VL quantization README", KV8 section: the hqq
+ * backend with nbits 8, axis_key = axis_value = 0, q_group_size 64 and
+ * residual_length 128; the history lives quantized and the bf16 tail of the
+ * latest positions is appended when it is read).  The section gives these
+ * settings, not HQQ's optimizer; the readings below are this library's.
+ *
+ * A K or V tensor of one layer is [T tokens][H heads][D] bf16, C = H * D
+ * columns.  A group is 64 consecutive tokens of one column (axis 0 = the
+ * token axis); each group has one scale s and one zero point z, fp32, from
+ * the asymmetric min-max fit, every step rounded to nearest even:
+ *   range = max - min;  s = max(range / 255, FLT_MIN) if range > 0, else
+ *   max(|min|, FLT_MIN);  z = rint(-min / s) (+0 for zero);
+ *   q = min(255, max(0, rint(x / s + z)));
+ *   dequantized value = bf16((q - z) * s).
+ * Values must be finite and max - min finite in fp32.  The latest 128
+ * positions stay bf16; older ones are quantized in whole groups
+ * (mfp8_kv8_history_tokens). */
+
+/* Quantize T tokens (T a multiple of 64) into codes and fits.
+ * KV_bf16 [T][H][D] device bf16; KV_u8 [T][H][D] device u8 codes (written);
+ * kv_scale, kv_zero [T/64][H][D] device fp32 (written).  To append to a
+ * history of Tq tokens pass KV_u8 + Tq*H*D, kv_scale + (Tq/64)*H*D and
+ * kv_zero + (Tq/64)*H*D.  Asynchronous on `stream`; the caller owns every
+ * buffer.  Errors: MFP8_ERR_INVALID_ARG (negative size, null pointer,
+ * overlapping buffers), MFP8_ERR_UNSUPPORTED_SHAPE (T % 64 != 0, H or D
+ * zero, D % 16 != 0, a size above 2^31 - 1 or T*H*D above 2^40),
+ * MFP8_ERR_MISALIGNED (a pointer not 16-byte aligned).  T = 0 is a no-op. */
+MFP8_API mfp8_status mfp8_kv8_quantize(const void* KV_bf16, int64_t T, int64_t H, int64_t D, void* KV_u8,
+                                       float* kv_scale, float* kv_zero, void* stream);
+
+/* Read the cache back: out [Tq + Tr][H][D] device bf16 (written) holds the
+ * Tq history tokens (Tq a multiple of 64) dequantized, then the Tr tail
+ * tokens tail_bf16 [Tr][H][D] copied unchanged.  KV_u8, kv_scale, kv_zero
+ * as written by mfp8_kv8_quantize (may be null when Tq = 0; tail_bf16 may be
+ * null when Tr = 0).  out must not overlap the inputs.  Same errors as
+ * mfp8_kv8_quantize, with Tq % 64 != 0 unsupported.  Tq + Tr = 0 is a
+ * no-op. */
+MFP8_API mfp8_status mfp8_kv8_read(const void* KV_u8, const float* kv_scale, const float* kv_zero, int64_t Tq,
+                                   const void* tail_bf16, int64_t Tr, int64_t H, int64_t D, void* out_bf16,
+                                   void* stream);
+
+/* Host only: how many of a cache's T positions are held quantized.  The
+ * latest 128 stay bf16 and older ones are quantized in whole groups of 64:
+ * 64 * floor((T - 128) / 64) for T >= 128, 0 for 0 <= T < 128, -1 for
+ * T < 0.  After appending n positions to a cache of T, the oldest
+ * mfp8_kv8_history_tokens(T + n) - mfp8_kv8_history_tokens(T) tail
+ * positions move into the history. */
+MFP8_API int64_t mfp8_kv8_history_tokens(int64_t T);
+
 /* Diagnostic: checks the quantizer's divide-free arithmetic against IEEE
  * divides.  The scale fl32(absmax / 448) of every absmax (0 and each positive
  * finite bf16) is computed as a corrected quotient by 7 times 2^-6, and each
@@ -256,6 +307,19 @@ MFP8_API mfp8_status mfp8_kv_dequantize(const void* KV_fp8, const float* kv_scal
  * them as (absmax_bits << 16) | x_bits (x_bits 0xffff: the scale).  Read it
  * after synchronising `stream`. */
 MFP8_API mfp8_status mfp8_debug_quantize_check(void* out_u64x2, void* stream);
+
+/* Diagnostic: checks the INT8 KV cache's divide-free codes against IEEE
+ * divides.  Each of n_scale_pairs blocks draws two groups from a hash of
+ * (seed, block): a random finite bf16 minimum and a maximum that is either
+ * another random finite bf16 or a few bf16 steps above it.  Each group is
+ * fitted as mfp8_kv8_quantize fits it, and every finite bf16 x between its
+ * minimum and maximum is coded both ways, q = min(255, max(0, rint(x / s +
+ * z))); groups whose scale is below 2^-64 (coded by the divide in the
+ * kernel) are skipped.  out_u64x2 [2] device uint64, zeroed then written:
+ * [0] the number of codes that differ, [1] one of them as (scale_bits << 32)
+ * | x_bits.  n_scale_pairs in [1, 2^31 - 1].  Read it after synchronising
+ * `stream`. */
+MFP8_API mfp8_status mfp8_debug_kv8_code_check(void* out_u64x2, int64_t n_scale_pairs, uint32_t seed, void* stream);
 
 /* Diagnostic: encode n fp32 values with the device's e4m3 conversion (the
  * one the quantize kernels use).  in [n] fp32, out [n] codes.  Used to check

@@ -116,6 +116,23 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert kd(FAKE, FAKE * 2 + 4, 2, 8, 128, FAKE * 3, None) == mfp8.ERR_MISALIGNED
     assert kd(FAKE, FAKE * 2, 2, 8, 128, FAKE + 16, None) == mfp8.ERR_INVALID_ARG  # output overlaps codes
     assert kd(FAKE, FAKE * 2, 0, 8, 128, FAKE * 3, None) == mfp8.OK
+    q8, r8 = mfp8.mfp8_kv8_quantize, mfp8.mfp8_kv8_read
+    assert q8(FAKE, 100, 8, 128, FAKE * 2, FAKE * 3, FAKE * 4, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # T % 64
+    assert q8(FAKE, 64, 8, 40, FAKE * 2, FAKE * 3, FAKE * 4, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # D % 16
+    assert q8(FAKE, -64, 8, 128, FAKE * 2, FAKE * 3, FAKE * 4, None) == mfp8.ERR_INVALID_ARG
+    assert q8(FAKE, 64, 8, 128, FAKE * 2, None, FAKE * 4, None) == mfp8.ERR_INVALID_ARG
+    assert q8(FAKE, 64, 8, 128, FAKE * 2, FAKE * 3 + 4, FAKE * 4, None) == mfp8.ERR_MISALIGNED
+    assert q8(FAKE, 64, 8, 128, FAKE + 256, FAKE * 3, FAKE * 4, None) == mfp8.ERR_INVALID_ARG  # codes overlap input
+    assert q8(FAKE, 64, 8, 128, FAKE * 2, FAKE * 3, FAKE * 3 + 16, None) == mfp8.ERR_INVALID_ARG  # zero overlaps scale
+    assert q8(FAKE, 0, 8, 128, None, None, None, None) == mfp8.OK
+    assert r8(FAKE, FAKE * 2, FAKE * 3, 100, FAKE * 4, 5, 8, 128, FAKE * 5, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert r8(FAKE, FAKE * 2, FAKE * 3, 64, None, 5, 8, 128, FAKE * 5, None) == mfp8.ERR_INVALID_ARG  # no tail
+    assert r8(FAKE, FAKE * 2, FAKE * 3, 64, FAKE * 4, 5, 8, 128, None, None) == mfp8.ERR_INVALID_ARG
+    assert r8(FAKE, FAKE * 2, FAKE * 3, 64, FAKE * 4 + 2, 5, 8, 128, FAKE * 5, None) == mfp8.ERR_MISALIGNED
+    assert r8(FAKE, FAKE * 2, FAKE * 3, 64, FAKE * 4, 5, 8, 128, FAKE + 64, None) == mfp8.ERR_INVALID_ARG  # overlap
+    assert r8(None, None, None, 0, None, 0, 8, 128, None, None) == mfp8.OK
+    assert [mfp8.mfp8_kv8_history_tokens(t) for t in (-1, 0, 127, 128, 191, 192, 255, 256, 1000)] == \
+        [-1, 0, 0, 0, 0, 64, 64, 128, 832]
 
     L = mfp8.mfp8_linear_ex
     args = dict(X=FAKE, M=4, K=64, W=FAKE * 2, sw=FAKE * 3, N=64, Y=FAKE * 4, ws=FAKE * 5, wsb=1 << 16)
