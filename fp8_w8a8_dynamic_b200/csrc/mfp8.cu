@@ -227,7 +227,7 @@ mfp8_status set_smem(Kern kern, int bytes, int dev, bool* done) {
 
 template <int BN, int STAGES>
 mfp8_status launch_tiled_bn(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
-                            const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                            const float* s_w, int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info,
                             cudaStream_t stream) {
     using L = tiled::Layout<BN, STAGES>;
     auto kern = tiled::gemm_tiled_kernel<BN, STAGES>;
@@ -236,7 +236,7 @@ mfp8_status launch_tiled_bn(const void* X8, const float* s_a, int64_t M, int64_t
     if (st != MFP8_OK) return st;
     CUtensorMap tmX, tmW, tmY;
     if ((st = make_map_u8(&tmX, X8, M, K, tiled::BM)) != MFP8_OK) return st;
-    if ((st = make_map_u8(&tmW, W8, N, K, BN)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmW, W8, w_rows, K, BN)) != MFP8_OK) return st;
     if ((st = make_map_y(&tmY, Y, M, N)) != MFP8_OK) return st;
     const int64_t tiles = ((M + tiled::BM - 1) / tiled::BM) * ((N + BN - 1) / BN);
     const unsigned grid = static_cast<unsigned>(tiles < info.sm_count ? tiles : info.sm_count);
@@ -271,13 +271,13 @@ int tiled_tile_width(int64_t M, int64_t N, const DeviceInfo& info) {
 }
 
 mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
-                         const float* s_w, int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                         const float* s_w, int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info,
                          cudaStream_t stream) {
     switch (tiled_tile_width(M, N, info)) {
-        case 256: return launch_tiled_bn<256, 4>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-        case 128: return launch_tiled_bn<128, 6>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-        case 64: return launch_tiled_bn<64, 8>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-        default: return launch_tiled_bn<32, 10>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+        case 256: return launch_tiled_bn<256, 4>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
+        case 128: return launch_tiled_bn<128, 6>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
+        case 64: return launch_tiled_bn<64, 8>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
+        default: return launch_tiled_bn<32, 10>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
     }
 }
 
@@ -314,7 +314,7 @@ int max_active_clusters(Kern kern, int S, int smem, int threads, int dev) {
 
 template <int BN, int STAGES>
 mfp8_status launch_pair_bn(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                           int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                           int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info,
                            cudaStream_t stream) {
     using L = pair::Layout<BN, STAGES>;
     auto kern = pair::gemm_pair_kernel<BN, STAGES>;
@@ -323,7 +323,7 @@ mfp8_status launch_pair_bn(const void* X8, const float* s_a, int64_t M, int64_t 
     if (st != MFP8_OK) return st;
     CUtensorMap tmX, tmW, tmY;
     if ((st = make_map_u8(&tmX, X8, M, K, pair::HALF)) != MFP8_OK) return st;
-    if ((st = make_map_u8(&tmW, W8, N, K, BN / 2)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmW, W8, w_rows, K, BN / 2)) != MFP8_OK) return st;
     if ((st = make_map_y(&tmY, Y, M, N)) != MFP8_OK) return st;
     const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + BN - 1) / BN);
     // The grid is persistent: only as many pairs as can be resident at once.
@@ -367,10 +367,10 @@ int pair_tile_width(int64_t M, int64_t N, const DeviceInfo& info) {
 }
 
 mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                        int64_t N, void* Y, bool dependent, int dev, const DeviceInfo& info, cudaStream_t stream) {
+                        int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info, cudaStream_t stream) {
     if (pair_tile_width(M, N, info) == 128)
-        return launch_pair_bn<128, 8>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-    return launch_pair_bn<256, 6>(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+        return launch_pair_bn<128, 8>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
+    return launch_pair_bn<256, 6>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
 }
 
 constexpr int64_t kStreamMaxM = stream::kMaxM;
@@ -397,7 +397,7 @@ int choose_path(int64_t M, int64_t N, int64_t K) {
 
 mfp8_status check_gemm_args(int64_t M, int64_t N, int64_t K, const void* W8, const float* s_w, const void* Y) {
     if (M < 0 || N < 0 || K < 0) return MFP8_ERR_INVALID_ARG;
-    if (K == 0 || K % 16 != 0 || N == 0 || N % 8 != 0 || K > kMaxDim || N > kMaxDim || M > kMaxDim)
+    if (K == 0 || K % 16 != 0 || N == 0 || K > kMaxDim || N > kMaxDim || M > kMaxDim)
         return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (M > 0 && M * (K > N ? K : N) > (int64_t(1) << 40)) return MFP8_ERR_UNSUPPORTED_SHAPE;
     if (!W8 || !s_w || (M > 0 && !Y)) return MFP8_ERR_INVALID_ARG;
@@ -425,6 +425,45 @@ Plan make_plan(int64_t M, int64_t K, bool codes) {
     p.total = p.sa_off + round_up(size_t(M) * 4, 256);
     return p;
 }
+
+// N not a multiple of 8: rows of Y are not 16-byte aligned, which the
+// kernels' vector stores and the TMA store maps need.  The kernels then run
+// on N8 = N rounded up to 8 channels: the weight tensor map keeps N rows
+// (rows N .. N8-1 read as zeros), the channel scales are copied into a
+// zero-padded [N8] array and the output goes to an [M, N8] scratch, whose
+// first N columns a copy kernel writes into Y.  Both scratch arrays follow
+// the codes in the workspace.
+struct PadPlan {
+    int64_t n8 = 0;
+    size_t sw_off = 0, y_off = 0, total = 0;
+};
+
+PadPlan make_pad_plan(int64_t M, int64_t N, size_t start) {
+    PadPlan p;
+    p.n8 = N;
+    p.total = start;
+    if (N % 8 == 0) return p;
+    p.n8 = (N + 7) / 8 * 8;
+    p.sw_off = round_up(start, 256);
+    p.y_off = round_up(p.sw_off + size_t(p.n8) * 4, 256);
+    p.total = round_up(p.y_off + size_t(M) * size_t(p.n8) * 2, 256);
+    return p;
+}
+
+__global__ void pad_scales_kernel(const float* __restrict__ s_w, int64_t N, float* __restrict__ sw8, int64_t N8) {
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < N8; i += int64_t(gridDim.x) * blockDim.x)
+        sw8[i] = i < N ? s_w[i] : 0.0f;
+}
+
+__global__ void crop_rows_kernel(const uint16_t* __restrict__ Y8, int64_t N8, uint16_t* __restrict__ Y, int64_t M,
+                                 int64_t N) {
+    const int64_t n = M * N;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t m = i / N;
+        Y[i] = Y8[m * N8 + (i - m * N)];
+    }
+}
+
 
 // ------------------------------------------- decode: one-kernel Linear --
 
@@ -466,6 +505,7 @@ bool stream_geometry(int64_t M, int64_t N, int64_t K, int sm_count, stream::Geom
 }
 
 mfp8_status launch_stream(const void* X, int64_t M, int64_t K, const void* W8, const float* s_w, int64_t N,
+                          int64_t w_rows,
                           void* Y, bool weights_static, bool dependent, void* x8_out, float* sa_out, int dev,
                           const DeviceInfo& info, cudaStream_t stream) {
     if (M < 1 || M > kStreamMaxM || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
@@ -482,7 +522,7 @@ mfp8_status launch_stream(const void* X, int64_t M, int64_t K, const void* W8, c
     const int64_t grid = tiles * g.S;
     if (grid > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
     CUtensorMap tmW;
-    if ((st = make_map_u8(&tmW, W8, N, K, stream::TILE)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmW, W8, w_rows, K, stream::TILE)) != MFP8_OK) return st;
 
     stream::Args args;
     args.X = static_cast<const __nv_bfloat16*>(X);
@@ -554,7 +594,7 @@ bool cluster_geometry(int64_t M, int64_t N, int64_t K, int sm_count, cluster::Ge
 }
 
 mfp8_status launch_cluster(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                           int64_t N, void* Y, bool weights_static, bool dependent, int dev, const DeviceInfo& info,
+                           int64_t N, int64_t w_rows, void* Y, bool weights_static, bool dependent, int dev, const DeviceInfo& info,
                            cudaStream_t stream) {
     cluster::Geometry g;
     if (!cluster_geometry(M, N, K, info.sm_count, &g)) return MFP8_ERR_UNSUPPORTED_SHAPE;
@@ -566,7 +606,7 @@ mfp8_status launch_cluster(const void* X8, const float* s_a, int64_t M, int64_t 
     const int64_t grid = tiles * g.S;
     if (grid > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
     CUtensorMap tmX, tmW;
-    if ((st = make_map_u8(&tmW, W8, N, K, cluster::TILE)) != MFP8_OK) return st;
+    if ((st = make_map_u8(&tmW, W8, w_rows, K, cluster::TILE)) != MFP8_OK) return st;
     if ((st = make_map_u8(&tmX, X8, M, K, g.mp)) != MFP8_OK) return st;
 
     cluster::Args args;
@@ -602,14 +642,14 @@ mfp8_status launch_cluster(const void* X8, const float* s_a, int64_t M, int64_t 
 
 // The GEMM on codes already in memory (tiled, pair, or split-K).
 mfp8_status run_gemm(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                     int64_t N, void* Y, int path, bool weights_static, bool dependent, int dev,
+                     int64_t N, int64_t w_rows, void* Y, int path, bool weights_static, bool dependent, int dev,
                      const DeviceInfo& info, cudaStream_t stream) {
     // The kernels take M, N, K as 32-bit.
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
-    if (path == MFP8_PATH_TILED) return launch_tiled(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
-    if (path == MFP8_PATH_PAIR) return launch_pair(X8, s_a, M, K, W8, s_w, N, Y, dependent, dev, info, stream);
+    if (path == MFP8_PATH_TILED) return launch_tiled(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
+    if (path == MFP8_PATH_PAIR) return launch_pair(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
     if (path == MFP8_PATH_SPLITK)
-        return launch_cluster(X8, s_a, M, K, W8, s_w, N, Y, weights_static, dependent, dev, info, stream);
+        return launch_cluster(X8, s_a, M, K, W8, s_w, N, w_rows, Y, weights_static, dependent, dev, info, stream);
     return MFP8_ERR_INVALID_ARG;
 }
 
@@ -764,6 +804,37 @@ struct PickSiluMul {
     static auto kern() { return producer::silu_mul_quant_kernel<VPT>; }
 };
 
+// The padded run: scales padded, X quantized (unless FUSED), the kernels on
+// N8 channels into the scratch, then the crop.  Every launch here is a plain
+// stream-ordered launch, so the scratch scales are complete before any
+// kernel reads them.
+mfp8_status run_padded(const void* X_bf16, const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
+                       const float* s_w, int64_t N, void* Y, const PadPlan& pad, uint8_t* base, int path,
+                       void* X_fp8_out, float* x_scale_out, int dev, const DeviceInfo& info, cudaStream_t stream) {
+    float* sw8 = reinterpret_cast<float*>(base + pad.sw_off);
+    void* y8 = base + pad.y_off;
+    const int64_t cap = int64_t(info.sm_count) * 8;
+    pad_scales_kernel<<<unsigned((pad.n8 + 255) / 256 < cap ? (pad.n8 + 255) / 256 : cap), 256, 0, stream>>>(
+        s_w, N, sw8, pad.n8);
+    mfp8_status st = launch_status();
+    if (st != MFP8_OK) return st;
+    if (path == MFP8_PATH_FUSED) {
+        st = launch_stream(X_bf16, M, K, W8, sw8, pad.n8, N, y8, /*weights_static=*/false, /*dependent=*/false,
+                           X_fp8_out, x_scale_out, dev, info, stream);
+    } else {
+        if (X_bf16 && (st = quantize_weight_rows(X_bf16, M, K, const_cast<void*>(X8), const_cast<float*>(s_a),
+                                                 stream)) != MFP8_OK)
+            return st;
+        st = run_gemm(X8, s_a, M, K, W8, sw8, pad.n8, N, y8, path, /*weights_static=*/false, /*dependent=*/false,
+                      dev, info, stream);
+    }
+    if (st != MFP8_OK) return st;
+    const int64_t nb = (M * N + 255) / 256;
+    crop_rows_kernel<<<unsigned(nb < cap ? nb : cap), 256, 0, stream>>>(static_cast<const uint16_t*>(y8), pad.n8,
+                                                                        static_cast<uint16_t*>(Y), M, N);
+    return launch_status();
+}
+
 }  // namespace
 }  // namespace mfp8
 
@@ -793,7 +864,7 @@ mfp8_status mfp8_quantize_act(const void* X_bf16, int64_t M, int64_t K, void* X_
 
 size_t mfp8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return 0;
-    return make_plan(M, K, true).total;
+    return make_pad_plan(M, N, make_plan(M, K, true).total).total;
 }
 
 mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void* W_fp8, const float* w_scale,
@@ -817,17 +888,20 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
             ranges_overlap(x_scale_out, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
             return MFP8_ERR_INVALID_ARG;
     }
-    if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
+    if (path == MFP8_PATH_AUTO) path = choose_path(M, (N + 7) / 8 * 8, K);
     const bool weights_static = (flags & MFP8_FLAG_STATIC_WEIGHTS) != 0;
     // FUSED (M <= 16): one kernel quantizes X on chip and streams the
     // weights; it keeps nothing in the workspace.
     const bool fused = path == MFP8_PATH_FUSED;
     const Plan plan = fused ? Plan() : make_plan(M, K, X_fp8_out == nullptr);
-    if (plan.total > 0) {
-        if (!workspace || workspace_bytes_given < plan.total) return MFP8_ERR_WORKSPACE;
+    const PadPlan pad = make_pad_plan(M, N, plan.total);
+    if (pad.total > 0) {
+        if (!workspace || workspace_bytes_given < pad.total) return MFP8_ERR_WORKSPACE;
         if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
-        if (ranges_overlap(workspace, plan.total, Y_bf16, size_t(M * N * 2)) ||
-            ranges_overlap(workspace, plan.total, X_bf16, size_t(M * K * 2)))
+        if (ranges_overlap(workspace, pad.total, Y_bf16, size_t(M * N * 2)) ||
+            ranges_overlap(workspace, pad.total, X_bf16, size_t(M * K * 2)) ||
+            (X_fp8_out && (ranges_overlap(workspace, pad.total, X_fp8_out, size_t(M * K)) ||
+                           ranges_overlap(workspace, pad.total, x_scale_out, size_t(M * 4)))))
             return MFP8_ERR_INVALID_ARG;
     }
 
@@ -836,13 +910,19 @@ mfp8_status mfp8_linear_ex(const void* X_bf16, int64_t M, int64_t K, const void*
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* base = static_cast<uint8_t*>(workspace);
+    if (pad.n8 != N) {
+        const void* X8 = fused ? nullptr : (X_fp8_out ? X_fp8_out : base + plan.x8_off);
+        const float* s_a = fused ? nullptr : (x_scale_out ? x_scale_out : reinterpret_cast<float*>(base + plan.sa_off));
+        return run_padded(X_bf16, X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, pad, base, path, X_fp8_out, x_scale_out,
+                          dev, info, s);
+    }
     if (fused)
-        return launch_stream(X_bf16, M, K, W_fp8, w_scale, N, Y_bf16, weights_static, /*dependent=*/true,
+        return launch_stream(X_bf16, M, K, W_fp8, w_scale, N, N, Y_bf16, weights_static, /*dependent=*/true,
                              X_fp8_out, x_scale_out, dev, info, s);
     void* X8 = X_fp8_out ? X_fp8_out : base + plan.x8_off;
     float* s_a = x_scale_out ? x_scale_out : reinterpret_cast<float*>(base + plan.sa_off);
     if ((st = quantize_act_rows(X_bf16, M, K, X8, s_a, s)) != MFP8_OK) return st;
-    return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, Y_bf16, path, weights_static,
+    return run_gemm(X8, s_a, M, K, W_fp8, w_scale, N, N, Y_bf16, path, weights_static,
                     /*dependent=*/true, dev, info, s);
 }
 
@@ -872,8 +952,8 @@ int mfp8_choose_path(int64_t M, int64_t N, int64_t K) {
 }
 
 size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    (void)M, (void)N, (void)K;
-    return 0;  // the GEMM kernels keep nothing in a workspace
+    if (M <= 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return 0;
+    return make_pad_plan(M, N, 0).total;  // only N % 8 != 0 needs scratch
 }
 
 mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K, const void* W_fp8,
@@ -889,14 +969,25 @@ mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_
     if (ranges_overlap(X_fp8, size_t(M * K), Y_bf16, size_t(M * N * 2)) ||
         ranges_overlap(x_scale, size_t(M * 4), Y_bf16, size_t(M * N * 2)))
         return MFP8_ERR_INVALID_ARG;
-    if (path == MFP8_PATH_AUTO) path = choose_path(M, N, K);
+    const PadPlan pad = make_pad_plan(M, N, 0);
+    if (path == MFP8_PATH_AUTO) path = choose_path(M, pad.n8, K);
     if (path == MFP8_PATH_FUSED) path = MFP8_PATH_SPLITK;  // codes given: the split-K kernel streams them
-    (void)workspace, (void)workspace_bytes_given;  // kept in the signature; nothing needs it
+    if (pad.total > 0) {
+        if (!workspace || workspace_bytes_given < pad.total) return MFP8_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MFP8_ERR_MISALIGNED;
+        if (ranges_overlap(workspace, pad.total, Y_bf16, size_t(M * N * 2)) ||
+            ranges_overlap(workspace, pad.total, X_fp8, size_t(M * K)) ||
+            ranges_overlap(workspace, pad.total, x_scale, size_t(M * 4)))
+            return MFP8_ERR_INVALID_ARG;
+    }
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, path, /*weights_static=*/false,
+    if (pad.n8 != N)
+        return run_padded(nullptr, X_fp8, x_scale, M, K, W_fp8, w_scale, N, Y_bf16, pad,
+                          static_cast<uint8_t*>(workspace), path, nullptr, nullptr, dev, info, s);
+    return run_gemm(X_fp8, x_scale, M, K, W_fp8, w_scale, N, N, Y_bf16, path, /*weights_static=*/false,
                     /*dependent=*/false, dev, info, s);
 }
 

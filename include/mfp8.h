@@ -28,7 +28,12 @@
  *     IEEE bfloat16 bit patterns; FP8 buffers hold float8_e4m3fn codes, one
  *     byte each; scales are fp32.
  *   - Every pointer must be 16-byte aligned.  K must be a positive multiple
- *     of 16, N a positive multiple of 8, M >= 0 (M == 0 is a no-op).
+ *     of 16, N >= 1, M >= 0 (M == 0 is a no-op).  When N is not a multiple
+ *     of 8 (rows of Y not 16-byte aligned) the Linear runs its kernels on N
+ *     rounded up to 8 channels into scratch taken from the workspace (the
+ *     workspace-size functions count it), then copies the first N columns
+ *     into Y: two small extra launches, and MFP8_FLAG_STATIC_WEIGHTS has no
+ *     effect.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
  *     enqueued on it; no call blocks the host except mfp8_get_device_status.
  *     The calls do not synchronise and may be captured in a CUDA graph.
@@ -59,7 +64,7 @@ typedef enum {
     MFP8_OK = 0,
     MFP8_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, overlapping in/out */
     MFP8_ERR_MISALIGNED = 2,        /* a pointer is not 16-byte aligned */
-    MFP8_ERR_UNSUPPORTED_SHAPE = 3, /* K not a positive multiple of 16, N not a positive multiple of 8, too large */
+    MFP8_ERR_UNSUPPORTED_SHAPE = 3, /* K not a positive multiple of 16, N < 1, too large */
     MFP8_ERR_WORKSPACE = 4,         /* workspace missing or smaller than mfp8_linear_workspace_bytes */
     MFP8_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
     MFP8_ERR_TIMEOUT = 6,           /* a kernel's bounded wait ran out (device status) */
@@ -146,7 +151,8 @@ MFP8_API int mfp8_choose_path(int64_t M, int64_t N, int64_t K);
  * MFP8_PATH_FUSED is one launch that quantizes X on chip (the CTAs of a
  * cluster share their slice maxima, so each has the full row scales) and
  * sums the K-split partial rows in the cluster's shared memory, so it keeps
- * nothing in the workspace (it may be NULL with 0 bytes).  When
+ * nothing in the workspace (it may be NULL with 0 bytes) unless N % 8 != 0
+ * (the padded scratch of the conventions).  When
  * X_fp8_out is given, the codes are written there as well (the quantize
  * pass writes them there instead of the workspace).  Returns MFP8_ERR_UNSUPPORTED_SHAPE if the chosen kernel
  * cannot take these sizes, MFP8_ERR_INVALID_ARG for an unknown path or flag. */
@@ -180,15 +186,18 @@ MFP8_API mfp8_status mfp8_linear_noalloc(const void* X_bf16, int64_t M, int64_t 
                                 const void* W_fp8, const float* w_scale, int64_t N,
                                 void* Y_bf16, void* stream);
 
-/* Workspace bytes mfp8_gemm needs: 0, since no GEMM kernel keeps anything
- * in one (kept for callers that size a workspace before they call). */
+/* Workspace bytes mfp8_gemm needs: 0 when N is a multiple of 8 (no GEMM
+ * kernel keeps anything in one; the workspace may then be NULL), else the
+ * padded scratch of the conventions above: the [N8] scales and the [M, N8]
+ * bf16 output, N8 = N rounded up to 8. */
 MFP8_API size_t mfp8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* The contraction and epilogue alone, on activations already quantized by
  * mfp8_quantize_act: Y = bf16((X_fp8 . W_fp8^T) * x_scale (x) w_scale).
  * Lets the GEMM be timed and checked without the quantize pass.  path is
  * AUTO, TILED, SPLITK or PAIR (FUSED is taken as SPLITK: the codes are
- * given).  `workspace` and `workspace_bytes` are not used. */
+ * given).  `workspace` (mfp8_gemm_workspace_bytes(M, N, K) bytes) is used
+ * only when N % 8 != 0; otherwise it may be NULL with 0 bytes. */
 MFP8_API mfp8_status mfp8_gemm(const void* X_fp8, const float* x_scale, int64_t M, int64_t K,
                       const void* W_fp8, const float* w_scale, int64_t N,
                       void* Y_bf16, void* workspace, size_t workspace_bytes,

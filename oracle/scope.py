@@ -45,6 +45,19 @@ def fp8_dynamic_selected(names, cross=CROSS_LAYERS):
     return out
 
 
+def fp8_dynamic_target_pattern(cross=CROSS_LAYERS, n_layers: int = N_LAYERS) -> str:
+    """The recipe's target as a regular expression over module names (the
+    README's FP8-Dynamic recipe targets one pattern: a language-model layer
+    index from the layers without cross-attention, then a self-attention
+    q/k/v/o projection or an MLP gate/up/down projection, anchored at both
+    ends).  Built here from this module's own tuples; ``re.fullmatch`` with
+    it must select exactly what ``fp8_dynamic_selected`` selects."""
+    layers = "|".join(str(i) for i in range(n_layers) if i not in cross)
+    attn = "|".join(ATTN_PROJ)
+    mlp = "|".join(MLP_PROJ)
+    return rf"model\.language_model\.layers\.({layers})\.(self_attn\.({attn})|mlp\.({mlp}))"
+
+
 def nf4_keep_ends_selected(names, keep: int = 4, n_layers: int = N_LAYERS):
     """Names the NF4 Keep-4 recipe quantizes: every language Linear except
     those in the first/last ``keep`` layers and those under ``cross_attn``."""

@@ -142,7 +142,10 @@ def test_argument_errors_are_reported_before_any_launch(lib):
         return L(a["X"], a["M"], a["K"], a["W"], a["sw"], a["N"], a["Y"], a["ws"], a["wsb"],
                  kw.get("path", 0), kw.get("flags", 0), kw.get("x8", None), kw.get("xs", None), None)
 
-    assert call(N=12) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert call(N=12, wsb=100) == mfp8.ERR_WORKSPACE  # N % 8 != 0 takes a padded scratch in the workspace
+    assert call(N=12, path=mfp8.PATH_FUSED, ws=None) == mfp8.ERR_WORKSPACE  # even on the fused path
+    assert mfp8.mfp8_linear_workspace_bytes(4, 12, 64) > mfp8.mfp8_linear_workspace_bytes(4, 16, 64)
+    assert mfp8.mfp8_gemm_workspace_bytes(4, 16, 64) == 0 and mfp8.mfp8_gemm_workspace_bytes(4, 13, 64) > 0
     assert call(N=0) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(K=8) == mfp8.ERR_UNSUPPORTED_SHAPE
     assert call(W=None) == mfp8.ERR_INVALID_ARG
@@ -160,7 +163,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert call(Y=FAKE + 64) == mfp8.ERR_INVALID_ARG  # Y overlaps X
     assert call(M=0) == mfp8.OK
     NA = mfp8.mfp8_linear_noalloc
-    assert NA(FAKE, 4, 64, FAKE * 2, FAKE * 3, 12, FAKE * 4, None) == mfp8.ERR_UNSUPPORTED_SHAPE
+    assert NA(FAKE, 4, 40, FAKE * 2, FAKE * 3, 12, FAKE * 4, None) == mfp8.ERR_UNSUPPORTED_SHAPE  # K % 16
     assert NA(FAKE, 0, 64, FAKE * 2, FAKE * 3, 64, FAKE * 4, None) == mfp8.OK
     # more than the library's fixed scratch: codes alone are 4096 * 8192 bytes
     assert NA(FAKE, 4096, 8192, FAKE * 2, FAKE * 3, 64, FAKE * 4, None) == mfp8.ERR_WORKSPACE
@@ -198,7 +201,7 @@ int main(void) {
     if (mfp8_choose_path(8, 4096, 4096) != MFP8_PATH_FUSED) return 13;
     /* argument errors come back before any device work */
     if (mfp8_linear(NULL, 4, 64, NULL, NULL, 64, NULL, NULL, 0, NULL) != MFP8_ERR_INVALID_ARG) return 14;
-    if (mfp8_linear_noalloc((void*)4096, 4, 64, (void*)8192, (float*)12288, 12, (void*)16384, NULL)
+    if (mfp8_linear_noalloc((void*)4096, 4, 40, (void*)8192, (float*)12288, 12, (void*)16384, NULL)
         != MFP8_ERR_UNSUPPORTED_SHAPE) return 15;
     printf("%%s\n", mfp8_status_string(MFP8_ERR_MISALIGNED));
     return 0;

@@ -41,6 +41,7 @@ CASES = [  # (M, N, K): ragged in M and N, several tiles
     (17, 136, 272), (37, 264, 400), (100, 520, 528), (128, 1160, 400),   # cluster split-K
     (130, 264, 384), (201, 776, 528), (256, 1032, 400),                  # 1-CTA tiles, split-K
     (300, 520, 400), (513, 1032, 528),                                   # CTA pairs
+    (3, 7, 272), (40, 101, 400), (200, 1001, 528), (600, 77, 400),       # N % 8 != 0: padded scratch + crop
 ]
 
 

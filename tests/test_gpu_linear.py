@@ -62,6 +62,47 @@ def test_linear_static_weights_flag(M, N, K, path):
     run_case(M, N, K, path, seed=M + 3, flags=mfp8.FLAG_STATIC_WEIGHTS)
 
 
+ODD_N = [(4, 1, 64), (3, 7, 128), (16, 100, 528), (40, 13, 272), (100, 1001, 256), (200, 77, 640),
+         (512, 1030, 1024), (2, 4099, 4096), (300, 4101, 128)]
+
+
+@pytest.mark.parametrize("M,N,K", ODD_N)
+@pytest.mark.parametrize("path", [mfp8.PATH_TILED, mfp8.PATH_SPLITK, mfp8.PATH_PAIR, mfp8.PATH_FUSED,
+                                  mfp8.PATH_AUTO])
+def test_linear_any_n(M, N, K, path):
+    """N not a multiple of 8 (rows of Y not 16-byte aligned): the kernels run
+    on N rounded up to 8 into a workspace scratch and the first N columns are
+    copied out; codes bit-exact, outputs within the tolerance."""
+    if path == mfp8.PATH_FUSED and M > 16:
+        pytest.skip("the fused decode kernel takes M <= 16")
+    if path == mfp8.PATH_SPLITK and M > 256:
+        pytest.skip("the split-K kernel takes M <= 256")
+    assert mfp8.mfp8_linear_workspace_bytes(M, N, K) > mfp8.mfp8_linear_workspace_bytes(M, (N + 7) // 8 * 8, K)
+    run_case(M, N, K, path, seed=M + N, flags=mfp8.FLAG_STATIC_WEIGHTS if M <= 16 else 0)
+
+
+@pytest.mark.parametrize("M,N,K", [(5, 13, 272), (64, 1001, 400), (700, 77, 528)])
+def test_gemm_any_n(M, N, K):
+    """mfp8_gemm on codes with N % 8 != 0 takes the scratch from its
+    workspace (mfp8_gemm_workspace_bytes > 0 only then) and equals the
+    Linear's output bit for bit."""
+    assert mfp8.mfp8_gemm_workspace_bytes(M, N, K) > 0
+    assert mfp8.mfp8_gemm_workspace_bytes(M, (N + 7) // 8 * 8, K) == 0
+    x = W.make_x(M, K, seed=N, device=DEV)
+    W8, sw = mfp8.quantize_weight(W.make_w(N, K, seed=N, device=DEV))
+    x8, xs = mfp8.quantize_act(x)
+    for path in (mfp8.PATH_AUTO, mfp8.PATH_TILED, mfp8.PATH_PAIR):
+        y = mfp8.gemm(x8, xs, W8, sw, path=path)
+        y_lin = mfp8.linear(x, W8, sw, path=path)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_lin.view(torch.int16)), f"path {path}"
+        assert_linear_parity(y, u8(x8), f32(xs), u8(W8), f32(sw), what=f"gemm M={M} N={N} K={K} path={path}")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    st = mfp8.mfp8_gemm(x8.data_ptr(), xs.data_ptr(), M, K, W8.data_ptr(), sw.data_ptr(), N, out.data_ptr(), None, 0,
+                        mfp8.PATH_AUTO, torch.cuda.current_stream().cuda_stream)
+    assert st == mfp8.ERR_WORKSPACE
+
+
 def test_linear_without_codes_out_matches_with():
     """The decode kernel writes the optional code copy only from its first
     cluster; the outputs must not depend on whether it is asked for."""

@@ -1,6 +1,7 @@
 """Which Linears are quantized: counts printed on the pages."""
 import json
 import os
+import re
 
 from oracle import scope
 
@@ -33,3 +34,23 @@ def test_workload_shapes_match_the_pages():
     assert W.N_KV_HEADS == GOLD["n_kv_heads"]["value"]
     assert len(W.SELF_LAYERS) * len(W.LAYER_LINEARS) == GOLD["fp8_dynamic_linears"]["value"]
     assert list(W.CROSS_LAYERS) == GOLD["cross_attention_layers"]["value"]
+
+
+def test_target_pattern_selects_the_same_252():
+    """The recipe's target pattern, applied to every language Linear and to
+    names it must not take (vision tower, lm_head, cross-attention modules,
+    the extra `model.` level of the SGLang ignore list, suffixes, other
+    projections), selects exactly the walked set."""
+    names = scope.language_linear_names()
+    decoys = ["model.visual.blocks.0.attn.qkv", "model.language_model.lm_head", "lm_head",
+              "model.language_model.model.layers.0.self_attn.q_proj",
+              "model.language_model.layers.0.self_attn.q_proj.weight",
+              "model.language_model.layers.0.self_attn.q_norm",
+              "model.language_model.layers.2.self_attn.q_proj",
+              "model.language_model.layers.48.mlp.up_proj",
+              "model.language_model.layers.10.mlp.gate_proj",
+              "xmodel.language_model.layers.0.mlp.down_proj"]
+    pat = re.compile(scope.fp8_dynamic_target_pattern())
+    by_pattern = [n for n in names + decoys if pat.fullmatch(n)]
+    assert by_pattern == scope.fp8_dynamic_selected(names)
+    assert len(by_pattern) == GOLD["fp8_dynamic_linears"]["value"]
