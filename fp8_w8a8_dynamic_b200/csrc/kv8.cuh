@@ -41,38 +41,6 @@ constexpr int kSliceRows = kGroup / (kQuantThreads / 32);
 constexpr int kReadThreads = 256;
 constexpr int kReadRows = 8;  // tokens per thread in the read
 
-// Two fp32 lanes in one 64-bit register: Blackwell's paired fp32 arithmetic
-// (add/mul/fma .f32x2) rounds each lane to nearest even like the scalar
-// instructions.
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-    uint64_t d;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-    return d;
-}
-__device__ __forceinline__ void unpack2(uint64_t d, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
 // The group's scale and zero point.
 __device__ __forceinline__ void fit(float mn, float mx, float& s, float& z) {
     const float range = __fsub_rn(mx, mn);

@@ -797,7 +797,7 @@ mfp8_status launch_pdl(void (*kern)(KArgs...), dim3 grid, int threads, cudaStrea
 
 template <int VPT>
 struct PickRmsnorm {
-    static auto kern() { return producer::rmsnorm_quant_kernel<VPT>; }
+    static auto kern() { return producer::rmsnorm_quant_kernel<producer::kThreads, VPT>; }
 };
 template <int VPT>
 struct PickSiluMul {
@@ -1007,9 +1007,23 @@ mfp8_status mfp8_rmsnorm_quantize(const void* X_bf16, const void* gamma_bf16, fl
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != MFP8_OK) return st;
-    return launch_producer<PickRmsnorm>(K / 8, M, static_cast<cudaStream_t>(stream),
-                                        static_cast<const uint4*>(X_bf16), static_cast<const uint4*>(gamma_bf16),
-                                        K, eps, static_cast<uint4*>(Y_bf16), static_cast<uint2*>(X_fp8), x_scale);
+    const int64_t nvec = K / 8;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint4* xv = static_cast<const uint4*>(X_bf16);
+    const uint4* gv = static_cast<const uint4*>(gamma_bf16);
+    uint4* yv = static_cast<uint4*>(Y_bf16);
+    uint2* qv = static_cast<uint2*>(X_fp8);
+    // Rows up to 4096 values: 128 threads per row.
+    if (nvec <= 128)
+        return launch_pdl(producer::rmsnorm_quant_kernel<128, 1>, dim3(unsigned(M)), 128, s, 0, xv, gv, K, eps, yv,
+                          qv, x_scale);
+    if (nvec <= 256)
+        return launch_pdl(producer::rmsnorm_quant_kernel<128, 2>, dim3(unsigned(M)), 128, s, 0, xv, gv, K, eps, yv,
+                          qv, x_scale);
+    if (nvec <= 512)
+        return launch_pdl(producer::rmsnorm_quant_kernel<128, 4>, dim3(unsigned(M)), 128, s, 0, xv, gv, K, eps, yv,
+                          qv, x_scale);
+    return launch_producer<PickRmsnorm>(nvec, M, s, xv, gv, K, eps, yv, qv, x_scale);
 }
 
 mfp8_status mfp8_silu_mul_quantize(const void* GU_bf16, int64_t M, int64_t I, void* Y_bf16, void* X_fp8,
@@ -1057,14 +1071,14 @@ mfp8_status mfp8_kv_quantize(const void* KV_bf16, int64_t T, int64_t H, int64_t 
     if (blocks > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
     const uint4* x = static_cast<const uint4*>(KV_bf16);
     uint2* q = static_cast<uint2*>(KV_fp8);
+    const dim3 grid{static_cast<unsigned>(blocks)};
     switch (lpr) {
-        case 2: quant_small_rows_kernel<2><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
-        case 4: quant_small_rows_kernel<4><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
-        case 8: quant_small_rows_kernel<8><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
-        case 16: quant_small_rows_kernel<16><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
-        default: quant_small_rows_kernel<32><<<unsigned(blocks), kQuantThreads, 0, s>>>(x, R, int(D), q, kv_scale); break;
+        case 2: return launch_pdl(quant_small_rows_kernel<2>, grid, kQuantThreads, s, 0, x, R, int(D), q, kv_scale);
+        case 4: return launch_pdl(quant_small_rows_kernel<4>, grid, kQuantThreads, s, 0, x, R, int(D), q, kv_scale);
+        case 8: return launch_pdl(quant_small_rows_kernel<8>, grid, kQuantThreads, s, 0, x, R, int(D), q, kv_scale);
+        case 16: return launch_pdl(quant_small_rows_kernel<16>, grid, kQuantThreads, s, 0, x, R, int(D), q, kv_scale);
+        default: return launch_pdl(quant_small_rows_kernel<32>, grid, kQuantThreads, s, 0, x, R, int(D), q, kv_scale);
     }
-    return launch_status();
 }
 
 mfp8_status mfp8_kv_dequantize(const void* KV_fp8, const float* kv_scale, int64_t T, int64_t H, int64_t D,

@@ -32,10 +32,10 @@
 namespace mfp8 {
 namespace producer {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kThreads = 256;  // block size of the SiLU kernel and of RMSNorm on long rows
 
 // Sum over the block, the same order on every run.
+template <int kWarps>
 __device__ __forceinline__ float block_sum(float v, float* red /* [kWarps] */) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -49,6 +49,7 @@ __device__ __forceinline__ float block_sum(float v, float* red /* [kWarps] */) {
 }
 
 // Max of a bf16 magnitude (as bits) over the block.
+template <int kWarps>
 __device__ __forceinline__ uint32_t block_max(uint32_t v, uint32_t* red /* [kWarps] */) {
     v = __reduce_max_sync(0xffffffffu, v);
     const int w = threadIdx.x >> 5;
@@ -67,29 +68,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // The row's codes and scale from its bf16 values y (held as VPT vectors):
 // the quantizer of quant.cuh on the same bits.
-template <int VPT>
+template <int THREADS, int VPT>
 __device__ __forceinline__ void quantize_row(const uint4 (&y)[VPT], int64_t nvec, int64_t row, uint2* __restrict__ Q,
                                              float* __restrict__ S, uint32_t* red) {
     uint32_t acc = 0;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) acc = absmax_bits_u4(y[i], acc);
-    const uint32_t amax = block_max(max(acc & 0xffffu, acc >> 16), red);
+    const uint32_t amax = block_max<THREADS / 32>(max(acc & 0xffffu, acc >> 16), red);
     const float s = scale_from_absmax_bits(amax);
     const float r = __frcp_rn(s);
     if (threadIdx.x == 0) S[row] = s;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-        const int64_t j = threadIdx.x + int64_t(i) * kThreads;
+        const int64_t j = threadIdx.x + int64_t(i) * THREADS;
         if (j < nvec) Q[row * nvec + j] = quantize8(y[i], s, r);
     }
 }
 
 // RMSNorm + quantize.  X [M, K], gain G [K], bf16; Y [M, K] bf16 (optional),
-// Q [M, K] codes, S [M] scales.  K / 8 <= VPT * 256.
-template <int VPT>
-__global__ void __launch_bounds__(kThreads)
+// Q [M, K] codes, S [M] scales.  K / 8 <= VPT * THREADS.  Rows up to 4096
+// values take 128 threads (fewer warps per reduction, more rows resident
+// per SM), longer rows 256.
+template <int THREADS, int VPT>
+__global__ void __launch_bounds__(THREADS)
 rmsnorm_quant_kernel(const uint4* __restrict__ X, const uint4* __restrict__ G, int64_t K, float eps,
                      uint4* __restrict__ Y, uint2* __restrict__ Q, float* __restrict__ S) {
+    constexpr int kWarps = THREADS / 32;
     grid_launch_dependents();
     grid_dependency_wait();  // X may be the previous kernel's output
     __shared__ float red_f[kWarps];
@@ -100,7 +104,7 @@ rmsnorm_quant_kernel(const uint4* __restrict__ X, const uint4* __restrict__ G, i
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-        const int64_t j = threadIdx.x + int64_t(i) * kThreads;
+        const int64_t j = threadIdx.x + int64_t(i) * THREADS;
         x[i] = j < nvec ? __ldg(X + row * nvec + j) : make_uint4(0u, 0u, 0u, 0u);
         const uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
 #pragma unroll
@@ -110,11 +114,11 @@ rmsnorm_quant_kernel(const uint4* __restrict__ X, const uint4* __restrict__ G, i
             ss = __fmaf_rn(hi, hi, ss);
         }
     }
-    const float total = block_sum(ss, red_f);
+    const float total = block_sum<kWarps>(ss, red_f);
     const float r = 1.0f / sqrtf(total / float(K) + eps);
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-        const int64_t j = threadIdx.x + int64_t(i) * kThreads;
+        const int64_t j = threadIdx.x + int64_t(i) * THREADS;
         const uint4 g = j < nvec ? __ldg(G + j) : make_uint4(0u, 0u, 0u, 0u);
         const uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
         const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
@@ -126,7 +130,7 @@ rmsnorm_quant_kernel(const uint4* __restrict__ X, const uint4* __restrict__ G, i
         x[i] = make_uint4(o[0], o[1], o[2], o[3]);  // now y
         if (Y != nullptr && j < nvec) Y[row * nvec + j] = x[i];
     }
-    quantize_row<VPT>(x, nvec, row, Q, S, red_u);
+    quantize_row<THREADS, VPT>(x, nvec, row, Q, S, red_u);
 }
 
 // silu(v) * u in fp32 with CUDA's fast exponential and division intrinsics
@@ -150,7 +154,7 @@ silu_mul_quant_kernel(const uint4* __restrict__ GU, int64_t I, uint4* __restrict
                       float* __restrict__ S) {
     grid_launch_dependents();
     grid_dependency_wait();  // GU may be the previous kernel's output
-    __shared__ uint32_t red_u[kWarps];
+    __shared__ uint32_t red_u[kThreads / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = I >> 3;
     const uint4* gate = GU + row * 2 * nvec;
@@ -173,7 +177,7 @@ silu_mul_quant_kernel(const uint4* __restrict__ GU, int64_t I, uint4* __restrict
         y[i] = make_uint4(o[0], o[1], o[2], o[3]);
         if (Y != nullptr && j < nvec) Y[row * nvec + j] = y[i];
     }
-    quantize_row<VPT>(y, nvec, row, Q, S, red_u);
+    quantize_row<kThreads, VPT>(y, nvec, row, Q, S, red_u);
 }
 
 }  // namespace producer

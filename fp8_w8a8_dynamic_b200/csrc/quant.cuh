@@ -100,9 +100,15 @@ __device__ __forceinline__ float div_rn_by_recip(float a, float s, float r) {
 // the low byte).
 // The quotients carry x's sign except for x = -0 (see div_rn_by_recip), so
 // the sign bits of x are OR-ed into the codes: a no-op for every other x.
-__device__ __forceinline__ uint32_t quantize2_fma(uint32_t w, float s, float r) {
-    const float lo = div_rn_by_recip(__uint_as_float(w << 16), s, r);
-    const float hi = div_rn_by_recip(__uint_as_float(w & 0xffff0000u), s, r);
+// Both values go through div_rn_by_recip's three steps at once in paired
+// fp32 arithmetic (ns2 = (-s, -s), r2 = (r, r)): each lane rounds exactly as
+// the scalar steps do, and x - q0 s is q0 * (-s) + x in one fused
+// multiply-add.
+__device__ __forceinline__ uint32_t quantize2_fma(uint32_t w, uint64_t ns2, uint64_t r2) {
+    const uint64_t x = pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    const uint64_t q0 = mul2(x, r2);
+    float lo, hi;
+    unpack2(fma2(fma2(q0, ns2, x), r2, q0), lo, hi);
     return e4m3x2(lo, hi) | (__byte_perm(w, 0u, 0x4431u) & 0x8080u);  // bits 15, 31 of w -> 7, 15
 }
 
@@ -115,8 +121,9 @@ constexpr float kFmaMinScale = 5.42101086242752217004e-20f;  // 2^-64
 // For s >= kFmaMinScale only (callers that check the scale once per row).
 __device__ __forceinline__ uint2 quantize8_fast(uint4 v, float s, float r) {
     uint2 out;
-    out.x = quantize2_fma(v.x, s, r) | (quantize2_fma(v.y, s, r) << 16);
-    out.y = quantize2_fma(v.z, s, r) | (quantize2_fma(v.w, s, r) << 16);
+    const uint64_t ns2 = pack2(-s, -s), r2 = pack2(r, r);
+    out.x = quantize2_fma(v.x, ns2, r2) | (quantize2_fma(v.y, ns2, r2) << 16);
+    out.y = quantize2_fma(v.z, ns2, r2) | (quantize2_fma(v.w, ns2, r2) << 16);
     return out;
 }
 
@@ -288,6 +295,8 @@ template <int LPR>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_small_rows_kernel(const uint4* __restrict__ X, int64_t R, int D, uint2* __restrict__ Q,
                         float* __restrict__ S) {
+    grid_launch_dependents();
+    grid_dependency_wait();  // X may be the previous kernel's output
     constexpr int kRowsPerWarp = 32 / LPR;
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp +
