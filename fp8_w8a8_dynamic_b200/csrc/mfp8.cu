@@ -799,9 +799,11 @@ template <int VPT>
 struct PickRmsnorm {
     static auto kern() { return producer::rmsnorm_quant_kernel<producer::kThreads, VPT>; }
 };
+constexpr int64_t kSiluWideFrom = 1024;  // rows above this many 8-value vectors take 512 threads
+
 template <int VPT>
 struct PickSiluMul {
-    static auto kern() { return producer::silu_mul_quant_kernel<VPT>; }
+    static auto kern() { return producer::silu_mul_quant_kernel<producer::kThreads, VPT>; }
 };
 
 // The padded run: scales padded, X quantized (unless FUSED), the kernels on
@@ -1046,9 +1048,18 @@ mfp8_status mfp8_silu_mul_quantize(const void* GU_bf16, int64_t M, int64_t I, vo
     DeviceInfo info;
     mfp8_status st = current_device(&dev, &info);
     if (st != MFP8_OK) return st;
-    return launch_producer<PickSiluMul>(I / 8, M, static_cast<cudaStream_t>(stream),
-                                        static_cast<const uint4*>(GU_bf16), I, static_cast<uint4*>(Y_bf16),
-                                        static_cast<uint2*>(X_fp8), x_scale);
+    const int64_t nvec = I / 8;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint4* gu = static_cast<const uint4*>(GU_bf16);
+    uint4* yv = static_cast<uint4*>(Y_bf16);
+    uint2* qv = static_cast<uint2*>(X_fp8);
+    // Long rows: 512 threads per row (more warps resident per SM to hide the
+    // loads behind the arithmetic).
+    if (nvec > kSiluWideFrom && nvec <= 1536)
+        return launch_pdl(producer::silu_mul_quant_kernel<512, 3>, dim3(unsigned(M)), 512, s, 0, gu, I, yv, qv, x_scale);
+    if (nvec > kSiluWideFrom && nvec <= 2048)
+        return launch_pdl(producer::silu_mul_quant_kernel<512, 4>, dim3(unsigned(M)), 512, s, 0, gu, I, yv, qv, x_scale);
+    return launch_producer<PickSiluMul>(nvec, M, s, gu, I, yv, qv, x_scale);
 }
 
 mfp8_status mfp8_kv_quantize(const void* KV_bf16, int64_t T, int64_t H, int64_t D, void* KV_fp8, float* kv_scale,

@@ -147,14 +147,14 @@ __device__ __forceinline__ float silu_mul(float v, float u) {
 
 // SiLU(gate) * up + quantize, on the packed gate_up output GU [M, 2I] (gate
 // in columns 0 .. I-1, up in I .. 2I-1); Y [M, I] bf16 (optional), Q [M, I]
-// codes, S [M] scales.  I / 8 <= VPT * 256.
-template <int VPT>
-__global__ void __launch_bounds__(kThreads)
+// codes, S [M] scales.  I / 8 <= VPT * THREADS.
+template <int THREADS, int VPT>
+__global__ void __launch_bounds__(THREADS)
 silu_mul_quant_kernel(const uint4* __restrict__ GU, int64_t I, uint4* __restrict__ Y, uint2* __restrict__ Q,
                       float* __restrict__ S) {
     grid_launch_dependents();
     grid_dependency_wait();  // GU may be the previous kernel's output
-    __shared__ uint32_t red_u[kThreads / 32];
+    __shared__ uint32_t red_u[THREADS / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = I >> 3;
     const uint4* gate = GU + row * 2 * nvec;
@@ -162,7 +162,7 @@ silu_mul_quant_kernel(const uint4* __restrict__ GU, int64_t I, uint4* __restrict
     uint4 y[VPT];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-        const int64_t j = threadIdx.x + int64_t(i) * kThreads;
+        const int64_t j = threadIdx.x + int64_t(i) * THREADS;
         uint4 gv = make_uint4(0u, 0u, 0u, 0u), uv = gv;
         if (j < nvec) {
             gv = __ldg(gate + j);
@@ -177,7 +177,7 @@ silu_mul_quant_kernel(const uint4* __restrict__ GU, int64_t I, uint4* __restrict
         y[i] = make_uint4(o[0], o[1], o[2], o[3]);
         if (Y != nullptr && j < nvec) Y[row * nvec + j] = y[i];
     }
-    quantize_row<kThreads, VPT>(y, nvec, row, Q, S, red_u);
+    quantize_row<THREADS, VPT>(y, nvec, row, Q, S, red_u);
 }
 
 }  // namespace producer
