@@ -14,7 +14,7 @@
 //    each step rounded to nearest even:
 //      range = max - min;  s = max(range / 255, FLT_MIN) when range > 0,
 //      s = max(|min|, FLT_MIN) for a constant group;  z = rint(-min / s) + 0
-//      q = min(255, max(0, rint(x / s + z)))          (NaN -> 0)
+//      q = min(255, max(0, rint(x / s + z)))
 //  - dequantize: bf16((q - z) * s), q - z exact.
 // Inputs must be finite with max - min finite in fp32; then |z| <= 255 *
 // 2^9 (a non-constant group of bf16 values has range >= 2^-9 max|x|, so
@@ -57,15 +57,15 @@ __device__ __forceinline__ uint32_t code_div(float x, float s, float z) {
     return c < 255u ? c : 255u;
 }
 
-// Two codes for one word of two bf16 values (lanes = its two columns).  x / s is the corrected quotient: q0 =
-// x r with r = fl32(1/s), the residual x - q0 s in one fused multiply-add
-// (ns = -s), and q0 + residual * r rounded once: the correctly rounded
-// quotient whenever the residual is exact (Markstein's theorem), which
-// holds for |x| >= 2^-103 (the residual, about 2^-23 |x|, stays normal).
-// Smaller x with s >= kFmaMinScale = 2^-64 give |x / s| < 2^-39, and then
-// t = q + z rounds to z or to within 2^-39 of 0 whatever the quotient's
-// last bits, so the code is the divide's.  code_check_kernel compares the
-// two forms on every finite bf16 x.
+// Two codes for one word of two bf16 values (lanes = its two columns).
+// x / s is the corrected quotient: q0 = x r with r = fl32(1/s), the residual
+// x - q0 s in one fused multiply-add (ns = -s), and q0 + residual * r
+// rounded once: the correctly rounded quotient whenever the residual is
+// exact (Markstein's theorem), which holds for |x| >= 2^-103 (the residual,
+// about 2^-23 |x|, stays normal).  Smaller x with s >= kFmaMinScale = 2^-64
+// give |x / s| < 2^-39, and then t = q + z rounds to z or to within 2^-39 of
+// 0 whatever the quotient's last bits, so the code is the divide's.
+// code_check_kernel compares the two forms on random groups.
 // Within a group t = fl32(q + z) lies in [-1/2, 256]: z - fl32(-min / s) is
 // in [-1/2, 1/2] exactly and q is monotone in x.  So no lower clamp is
 // needed: t is clamped to 255 from above, and adding 1.5 * 2^23 rounds it to
@@ -174,7 +174,8 @@ __device__ __noinline__ void codes_div_rows(const uint4* src, int64_t C8, uint2*
             c[2 * q] = code_div(bf16_lo(w[q]), s_sm[2 * q], z_sm[2 * q]);
             c[2 * q + 1] = code_div(bf16_hi(w[q]), s_sm[2 * q + 1], z_sm[2 * q + 1]);
         }
-        dst[i * C8] = make_uint2(c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24, c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24);
+        dst[i * C8] = make_uint2(c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24,
+                                 c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24);
     }
 }
 

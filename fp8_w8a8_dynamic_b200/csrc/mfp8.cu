@@ -227,7 +227,8 @@ mfp8_status set_smem(Kern kern, int bytes, int dev, bool* done) {
 
 template <int BN, int STAGES>
 mfp8_status launch_tiled_bn(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
-                            const float* s_w, int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                            const float* s_w, int64_t N, int64_t w_rows, void* Y, bool dependent, int dev,
+                            const DeviceInfo& info,
                             cudaStream_t stream) {
     using L = tiled::Layout<BN, STAGES>;
     auto kern = tiled::gemm_tiled_kernel<BN, STAGES>;
@@ -271,7 +272,8 @@ int tiled_tile_width(int64_t M, int64_t N, const DeviceInfo& info) {
 }
 
 mfp8_status launch_tiled(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8,
-                         const float* s_w, int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                         const float* s_w, int64_t N, int64_t w_rows, void* Y, bool dependent, int dev,
+                         const DeviceInfo& info,
                          cudaStream_t stream) {
     switch (tiled_tile_width(M, N, info)) {
         case 256: return launch_tiled_bn<256, 4>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
@@ -367,7 +369,8 @@ int pair_tile_width(int64_t M, int64_t N, const DeviceInfo& info) {
 }
 
 mfp8_status launch_pair(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                        int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info, cudaStream_t stream) {
+                        int64_t N, int64_t w_rows, void* Y, bool dependent, int dev, const DeviceInfo& info,
+                        cudaStream_t stream) {
     if (pair_tile_width(M, N, info) == 128)
         return launch_pair_bn<128, 8>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
     return launch_pair_bn<256, 6>(X8, s_a, M, K, W8, s_w, N, w_rows, Y, dependent, dev, info, stream);
@@ -594,7 +597,8 @@ bool cluster_geometry(int64_t M, int64_t N, int64_t K, int sm_count, cluster::Ge
 }
 
 mfp8_status launch_cluster(const void* X8, const float* s_a, int64_t M, int64_t K, const void* W8, const float* s_w,
-                           int64_t N, int64_t w_rows, void* Y, bool weights_static, bool dependent, int dev, const DeviceInfo& info,
+                           int64_t N, int64_t w_rows, void* Y, bool weights_static, bool dependent, int dev,
+                           const DeviceInfo& info,
                            cudaStream_t stream) {
     cluster::Geometry g;
     if (!cluster_geometry(M, N, K, info.sm_count, &g)) return MFP8_ERR_UNSUPPORTED_SHAPE;
