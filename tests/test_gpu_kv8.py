@@ -147,3 +147,25 @@ def test_kv8_divide_free_codes_match_the_divide():
     torch.cuda.synchronize()
     bad, witness = out.tolist()
     assert bad == 0, f"{bad} codes differ; scale bits {witness >> 32:08x}, x bits {witness & 0xffff:04x}"
+
+
+def test_kv8_nonfinite_inputs_are_contained():
+    """Non-finite values are outside the contract: the kernels must neither
+    fault nor hang on them, and groups without them must still match the
+    oracle bit for bit."""
+    T, H, D = 128, 2, 64
+    kv = W.make_kv(T, H, D, seed=11, device=DEV)
+    kv[3, 0, 5] = float("inf")
+    kv[70, 1, 9] = float("nan")
+    kv[100, 0, 60] = float("-inf")
+    codes, scale, zero = mfp8.kv8_quantize(kv)
+    out = mfp8.kv8_read(codes, scale, zero, kv[:0])
+    torch.cuda.synchronize()
+    assert mfp8.device_status() == mfp8.OK
+    q_ref, s_ref, z_ref = oracle.kv8_quantize(bits16(kv))
+    bad = np.zeros((T // 64, H, D), bool)
+    bad[0, 0, 5] = bad[1, 1, 9] = bad[1, 0, 60] = True
+    ok = ~np.repeat(bad, 64, axis=0)
+    assert np.array_equal(u8(codes)[ok], q_ref[ok])
+    assert np.array_equal(f32(scale)[~bad].view(np.uint32), s_ref[~bad].view(np.uint32))
+    assert np.array_equal(bits16(out)[ok], oracle.kv8_read(q_ref, s_ref, z_ref, bits16(kv[:0]))[ok])
