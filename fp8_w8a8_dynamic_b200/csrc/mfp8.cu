@@ -828,6 +828,8 @@ mfp8_status run_padded(const void* X_bf16, const void* X8, const float* s_a, int
         st = launch_stream(X_bf16, M, K, W8, sw8, pad.n8, N, y8, /*weights_static=*/false, /*dependent=*/false,
                            X_fp8_out, x_scale_out, dev, info, stream);
     } else {
+        // the per-row quantizer without the early trigger: the same codes as
+        // mfp8_quantize_act, launched in plain stream order
         if (X_bf16 && (st = quantize_weight_rows(X_bf16, M, K, const_cast<void*>(X8), const_cast<float*>(s_a),
                                                  stream)) != MFP8_OK)
             return st;
