@@ -1083,7 +1083,7 @@ mfp8_status mfp8_kv_quantize(const void* KV_bf16, int64_t T, int64_t H, int64_t 
     if (D > 256) return quantize_weight_rows(KV_bf16, R, D, KV_fp8, kv_scale, s);  // long rows: the row kernels
     const int vpr = int(D / 8);
     const int lpr = vpr <= 2 ? 2 : vpr <= 4 ? 4 : vpr <= 8 ? 8 : vpr <= 16 ? 16 : 32;
-    const int64_t rows_per_block = int64_t(kQuantThreads / 32) * (32 / lpr);
+    const int64_t rows_per_block = int64_t(kQuantThreads / 32) * (32 / lpr) * kSmallRowItems;
     const int64_t blocks = (R + rows_per_block - 1) / rows_per_block;
     if (blocks > INT32_MAX) return MFP8_ERR_UNSUPPORTED_SHAPE;
     const uint4* x = static_cast<const uint4*>(KV_bf16);

@@ -289,8 +289,11 @@ quant_rows_loop_kernel(const uint4* __restrict__ X, int64_t K, uint2* __restrict
 
 // Rows of D <= 256 values (D % 16 == 0): LPR lanes per row (a power of two
 // >= D / 8), each holding one 16-byte vector of 8 values, 32 / LPR rows per
-// warp, so a warp's loads and stores are contiguous.  The absmax is a
-// shuffle reduction over the row's lanes.
+// warp and kSmallRowItems such row groups per warp, all loads issued first;
+// a warp's loads and stores are contiguous.  The absmax is a shuffle
+// reduction over the row's lanes.
+constexpr int kSmallRowItems = 4;
+
 template <int LPR>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_small_rows_kernel(const uint4* __restrict__ X, int64_t R, int D, uint2* __restrict__ Q,
@@ -299,21 +302,29 @@ quant_small_rows_kernel(const uint4* __restrict__ X, int64_t R, int D, uint2* __
     grid_dependency_wait();  // X may be the previous kernel's output
     constexpr int kRowsPerWarp = 32 / LPR;
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp +
-                        lane / LPR;
+    const int64_t row0 = (int64_t(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp *
+                             kSmallRowItems + lane / LPR;
     const int v = lane % LPR;
     const int vpr = D >> 3;  // vectors per row
-    const bool live = row < R && v < vpr;
-    const uint4 x = live ? __ldg(X + row * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
-    uint32_t acc = absmax_bits_u4(x, 0u);
-    uint32_t amax = max(acc & 0xffffu, acc >> 16);
+    uint4 x[kSmallRowItems];
 #pragma unroll
-    for (int off = 1; off < LPR; off <<= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (!live) return;
-    const float s = scale_from_absmax_bits(amax);
-    const float r = __frcp_rn(s);
-    if (v == 0) S[row] = s;
-    Q[row * vpr + v] = quantize8(x, s, r);
+    for (int k = 0; k < kSmallRowItems; ++k) {
+        const int64_t row = row0 + k * kRowsPerWarp;
+        x[k] = row < R && v < vpr ? __ldg(X + row * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < kSmallRowItems; ++k) {
+        const int64_t row = row0 + k * kRowsPerWarp;
+        const uint32_t acc = absmax_bits_u4(x[k], 0u);
+        uint32_t amax = max(acc & 0xffffu, acc >> 16);
+#pragma unroll
+        for (int off = 1; off < LPR; off <<= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (row < R && v < vpr) {
+            const float s = scale_from_absmax_bits(amax);
+            if (v == 0) S[row] = s;
+            Q[row * vpr + v] = quantize8(x[k], s, __frcp_rn(s));
+        }
+    }
 }
 
 // Dequantize: each thread turns 16 codes (16 bytes) into 16 bf16 (32 bytes).
