@@ -56,6 +56,7 @@ constexpr int kMaxCluster = 8;
 constexpr int kMaxStages = 8;
 constexpr int kWBlockBytes = TILE * SUB;    // one weight K block of the tile: 16 KB
 constexpr int kRingBytes = 96 * 1024;       // weight + code ring; later the partial-row receive area
+constexpr int kRingBig = 192 * 1024;        // the ring when the grid has at most one CTA per SM
 constexpr int kMinStages = 2;
 static_assert(SUB / MMA_K == 4, "a K block is four MMAs");
 
@@ -65,6 +66,7 @@ struct Geometry {
     int mp;      // token columns of the MMA: M rounded up to 16
     int stages;  // ring depth; a stage is a weight block and a code block
     int tc;      // token columns per exchange round (S > 1): a multiple of 16, <= mp
+    int ring;    // ring bytes: kRingBytes (two CTAs fit on an SM) or kRingBig (grids of at most one CTA per SM)
 };
 
 __host__ __device__ constexpr int stage_bytes(int mp) { return kWBlockBytes + mp * SUB; }
@@ -81,20 +83,24 @@ __host__ __device__ constexpr int exchange_bytes(int S, int tc) {
 }
 
 // Shared memory, from a 1024-byte aligned base:
-//   [ring] kRingBytes: stage s at s * stage_bytes(mp) (weights, then codes);
-//          with S > 1 it later holds the exchange slots (exchange_bytes)
-//   [sa] [256] f32, [sw] [128] f32, barriers, TMEM base and abort flag
+//   [ring] g.ring bytes: stage s at s * stage_bytes(mp) (weights, then
+//          codes); with S > 1 it later holds the exchange slots
+//          (exchange_bytes)
+//   then, at offset g.ring: [sa] [256] f32, [sw] [128] f32, barriers, TMEM
+//          base and abort flag
 struct Smem {
-    static constexpr int SA_OFF = kRingBytes;
+    static constexpr int SA_OFF = 0;  // from the end of the ring
     static constexpr int SW_OFF = SA_OFF + kMaxM * 4;
     static constexpr int BAR_OFF = SW_OFF + TILE * 4;
     // full[8], empty[8], tfull, rbar, drain, (pad)
     static constexpr int NUM_BARS = 2 * kMaxStages + 4;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int USED = MISC_OFF + 16;
-    static constexpr int BYTES = USED + 1024;  // alignment slack
+    static constexpr int bytes(int ring) { return ring + USED + 1024; }  // + alignment slack
+    static constexpr int MAX_BYTES = kRingBig + USED + 1024;
     static_assert(exchange_bytes(2, 16) <= kRingBytes, "one round of the narrowest exchange fits in the ring");
     static_assert(kMinStages * stage_bytes(kMaxM) <= kRingBytes, "ring room");
+    static_assert(MAX_BYTES <= 227 * 1024, "shared memory of one CTA");
 };
 
 struct Args {
@@ -115,16 +121,17 @@ gemm_cluster_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     const int M = args.M, N = args.N, K = args.K;
     const int S = args.g.S, MP = args.g.mp, STAGES = args.g.stages;
     const int SB = stage_bytes(MP);
-    const uint32_t bar0 = sbase + Smem::BAR_OFF;
+    uint8_t* fixed = smem + args.g.ring;  // scales, barriers and flags follow the ring
+    const uint32_t bar0 = smem_u32(fixed) + Smem::BAR_OFF;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kMaxStages + s); };
     const uint32_t tfull_bar = bar0 + 8u * (2 * kMaxStages);  // accumulator complete
     const uint32_t rbar = tfull_bar + 8u;                     // all partials of my channels received
     const uint32_t drain_bar = tfull_bar + 16u;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Smem::MISC_OFF);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::MISC_OFF + 4);
-    float* sa_sm = reinterpret_cast<float*>(smem + Smem::SA_OFF);
-    float* sw_sm = reinterpret_cast<float*>(smem + Smem::SW_OFF);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fixed + Smem::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(fixed + Smem::MISC_OFF + 4);
+    float* sa_sm = reinterpret_cast<float*>(fixed + Smem::SA_OFF);
+    float* sw_sm = reinterpret_cast<float*>(fixed + Smem::SW_OFF);
 
     const uint32_t warp = warp_id_sync();
     const uint32_t lane = lane_id();

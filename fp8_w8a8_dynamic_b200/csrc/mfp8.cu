@@ -578,7 +578,11 @@ bool cluster_geometry(int64_t M, int64_t N, int64_t K, int sm_count, cluster::Ge
     while (grow(S)) S *= 2;
     g->S = S;
     g->mp = int((M + 15) / 16 * 16);
-    const int st = cluster::kRingBytes / cluster::stage_bytes(g->mp);
+    // A grid of at most one CTA per SM takes the deeper ring (more bytes in
+    // flight per CTA, fewer exchange rounds); larger grids keep two CTAs per
+    // SM resident.
+    g->ring = tiles * S <= sm_count ? cluster::kRingBig : cluster::kRingBytes;
+    const int st = g->ring / cluster::stage_bytes(g->mp);
     g->stages = st > cluster::kMaxStages ? cluster::kMaxStages : st;
     // Exchange rounds: as few as the ring allows, of equal width (a multiple
     // of 32 token columns where the round is that wide, else of 16: whole
@@ -590,7 +594,7 @@ bool cluster_geometry(int64_t M, int64_t N, int64_t K, int sm_count, cluster::Ge
             const int w = (g->mp + r - 1) / r;
             return w > 16 ? (w + 31) / 32 * 32 : 16;
         };
-        while (cluster::exchange_bytes(S, width(rounds)) > cluster::kRingBytes) ++rounds;
+        while (cluster::exchange_bytes(S, width(rounds)) > g->ring) ++rounds;
         g->tc = width(rounds) < g->mp ? width(rounds) : g->mp;
     }
     return g->stages >= cluster::kMinStages;
@@ -604,7 +608,7 @@ mfp8_status launch_cluster(const void* X8, const float* s_a, int64_t M, int64_t 
     if (!cluster_geometry(M, N, K, info.sm_count, &g)) return MFP8_ERR_UNSUPPORTED_SHAPE;
     auto kern = cluster::gemm_cluster_kernel;
     static bool attr_done[kMaxDevices] = {};
-    mfp8_status st = set_smem(kern, cluster::Smem::BYTES, dev, attr_done);
+    mfp8_status st = set_smem(kern, cluster::Smem::MAX_BYTES, dev, attr_done);
     if (st != MFP8_OK) return st;
     const int64_t tiles = (N + cluster::TILE - 1) / cluster::TILE;
     const int64_t grid = tiles * g.S;
@@ -626,7 +630,7 @@ mfp8_status launch_cluster(const void* X8, const float* s_a, int64_t M, int64_t 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(grid));
     cfg.blockDim = dim3(cluster::kThreads);
-    cfg.dynamicSmemBytes = cluster::Smem::BYTES;
+    cfg.dynamicSmemBytes = size_t(cluster::Smem::bytes(g.ring));
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
